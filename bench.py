@@ -1,0 +1,349 @@
+"""Benchmark: anisotropic-AH search throughput (queries/s at top-10) on B200.
+
+One step = one batched search of the whole hot path (centroid scores -> top-L
+leaves -> lookup tables -> 4-bit code scan -> top-R -> exact reorder -> top-k)
+over one batch of synthetic queries, through the C ABI.  Default workload: the
+GloVe-shaped IVF-AH configuration (n = 1,000,000, d = 100, 1,000 leaves,
+32 searched, 1,000 queries, k = 10, reorder 100).
+
+Single GPU:  python bench.py [--steps K --warmup W]
+N GPUs:      python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
+             (one process per GPU; every rank holds a replica of the index and
+             searches its own query batch; no data-path collective -> weak
+             scaling; timing is the max over ranks)
+Reference:   python bench.py --impl reference  (the CPU oracle, rank 0 only)
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "AH search queries/sec at top-10 (1 B200); code-scan GB/s vs HBM/smem roofline"
+L2_BYTES = 126 * 1024 * 1024
+SM_COUNT = 148
+SMEM_BYTES_PER_CLK = 128          # per SM: 32 banks x 4 B
+SM_MAX_MHZ_FALLBACK = 1965.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="glove")
+    p.add_argument("--lut-mode", type=int, default=0, choices=[0, 1])
+    p.add_argument("--nq", type=int, default=None)
+    p.add_argument("--leaves", type=int, default=None)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--e2e-steps", type=int, default=100)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_spec(args):
+    from mips_ivf_centroid_b200 import datagen
+    w = datagen.WORKLOADS[args.workload]
+    if args.nq:
+        w = w.scaled(nq=args.nq)
+    if args.leaves:
+        w = w.scaled(num_leaves_to_search=args.leaves)
+    return w
+
+
+def config_dict(w, args):
+    return {"workload": f"{w.name}-shaped IVF-AH: n={w.n:,} d={w.d} dims_per_block={w.dims_per_block} "
+                        f"num_leaves={w.num_leaves} num_leaves_to_search={w.num_leaves_to_search} nq={w.nq} "
+                        f"k={w.k} reorder_num={w.reorder_num} ({w.reorder_dtype} reorder copy)",
+            "n": w.n, "d": w.d, "dims_per_block": w.dims_per_block, "num_leaves": w.num_leaves,
+            "num_leaves_to_search": w.num_leaves_to_search, "nq": w.nq, "k": w.k, "reorder_num": w.reorder_num,
+            "lut_mode": "u8" if args.lut_mode else "f32", "l2_flush_between_steps": True}
+
+
+def oracle_rate(orc, Q, w, lut_mode, seconds):
+    """Queries/s of the oracle on this host, on consecutive query chunks until
+    ``seconds`` have elapsed (a bounded sample of the workload)."""
+    import oracle
+    nthreads = os.cpu_count() or 1
+    done, t0, i = 0, time.perf_counter(), 0
+    chunk = max(8, nthreads * 2)
+    while True:
+        qs = Q[(i % Q.shape[0]):(i % Q.shape[0]) + chunk]
+        orc.search(qs, w.k, w.num_leaves_to_search, w.reorder_num, lut_mode, nthreads=nthreads, trace=False)
+        done += qs.shape[0]
+        i += chunk
+        el = time.perf_counter() - t0
+        if el >= seconds or done >= 50 * Q.shape[0]:
+            break
+    return done / el, done, el, oracle.max_threads()
+
+
+def run_reference(args):
+    import torch
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from mips_ivf_centroid_b200 import datagen
+    w = workload_spec(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    X = datagen.make_data(w)
+    Q = datagen.make_queries(w)
+    arr = datagen.build_index(w, X, dev).numpy()
+    del X
+    orc = oracle.OracleIndex(arr)
+    nthreads = os.cpu_count() or 1
+    # calibrate the per-step sample so W + K steps take about 90 s
+    t0 = time.perf_counter()
+    orc.search(Q[:nthreads], w.k, w.num_leaves_to_search, w.reorder_num, args.lut_mode, nthreads=nthreads, trace=False)
+    per_q = (time.perf_counter() - t0) / nthreads
+    S = int(max(1, min(w.nq, 90.0 / max(1, args.steps + args.warmup) / max(per_q, 1e-6))))
+    times = []
+    for s in range(args.warmup + args.steps):
+        qs = Q[(s * S) % w.nq:][:S]
+        t0 = time.perf_counter()
+        orc.search(qs, w.k, w.num_leaves_to_search, w.reorder_num, args.lut_mode, nthreads=nthreads, trace=False)
+        if s >= args.warmup:
+            times.append((time.perf_counter() - t0, qs.shape[0]))
+    tot = sum(t for t, _ in times)
+    nqs = sum(n for _, n in times)
+    value = nqs / tot
+    line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64" if args.lut_mode == 0 else "u8",
+            "data": "synthetic (seeded Gaussian mixture, GloVe-shaped)", "config": config_dict(w, args),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": f"{S} of {w.nq} queries per step, {len(times)} steps"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from mips_ivf_centroid_b200 import Index, build as ahbuild, datagen
+    ahbuild.build()
+    w = workload_spec(args)
+    wq = w.scaled(query_seed=w.query_seed + 1000 * rank)          # each rank: its own batch
+    X = datagen.make_data(w)
+    Q = datagen.make_queries(wq)
+    ix = datagen.build_index(w, X, dev)
+    del X
+    torch.cuda.empty_cache()            # release the index build's temporaries
+    index = Index(ix)
+    qg = torch.from_numpy(Q).to(dev)
+    L, k, R, mode = w.num_leaves_to_search, w.k, w.reorder_num, args.lut_mode
+    index.reserve(w.nq, k, L, R, mode)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    # warm-up
+    for _ in range(args.warmup):
+        index.search(qg, k, L, R, mode)
+    index.sync_status()
+    _, _, tr = index.search(qg, k, L, R, mode, trace=True)
+    scanned = int(tr["scanned"].sum().item())
+    leaves = tr["leaf_ids"].cpu().numpy()
+    offs = ix.leaf_offsets.cpu().numpy()
+    touched = np.unique(leaves)
+    unique_code_bytes = int((offs[touched + 1] - offs[touched]).sum()) * w.code_bytes
+    index.sync_status()
+
+    # timed region: K steps, L2 flushed before each (outside the step's events)
+    index.set_profiling(True)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = {}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_wall = time.perf_counter()
+        for s in range(args.steps):
+            flush.zero_()
+            ev0[s].record(stream)
+            index.search(qg, k, L, R, mode)
+            ev1[s].record(stream)
+            if s % 50 == 49 or s == args.steps - 1:
+                for kname, v in index.stage_times().items():
+                    stage_ms.setdefault(kname, []).append(v)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    index.set_profiling(False)
+    index.sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    dev_ms = sum(step_ms)
+    launches = index.last_search_info()["launches"]
+    if world > 1:
+        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dev_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = dev_ms / args.steps
+    value = world * w.nq / (ms_per_step * 1e-3)
+
+    # e2e through the host entry point: pinned host queries in, host results out
+    hq = torch.from_numpy(Q).pin_memory()
+    hids = torch.empty((w.nq, k), dtype=torch.int32).pin_memory()
+    hsc = torch.empty((w.nq, k), dtype=torch.float32).pin_memory()
+    for _ in range(3):
+        index.search_host(hq, k, L, R, mode, out_ids=hids, out_scores=hsc)
+    e2e_times = []
+    if world > 1:
+        dist.barrier()
+    for _ in range(args.e2e_steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        index.search_host(hq, k, L, R, mode, out_ids=hids, out_scores=hsc)
+        e2e_times.append(time.perf_counter() - t0)
+    e2e_s = sum(e2e_times)
+    if world > 1:
+        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_value = world * w.nq * args.e2e_steps / e2e_s
+
+    if rank == 0:
+        med = {kname: statistics.median(v) for kname, v in stage_ms.items()}
+        scan_ms = med.get("scan", float("nan"))
+        clocks = clk.summary()
+        lookups = scanned * w.blocks
+        bytes_per_lookup = 4 if mode == 0 else 1
+        lut_bytes = lookups * bytes_per_lookup
+        mhz = SM_MAX_MHZ_FALLBACK
+        peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        hbm_peak = None
+        if os.path.exists(peaks_path):
+            pk = json.load(open(peaks_path))
+            mhz = float(pk.get("sm_max_mhz", mhz))
+            hbm_peak = pk.get("hbm_gbs")
+        smem_peak_gbs = SM_COUNT * SMEM_BYTES_PER_CLK * mhz * 1e6 / 1e9
+        achieved = lut_bytes / (scan_ms * 1e-3) / 1e9
+        roofline = {"bound": "smem", "achieved": achieved, "peak": smem_peak_gbs, "unit": "GB/s",
+                    "frac": achieved / smem_peak_gbs, "traffic": None,
+                    "kernel": "scan_kernel", "unit_bytes": f"{bytes_per_lookup} B per table lookup",
+                    "lookups_per_launch": lookups,
+                    "peak_source": f"derived: {SM_COUNT} SMs x {SMEM_BYTES_PER_CLK} B/clk x {mhz:.0f} MHz"}
+        line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32" if mode == 0 else "u8",
+                "data": "synthetic (seeded Gaussian mixture, GloVe-shaped; index trained on it)",
+                "config": config_dict(w, args),
+                "roofline": roofline,
+                "scan": {"ms": scan_ms, "hbm_unique_code_gbs": unique_code_bytes / (scan_ms * 1e-3) / 1e9,
+                         "unique_code_bytes": unique_code_bytes, "hbm_peak_gbs": hbm_peak,
+                         "lookups_per_s": lookups / (scan_ms * 1e-3)},
+                "stages_ms": med,
+                "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": int(Q.nbytes),
+                        "d2h_bytes_per_step": int(w.nq * k * 8)},
+                "gpu_launches": launches * args.steps,
+                "clocks": clocks, "wall_s_timed": t_wall}
+        if not args.no_cpu_baseline and world == 1:
+            import oracle
+            orc = oracle.OracleIndex(ix.numpy())
+            rate, done, el, cores = oracle_rate(orc, Q, w, mode, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{done} queries of the batch in {el:.1f} s"}
+        print(json.dumps(line), flush=True)
+    index.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

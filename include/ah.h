@@ -1,0 +1,233 @@
+/*
+ * ah.h: C ABI of the B200 anisotropic-AH maximum inner product search library.
+ *
+ * The search path is the one the ScaNN blog post describes in "Three stages of
+ * a search" (ScaNN: Anisotropic Vector Quantization for Maximum Inner Product
+ * Search):
+ *   partitioning  -> the query scores every centroid and keeps the best
+ *                    num_leaves_to_search leaves;
+ *   asymmetric hashing (AH) -> a per-query lookup table of q . center for each
+ *                    block's 16 centers; a point's approximate score is the sum
+ *                    of its table entries, read through its 4-bit codes;
+ *   reordering    -> the best few hundred candidates are rescored with exact
+ *                    dot products, and the best k are returned.
+ * The search-time knobs follow the post's "Using the library" section
+ * (search_batched with leaves_to_search and pre_reorder_num_neighbors, and
+ * final_num_neighbors).  Training an index is not part of this library.
+ *
+ * Conventions for every entry point:
+ *  - Status codes only: no exceptions cross the ABI, nothing calls exit/abort.
+ *  - Device pointers are CUDA device memory on the current device; the library
+ *    never frees memory it did not allocate.
+ *  - Work is enqueued on the given stream (a cudaStream_t passed as void*; NULL
+ *    means the legacy default stream) and is asynchronous unless stated
+ *    otherwise: outputs are valid once that stream has been synchronised.
+ *  - Errors a kernel detects are recorded in a per-index device error word;
+ *    ah_sync_status() reports (and clears) them.
+ *  - Ordering everywhere is (score descending, then lower id).  Results shorter
+ *    than k are padded with id -1 and score -INFINITY.
+ *  - Ids are the original datapoint ids (int32).
+ *  - An index may be searched from one stream at a time (it owns one
+ *    workspace); different indexes are independent.
+ */
+#ifndef AH_H_
+#define AH_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AH_API __attribute__((visibility("default")))
+#else
+#define AH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AH_OK = 0,
+    AH_ERR_INVALID_ARG = 1,  /* a null pointer, an out-of-range size or knob   */
+    AH_ERR_UNSUPPORTED = 2,  /* valid request beyond this build's limits       */
+    AH_ERR_OOM = 3,          /* device allocation failed                       */
+    AH_ERR_CUDA = 4,         /* a CUDA runtime call failed                     */
+    AH_ERR_DEVICE = 5,       /* a kernel reported an error (see ah_sync_status) */
+    AH_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up        */
+} ah_status;
+
+/* reorder_dtype values */
+enum { AH_F32 = 0, AH_BF16 = 1 };
+/* lut_mode values */
+enum { AH_LUT_F32 = 0, AH_LUT_U8 = 1 };
+
+/* Library limits (AH_ERR_UNSUPPORTED beyond them). */
+#define AH_MAX_K 1024            /* final neighbours per query                 */
+#define AH_MAX_R 4096            /* max(reorder_num, k)                        */
+#define AH_MAX_LEAVES_SEARCHED 4096
+#define AH_MAX_D 8192
+#define AH_MAX_BLOCKS 1024       /* d / dims_per_block                         */
+
+/*
+ * Index arrays, all in device memory and BORROWED: they must stay allocated
+ * and unchanged until ah_destroy().  Source: ScaNN blog, "Three stages of a
+ * search" (leaves, 16 centers per block, 4-bit codes) and "Worked example"
+ * (64 blocks of 4 bits = 32 B per point at d = 128, dims_per_block = 2).
+ *   n               points; 0 < n < 2^31 - 64
+ *   d               dimension; divisible by 2 * dims_per_block
+ *   num_leaves      NL >= 1 partitions
+ *   dims_per_block  dimensions per AH block; B = d / dims_per_block blocks
+ *   centroids       float [NL][d]
+ *   leaf_offsets    int64 [NL+1]: leaf c holds slots leaf_offsets[c] ..
+ *                   leaf_offsets[c+1]-1; non-decreasing, 0 .. n
+ *   slot_ids        int32 [n]: original id of the point in each slot
+ *   codes           uint8 [n][B/2], slot order; block 2i in the low nibble and
+ *                   block 2i+1 in the high nibble of byte i
+ *   codebook        float [B][16][dims_per_block]
+ *   reorder_vecs    [n][d] slot order, float (AH_F32) or bfloat16 (AH_BF16);
+ *                   may be NULL if the index is only searched with
+ *                   reorder_num = 0
+ */
+typedef struct {
+    int64_t n;
+    int32_t d;
+    int32_t num_leaves;
+    int32_t dims_per_block;
+    const float *centroids;
+    const int64_t *leaf_offsets;
+    const int32_t *slot_ids;
+    const uint8_t *codes;
+    const float *codebook;
+    const void *reorder_vecs;
+    int32_t reorder_dtype;
+} ah_index_views;
+
+typedef struct ah_index ah_index;
+
+/*
+ * Validate the views and build the derived device state on cuda_stream:
+ * int32 leaf offsets and a re-laid-out copy of the codes (32-point tiles of
+ * 32-bit words, so a warp reads each code word of 32 consecutive slots with
+ * one coalesced 128-byte access).  The copy is owned by the index.  This call
+ * synchronises cuda_stream before returning.
+ * Errors: AH_ERR_INVALID_ARG (null pointer, bad sizes), AH_ERR_UNSUPPORTED
+ * (sizes beyond the limits), AH_ERR_OOM, AH_ERR_CUDA.  *out is NULL on error.
+ */
+AH_API ah_status ah_build_index_views(const ah_index_views *views, void *cuda_stream, ah_index **out);
+
+/*
+ * Search a batch (ScaNN blog, "Three stages of a search"; knobs as in
+ * "Using the library": num_leaves_to_search = leaves_to_search, reorder_num =
+ * pre_reorder_num_neighbors, k = final_num_neighbors).
+ *   queries      float [nq][d], device
+ *   nq           >= 0 (0 returns AH_OK with nothing enqueued)
+ *   k            1 .. AH_MAX_K
+ *   num_leaves_to_search  1 .. min(num_leaves, AH_MAX_LEAVES_SEARCHED)
+ *   reorder_num  0 (no exact rescoring: scores are approximate) or >= k;
+ *                the R = max(reorder_num, k) best candidates by approximate
+ *                score are kept, then rescored exactly ("reorder not above k"
+ *                in the post's failure modes); R <= AH_MAX_R
+ *   lut_mode     AH_LUT_F32: fp32 table and fp32 sums;
+ *                AH_LUT_U8: uint8 table, integer sums; the table is
+ *                lut = q0*c0 then fmaf(q_t, c_t, lut), m_b = min_j lut,
+ *                delta = max_b(max_j lut - m_b)/255 (1 if 0),
+ *                u = min(255, rint((lut - m_b)/delta)), bias = sum_b m_b in
+ *                fp32 in block order; approximate score = fmaf(delta, sum, bias).
+ *   out_ids      int32 [nq][k], device
+ *   out_scores   float [nq][k], device: exact fp32 dot products when
+ *                reorder_num > 0, otherwise approximate scores
+ * Errors: AH_ERR_INVALID_ARG, AH_ERR_UNSUPPORTED, AH_ERR_OOM (workspace
+ * growth), AH_ERR_CUDA (launch failure).  Device-side errors of this call are
+ * reported by a later ah_sync_status().
+ */
+AH_API ah_status ah_search(ah_index *ix, const float *queries, int32_t nq, int32_t k,
+                    int32_t num_leaves_to_search, int32_t reorder_num, int32_t lut_mode,
+                    int32_t *out_ids, float *out_scores, void *cuda_stream);
+
+/*
+ * Intermediate results of one search, for inspection and testing.  Every
+ * pointer is device memory and optional (NULL to skip).
+ *   leaf_ids, leaf_scores  [nq][L]  kept leaves and their fp32 centroid scores
+ *   cand_ids, cand_scores  [nq][R]  best R by approximate score (padded -1/-inf)
+ *   cand_sums              [nq][R]  uint8 mode: integer sums (0 otherwise)
+ *   ncand                  [nq]     candidates kept (<= R)
+ *   scanned                [nq]     points whose codes the query scanned
+ *   passed                 [nq]     points whose approximate score reached the
+ *                                   query's filter bound in the first scan pass
+ *   rescans                [1]      queries rescanned after a buffer overflow
+ */
+typedef struct {
+    int32_t *leaf_ids;
+    float *leaf_scores;
+    int32_t *cand_ids;
+    float *cand_scores;
+    uint32_t *cand_sums;
+    int32_t *ncand;
+    int64_t *scanned;
+    int32_t *passed;
+    int32_t *rescans;
+} ah_search_trace;
+
+/* ah_search plus the intermediate results named in *trace (may be NULL). */
+AH_API ah_status ah_search_traced(ah_index *ix, const float *queries, int32_t nq, int32_t k,
+                           int32_t num_leaves_to_search, int32_t reorder_num, int32_t lut_mode,
+                           int32_t *out_ids, float *out_scores, const ah_search_trace *trace,
+                           void *cuda_stream);
+
+/*
+ * ah_search on HOST buffers: host_queries [nq][d], host_ids [nq][k] and
+ * host_scores [nq][k] are host memory (pinned memory gives asynchronous
+ * copies).  The queries are copied to the device, searched, and the results
+ * copied back, all on cuda_stream; the call synchronises cuda_stream and
+ * returns with the results in place, including any device-side error.
+ */
+AH_API ah_status ah_search_host(ah_index *ix, const float *host_queries, int32_t nq, int32_t k,
+                         int32_t num_leaves_to_search, int32_t reorder_num, int32_t lut_mode,
+                         int32_t *host_ids, float *host_scores, void *cuda_stream);
+
+/*
+ * Reserve workspace for searches up to max_nq queries with the given knobs,
+ * so later searches allocate nothing.  Synchronous.
+ */
+AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num_leaves_to_search,
+                     int32_t reorder_num, int32_t lut_mode);
+
+/*
+ * Synchronise cuda_stream, then report and clear the index's device error
+ * word: AH_OK, or AH_ERR_DEVICE with ah_last_error() describing it.
+ */
+AH_API ah_status ah_sync_status(ah_index *ix, void *cuda_stream);
+
+/*
+ * Stage timing.  With profiling on, each search records CUDA events around its
+ * stages on the search stream; ah_stage_times() synchronises on the last
+ * event and writes up to max_stages durations in milliseconds (stage order as
+ * ah_stage_name(i)), setting *n_stages.  Synchronous.
+ */
+AH_API ah_status ah_set_profiling(ah_index *ix, int32_t on);
+AH_API ah_status ah_stage_times(ah_index *ix, float *ms, int32_t max_stages, int32_t *n_stages);
+AH_API const char *ah_stage_name(int32_t stage);
+
+/*
+ * Counters of the last search: kernels launched (*launches) and the points
+ * whose codes were scanned, summed over its queries (*points_scanned; asking
+ * for it synchronises the device).  Either pointer may be NULL.
+ */
+AH_API ah_status ah_last_search_info(ah_index *ix, int32_t *launches, int64_t *points_scanned);
+
+/* Device bytes owned by the index (derived state + workspace). */
+AH_API ah_status ah_index_memory(ah_index *ix, int64_t *bytes);
+
+/* Release everything the index owns.  Does not touch the borrowed views. */
+AH_API void ah_destroy(ah_index *ix);
+
+/* Static text for a status code. */
+AH_API const char *ah_status_string(ah_status s);
+
+/* Detail of the last error on the calling thread ("" if none). */
+AH_API const char *ah_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AH_H_ */

@@ -1,0 +1,493 @@
+// C ABI of the B200 anisotropic-AH MIPS search library (declared in include/ah.h).
+//
+// Host-side orchestration only: argument validation, the index's owned device
+// state, workspace management and the launch sequence of the search kernels
+// (kernels.cu) on the caller's stream.  No search arithmetic happens here.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "ah.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ah_status fail(ah_status s, const std::string& msg) {
+    g_last_error = msg;
+    return s;
+}
+
+ah_status cuda_fail(cudaError_t e, const char* what) {
+    g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return e == cudaErrorMemoryAllocation ? AH_ERR_OOM : AH_ERR_CUDA;
+}
+
+constexpr int kStages = 9;
+const char* kStageNames[kStages] = {"centroid_scores", "top_leaves", "invert", "lut",
+                                    "threshold", "scan", "select", "rescan", "reorder"};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Workspace {
+    void* base = nullptr;
+    size_t bytes = 0;
+    // capacity this carving was made for
+    int nq = 0, L = 0, R = 0, lut_mode = -1;
+    ah::SearchBuffers buf{};
+    // host-call staging
+    float* dq = nullptr;
+    int32_t* dids = nullptr;
+    float* dscores = nullptr;
+    int k = 0;
+};
+
+int cap_for(int R) { return std::max(8192, 16 * R); }
+
+}  // namespace
+
+struct ah_index {
+    ah_index_views views{};
+    ah::DeviceIndex dix{};
+    int device = 0;
+    int num_sms = 0;
+    int32_t* offs32 = nullptr;
+    uint32_t* codes_il = nullptr;
+    int* err = nullptr;
+    size_t owned_bytes = 0;
+    Workspace ws;
+    bool profiling = false;
+    cudaEvent_t ev[kStages + 1]{};
+    bool ev_ready = false;
+    bool ev_recorded = false;
+    int last_launches = 0;
+    int last_nq = 0;
+};
+
+namespace {
+
+ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool host_staging) {
+    Workspace& w = ix->ws;
+    const bool fits = w.base && nq <= w.nq && L <= w.L && R <= w.R && (lut_mode == w.lut_mode || w.lut_mode == 2) &&
+                      (!host_staging || (w.dq && k <= w.k));
+    if (fits) return AH_OK;
+    // grow: keep the larger of old and new needs
+    int cnq = std::max(nq, w.nq), cL = std::max(L, w.L), cR = std::max(R, w.R);
+    int mode = (w.lut_mode >= 0 && w.lut_mode != lut_mode) ? 2 : lut_mode;
+    int ck = std::max(k, w.k);
+    bool stage = host_staging || w.dq;
+    const int NL = ix->dix.nl, B = ix->dix.B, d = ix->dix.d;
+    const int cap = cap_for(cR);
+    size_t sz[32];
+    int n = 0;
+    auto add = [&](size_t bytes) { sz[n++] = align_up(bytes, 256); };
+    add(sizeof(float) * (size_t)cnq * NL);                      // 0 cscore
+    add(sizeof(int32_t) * (size_t)cnq * cL);                    // 1 leaves
+    add(sizeof(float) * (size_t)cnq * cL);                      // 2 leaf_scores
+    add(sizeof(int64_t) * (size_t)cnq);                         // 3 scanned
+    add((mode == 0 || mode == 2) ? sizeof(float) * (size_t)cnq * B * 16 : 0);   // 4 lut_f32
+    add((mode == 1 || mode == 2) ? (size_t)cnq * B * 16 : 0);                   // 5 lut_u8
+    add(sizeof(float) * (size_t)cnq);                           // 6 delta
+    add(sizeof(float) * (size_t)cnq);                           // 7 bias
+    add(sizeof(uint64_t) * (size_t)cnq);                        // 8 tau
+    add(sizeof(uint64_t) * (size_t)cnq * cap);                  // 9 candidate keys
+    add(sizeof(int32_t) * (size_t)(2 * NL + cnq + 8));          // 10 zero region: qcount, qcursor, count, counters
+    add(sizeof(int32_t) * (size_t)2 * cnq);                     // 11 redo
+    add(sizeof(int32_t) * (size_t)(NL + 1));                    // 12 qoff
+    add(sizeof(int32_t) * (size_t)(NL + 1));                    // 13 item_off
+    add(sizeof(int32_t) * (size_t)cnq * cL);                    // 14 qlist
+    add(stage ? sizeof(float) * (size_t)cnq * d : 0);           // 15 dq
+    add(stage ? sizeof(int32_t) * (size_t)cnq * ck : 0);        // 16 dids
+    add(stage ? sizeof(float) * (size_t)cnq * ck : 0);          // 17 dscores
+    add(sizeof(int32_t) * (size_t)cnq * cap);                   // 18 candidate slots
+    add(sizeof(uint64_t) * (size_t)cnq * cR);                   // 19 rkey
+    add(sizeof(int32_t) * (size_t)cnq * cR);                    // 20 rslot
+    add(sizeof(int32_t) * (size_t)cnq);                         // 21 rcount
+    add(sizeof(uint64_t) * (size_t)cnq * cR);                   // 22 ekey
+    size_t total = 0;
+    for (int i = 0; i < n; ++i) total += sz[i];
+    if (w.base) {
+        cudaError_t e = cudaDeviceSynchronize();   // the old workspace may still be in use
+        if (e != cudaSuccess) return cuda_fail(e, "workspace growth sync");
+        cudaFree(w.base);
+        ix->owned_bytes -= w.bytes;
+        w.base = nullptr;
+        w.bytes = 0;
+    }
+    void* base = nullptr;
+    cudaError_t e = cudaMalloc(&base, total);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace allocation");
+    w.base = base;
+    w.bytes = total;
+    ix->owned_bytes += total;
+    char* p = static_cast<char*>(base);
+    char* part[32];
+    for (int i = 0; i < n; ++i) {
+        part[i] = p;
+        p += sz[i];
+    }
+    ah::SearchBuffers& b = w.buf;
+    b.cscore = reinterpret_cast<float*>(part[0]);
+    b.leaves = reinterpret_cast<int32_t*>(part[1]);
+    b.leaf_scores = reinterpret_cast<float*>(part[2]);
+    b.scanned = reinterpret_cast<int64_t*>(part[3]);
+    b.lut_f32 = reinterpret_cast<float*>(part[4]);
+    b.lut_u8 = reinterpret_cast<uint8_t*>(part[5]);
+    b.lut_delta = reinterpret_cast<float*>(part[6]);
+    b.lut_bias = reinterpret_cast<float*>(part[7]);
+    b.tau = reinterpret_cast<uint64_t*>(part[8]);
+    b.ckey = reinterpret_cast<uint64_t*>(part[9]);
+    b.cslot = reinterpret_cast<int32_t*>(part[18]);
+    b.rkey = reinterpret_cast<uint64_t*>(part[19]);
+    b.rslot = reinterpret_cast<int32_t*>(part[20]);
+    b.rcount = reinterpret_cast<int32_t*>(part[21]);
+    b.ekey = reinterpret_cast<uint64_t*>(part[22]);
+    int32_t* zr = reinterpret_cast<int32_t*>(part[10]);
+    b.qcount = zr;
+    b.qcursor = zr + NL;
+    b.count = zr + 2 * NL;
+    b.counters = zr + 2 * NL + cnq;
+    b.redo = reinterpret_cast<int32_t*>(part[11]);
+    b.qoff = reinterpret_cast<int32_t*>(part[12]);
+    b.item_off = reinterpret_cast<int32_t*>(part[13]);
+    b.qlist = reinterpret_cast<int32_t*>(part[14]);
+    b.err = ix->err;
+    b.cap = cap;
+    w.dq = stage ? reinterpret_cast<float*>(part[15]) : nullptr;
+    w.dids = stage ? reinterpret_cast<int32_t*>(part[16]) : nullptr;
+    w.dscores = stage ? reinterpret_cast<float*>(part[17]) : nullptr;
+    w.nq = cnq;
+    w.L = cL;
+    w.R = cR;
+    w.lut_mode = mode;
+    w.k = stage ? ck : 0;
+    return AH_OK;
+}
+
+ah_status validate_search(ah_index* ix, const void* queries, int32_t nq, int32_t k, int32_t L, int32_t reorder_num,
+                          int32_t lut_mode, const void* out_ids, const void* out_scores) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    if (nq < 0) return fail(AH_ERR_INVALID_ARG, "nq < 0");
+    if (nq > 0 && (!queries || !out_ids || !out_scores)) return fail(AH_ERR_INVALID_ARG, "NULL queries or outputs");
+    if (k <= 0) return fail(AH_ERR_INVALID_ARG, "k must be >= 1");
+    if (k > AH_MAX_K) return fail(AH_ERR_UNSUPPORTED, "k above AH_MAX_K");
+    if (L < 1 || L > ix->dix.nl) return fail(AH_ERR_INVALID_ARG, "num_leaves_to_search outside [1, num_leaves]");
+    if (L > AH_MAX_LEAVES_SEARCHED) return fail(AH_ERR_UNSUPPORTED, "num_leaves_to_search above AH_MAX_LEAVES_SEARCHED");
+    if (reorder_num < 0 || (reorder_num > 0 && reorder_num < k))
+        return fail(AH_ERR_INVALID_ARG, "reorder_num must be 0 or >= k");
+    if (std::max(reorder_num, k) > AH_MAX_R) return fail(AH_ERR_UNSUPPORTED, "max(reorder_num, k) above AH_MAX_R");
+    if (reorder_num > 0 && !ix->views.reorder_vecs)
+        return fail(AH_ERR_INVALID_ARG, "reorder_num > 0 but the index has no reorder vectors");
+    if (lut_mode != AH_LUT_F32 && lut_mode != AH_LUT_U8) return fail(AH_ERR_INVALID_ARG, "unknown lut_mode");
+    const int64_t per_query_cand = static_cast<int64_t>(cap_for(std::max(reorder_num, k)));
+    if (static_cast<int64_t>(nq) * per_query_cand > (int64_t(1) << 40)) return fail(AH_ERR_UNSUPPORTED, "batch too large");
+    return AH_OK;
+}
+
+ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, int32_t L, int32_t reorder_num,
+                     int32_t lut_mode, int32_t* out_ids, float* out_scores, const ah_search_trace* tr,
+                     cudaStream_t s) {
+    const int R = std::max(reorder_num, k);
+    ah_status st = carve(ix, nq, L, R, lut_mode, 0, false);
+    if (st != AH_OK) return st;
+    ah::SearchBuffers b = ix->ws.buf;
+    ah::SearchArgs a{};
+    a.queries = queries;
+    a.nq = nq;
+    a.k = k;
+    a.L = L;
+    a.reorder_num = reorder_num;
+    a.R = R;
+    a.lut_mode = lut_mode;
+    a.chunk = nq >= 64 ? 1024 : 256;
+    a.out_ids = out_ids;
+    a.out_scores = out_scores;
+    if (tr) {
+        a.tr_leaf_ids = tr->leaf_ids;
+        a.tr_leaf_scores = tr->leaf_scores;
+        a.tr_cand_ids = tr->cand_ids;
+        a.tr_cand_scores = tr->cand_scores;
+        a.tr_cand_sums = tr->cand_sums;
+        a.tr_ncand = tr->ncand;
+        a.tr_scanned = tr->scanned;
+        a.tr_passed = tr->passed;
+        a.tr_rescans = tr->rescans;
+    }
+    const ah::DeviceIndex& dix = ix->dix;
+    const bool prof = ix->profiling && ix->ev_ready;
+    int launches = 0;
+    cudaError_t e;
+    auto mark = [&](int i) {
+        if (prof) cudaEventRecord(ix->ev[i], s);
+    };
+    e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)(2 * dix.nl + ix->ws.nq + 8), s);
+    if (e != cudaSuccess) return cuda_fail(e, "memset");
+    mark(0);
+    if ((e = ah::launch_centroid_scores(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "centroid scores");
+    launches += 1;
+    mark(1);
+    if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
+    launches += 1;
+    mark(2);
+    if ((e = ah::launch_invert(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "invert");
+    launches += 2;
+    mark(3);
+    if ((e = ah::launch_lut(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "lut");
+    launches += 1;
+    mark(4);
+    if ((e = ah::launch_threshold(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "threshold");
+    launches += 1;
+    mark(5);
+    if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
+    launches += 1;
+    mark(6);
+    if ((e = ah::launch_select(dix, a, b, 0, s)) != cudaSuccess) return cuda_fail(e, "select");
+    launches += 1;
+    mark(7);
+    for (int round = 1; round <= 2; ++round) {
+        if ((e = ah::launch_redo_scan(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "rescan");
+        if ((e = ah::launch_select(dix, a, b, round, s)) != cudaSuccess) return cuda_fail(e, "select after rescan");
+        launches += 2;
+    }
+    mark(8);
+    if (reorder_num > 0) {
+        if ((e = ah::launch_reorder(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "reorder");
+        launches += 2;
+    }
+    mark(9);
+    if (prof) ix->ev_recorded = true;
+    if (tr) {
+        const size_t nL = (size_t)nq * L;
+        if (tr->leaf_ids && (e = cudaMemcpyAsync(tr->leaf_ids, b.leaves, nL * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+            return cuda_fail(e, "trace copy");
+        if (tr->leaf_scores &&
+            (e = cudaMemcpyAsync(tr->leaf_scores, b.leaf_scores, nL * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+            return cuda_fail(e, "trace copy");
+        if (tr->scanned &&
+            (e = cudaMemcpyAsync(tr->scanned, b.scanned, (size_t)nq * 8, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+            return cuda_fail(e, "trace copy");
+        if (tr->rescans &&
+            (e = cudaMemcpyAsync(tr->rescans, b.counters + 1, 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+            return cuda_fail(e, "trace copy");
+    }
+    ix->last_launches = launches;
+    ix->last_nq = nq;
+    return AH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ah_status_string(ah_status s) {
+    switch (s) {
+        case AH_OK: return "ok";
+        case AH_ERR_INVALID_ARG: return "invalid argument";
+        case AH_ERR_UNSUPPORTED: return "unsupported";
+        case AH_ERR_OOM: return "out of device memory";
+        case AH_ERR_CUDA: return "CUDA error";
+        case AH_ERR_DEVICE: return "device-side error";
+        case AH_ERR_TIMEOUT: return "timeout";
+    }
+    return "unknown status";
+}
+
+const char* ah_last_error(void) { return g_last_error.c_str(); }
+
+ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_index** out) {
+    if (!out) return fail(AH_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!v) return fail(AH_ERR_INVALID_ARG, "views is NULL");
+    if (v->n <= 0 || v->n >= (int64_t(1) << 31) - 64) return fail(AH_ERR_INVALID_ARG, "n outside (0, 2^31 - 64)");
+    if (v->d <= 0 || v->dims_per_block <= 0 || v->num_leaves <= 0) return fail(AH_ERR_INVALID_ARG, "non-positive size");
+    if (v->d % (2 * v->dims_per_block) != 0) return fail(AH_ERR_INVALID_ARG, "d not divisible by 2 * dims_per_block");
+    if (v->d > AH_MAX_D) return fail(AH_ERR_UNSUPPORTED, "d above AH_MAX_D");
+    if (v->d / v->dims_per_block > AH_MAX_BLOCKS) return fail(AH_ERR_UNSUPPORTED, "blocks above AH_MAX_BLOCKS");
+    if (!v->centroids || !v->leaf_offsets || !v->slot_ids || !v->codes || !v->codebook)
+        return fail(AH_ERR_INVALID_ARG, "NULL index array");
+    if (v->reorder_dtype != AH_F32 && v->reorder_dtype != AH_BF16) return fail(AH_ERR_INVALID_ARG, "unknown reorder_dtype");
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    ah_index* ix = new (std::nothrow) ah_index();
+    if (!ix) return fail(AH_ERR_OOM, "host allocation");
+    ix->views = *v;
+    cudaError_t e = cudaGetDevice(&ix->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ix->num_sms, cudaDevAttrMultiProcessorCount, ix->device);
+    if (e != cudaSuccess) {
+        delete ix;
+        return cuda_fail(e, "device query");
+    }
+    const int B = v->d / v->dims_per_block;
+    const int cb = B / 2;
+    const int W = (cb + 3) / 4;
+    const int64_t tiles = (v->n + 31) / 32;
+    const size_t il_bytes = (size_t)tiles * W * 32 * sizeof(uint32_t);
+    const size_t offs_bytes = sizeof(int32_t) * (size_t)(v->num_leaves + 1);
+    if ((e = cudaMalloc(&ix->codes_il, il_bytes)) != cudaSuccess ||
+        (e = cudaMalloc(&ix->offs32, offs_bytes)) != cudaSuccess ||
+        (e = cudaMalloc(&ix->err, sizeof(int))) != cudaSuccess) {
+        ah_destroy(ix);
+        return cuda_fail(e, "index allocation");
+    }
+    ix->owned_bytes = il_bytes + offs_bytes + sizeof(int);
+    if ((e = cudaMemsetAsync(ix->err, 0, sizeof(int), s)) != cudaSuccess ||
+        (e = ah::launch_prepare_index(v->leaf_offsets, v->num_leaves, ix->offs32, v->codes, v->n, cb, W, ix->codes_il, s)) !=
+            cudaSuccess ||
+        (e = cudaStreamSynchronize(s)) != cudaSuccess) {
+        ah_destroy(ix);
+        return cuda_fail(e, "index preparation");
+    }
+    ah::DeviceIndex& d = ix->dix;
+    d.n = v->n;
+    d.d = v->d;
+    d.nl = v->num_leaves;
+    d.dpb = v->dims_per_block;
+    d.B = B;
+    d.W = W;
+    d.centroids = v->centroids;
+    d.offs = ix->offs32;
+    d.slot_ids = v->slot_ids;
+    d.codes_il = ix->codes_il;
+    d.codebook = v->codebook;
+    d.reorder_vecs = v->reorder_vecs;
+    d.reorder_bf16 = v->reorder_dtype == AH_BF16 ? 1 : 0;
+    *out = ix;
+    return AH_OK;
+}
+
+ah_status ah_reserve(ah_index* ix, int32_t max_nq, int32_t k, int32_t L, int32_t reorder_num, int32_t lut_mode) {
+    ah_status st = validate_search(ix, reinterpret_cast<void*>(1), max_nq, k, L, reorder_num, lut_mode,
+                                   reinterpret_cast<void*>(1), reinterpret_cast<void*>(1));
+    if (st != AH_OK) return st;
+    return carve(ix, std::max(max_nq, 1), L, std::max(reorder_num, k), lut_mode, k, false);
+}
+
+ah_status ah_search_traced(ah_index* ix, const float* queries, int32_t nq, int32_t k, int32_t L, int32_t reorder_num,
+                           int32_t lut_mode, int32_t* out_ids, float* out_scores, const ah_search_trace* trace,
+                           void* cuda_stream) {
+    ah_status st = validate_search(ix, queries, nq, k, L, reorder_num, lut_mode, out_ids, out_scores);
+    if (st != AH_OK || nq == 0) return st;
+    return run_search(ix, queries, nq, k, L, reorder_num, lut_mode, out_ids, out_scores, trace,
+                      static_cast<cudaStream_t>(cuda_stream));
+}
+
+ah_status ah_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, int32_t L, int32_t reorder_num,
+                    int32_t lut_mode, int32_t* out_ids, float* out_scores, void* cuda_stream) {
+    return ah_search_traced(ix, queries, nq, k, L, reorder_num, lut_mode, out_ids, out_scores, nullptr, cuda_stream);
+}
+
+ah_status ah_search_host(ah_index* ix, const float* host_queries, int32_t nq, int32_t k, int32_t L,
+                         int32_t reorder_num, int32_t lut_mode, int32_t* host_ids, float* host_scores,
+                         void* cuda_stream) {
+    ah_status st = validate_search(ix, host_queries, nq, k, L, reorder_num, lut_mode, host_ids, host_scores);
+    if (st != AH_OK || nq == 0) return st;
+    const int R = std::max(reorder_num, k);
+    st = carve(ix, nq, L, R, lut_mode, k, true);
+    if (st != AH_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    Workspace& w = ix->ws;
+    cudaError_t e = cudaMemcpyAsync(w.dq, host_queries, sizeof(float) * (size_t)nq * ix->dix.d, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "query upload");
+    st = run_search(ix, w.dq, nq, k, L, reorder_num, lut_mode, w.dids, w.dscores, nullptr, s);
+    if (st != AH_OK) return st;
+    if ((e = cudaMemcpyAsync(host_ids, w.dids, sizeof(int32_t) * (size_t)nq * k, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(host_scores, w.dscores, sizeof(float) * (size_t)nq * k, cudaMemcpyDeviceToHost, s)) !=
+            cudaSuccess)
+        return cuda_fail(e, "result download");
+    return ah_sync_status(ix, cuda_stream);
+}
+
+ah_status ah_sync_status(ah_index* ix, void* cuda_stream) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int code = 0;
+    if ((e = cudaMemcpy(&code, ix->err, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "error word read");
+    if (code == 0) return AH_OK;
+    int zero = 0;
+    cudaMemcpy(ix->err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    switch (code) {
+        case ah::kDevCandOverflow: return fail(AH_ERR_DEVICE, "candidate buffer overflow after the last rescan round");
+        case ah::kDevBadLeaf: return fail(AH_ERR_DEVICE, "leaf id out of range");
+        case ah::kDevSelectSize: return fail(AH_ERR_DEVICE, "selection size mismatch (duplicate keys)");
+        default: return fail(AH_ERR_DEVICE, "device error " + std::to_string(code));
+    }
+}
+
+ah_status ah_set_profiling(ah_index* ix, int32_t on) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    if (on && !ix->ev_ready) {
+        for (int i = 0; i <= kStages; ++i) {
+            cudaError_t e = cudaEventCreate(&ix->ev[i]);
+            if (e != cudaSuccess) return cuda_fail(e, "event create");
+        }
+        ix->ev_ready = true;
+    }
+    ix->profiling = on != 0;
+    ix->ev_recorded = false;
+    return AH_OK;
+}
+
+ah_status ah_stage_times(ah_index* ix, float* ms, int32_t max_stages, int32_t* n_stages) {
+    if (!ix || !ms || !n_stages) return fail(AH_ERR_INVALID_ARG, "NULL argument");
+    if (!ix->ev_recorded) return fail(AH_ERR_INVALID_ARG, "no profiled search recorded");
+    cudaError_t e = cudaEventSynchronize(ix->ev[kStages]);
+    if (e != cudaSuccess) return cuda_fail(e, "event synchronize");
+    int n = std::min<int>(kStages, max_stages);
+    for (int i = 0; i < n; ++i) {
+        e = cudaEventElapsedTime(&ms[i], ix->ev[i], ix->ev[i + 1]);
+        if (e != cudaSuccess) return cuda_fail(e, "event elapsed");
+    }
+    *n_stages = n;
+    return AH_OK;
+}
+
+const char* ah_stage_name(int32_t stage) {
+    if (stage < 0 || stage >= kStages) return "";
+    return kStageNames[stage];
+}
+
+ah_status ah_last_search_info(ah_index* ix, int32_t* launches, int64_t* points_scanned) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    if (launches) *launches = ix->last_launches;
+    if (points_scanned) {
+        *points_scanned = 0;
+        if (ix->last_nq > 0) {
+            cudaError_t e = cudaDeviceSynchronize();
+            if (e != cudaSuccess) return cuda_fail(e, "synchronize");
+            std::vector<int64_t> h(ix->last_nq);
+            e = cudaMemcpy(h.data(), ix->ws.buf.scanned, sizeof(int64_t) * h.size(), cudaMemcpyDeviceToHost);
+            if (e != cudaSuccess) return cuda_fail(e, "scanned read");
+            for (int64_t v : h) *points_scanned += v;
+        }
+    }
+    return AH_OK;
+}
+
+ah_status ah_index_memory(ah_index* ix, int64_t* bytes) {
+    if (!ix || !bytes) return fail(AH_ERR_INVALID_ARG, "NULL argument");
+    *bytes = static_cast<int64_t>(ix->owned_bytes);
+    return AH_OK;
+}
+
+void ah_destroy(ah_index* ix) {
+    if (!ix) return;
+    cudaDeviceSynchronize();
+    if (ix->ws.base) cudaFree(ix->ws.base);
+    if (ix->codes_il) cudaFree(ix->codes_il);
+    if (ix->offs32) cudaFree(ix->offs32);
+    if (ix->err) cudaFree(ix->err);
+    if (ix->ev_ready)
+        for (int i = 0; i <= kStages; ++i) cudaEventDestroy(ix->ev[i]);
+    delete ix;
+}
+
+}  // extern "C"

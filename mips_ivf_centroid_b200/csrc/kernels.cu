@@ -1,0 +1,960 @@
+// Search kernels of the B200 anisotropic-AH MIPS library.
+//
+// Path (ScaNN blog post, "Three stages of a search"):
+//   centroid_scores_kernel   s[q][c] = q . centroid_c                 (partitioning)
+//   top_leaves_kernel        best L leaves per query
+//   invert_*                 query->leaf lists become leaf->query lists, so a
+//                            leaf's codes are read once per query group
+//   lut_*_kernel             lut[q][b][j] = q_b . center[b][j]        (AH table)
+//   threshold_kernel         a lower bound on each query's R-th best approximate
+//                            score, from a prefix of its best leaves
+//   scan_kernel              leaf-major 4-bit code scan: per slot, the sum of
+//                            table entries for every query of the group;
+//                            scores at or above the bound are kept
+//   redo_scan_kernel         query-major rescan for the rare query whose kept
+//                            set overflowed its buffer (with a tighter bound)
+//   rerank_kernel            best R by approximate score, exact fp32 dot
+//                            products for them (reordering), best k
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "select.cuh"
+
+namespace ah {
+
+// ---------------------------------------------------------------------------
+// index preparation
+// ---------------------------------------------------------------------------
+
+__global__ void offsets_to_i32_kernel(const int64_t* __restrict__ o64, int nl, int32_t* __restrict__ o32) {
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i <= nl) o32[i] = static_cast<int32_t>(o64[i]);
+}
+
+// codes [n][cb] bytes -> il[tile][w][lane] 32-bit words (slot = 32*tile + lane,
+// word w holds code bytes 4w..4w+3; bytes past cb and slots past n are 0).
+__global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, int64_t n, int cb, int W,
+                                        uint32_t* __restrict__ il, int64_t total_words) {
+    int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (e >= total_words) return;
+    int lane = static_cast<int>(e & 31);
+    int64_t tw = e >> 5;                 // tile*W + w
+    int w = static_cast<int>(tw % W);
+    int64_t tile = tw / W;
+    int64_t slot = tile * 32 + lane;
+    uint32_t v = 0;
+    if (slot < n) {
+        const uint8_t* row = codes + slot * cb;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int byte = 4 * w + i;
+            if (byte < cb) v |= static_cast<uint32_t>(row[byte]) << (8 * i);
+        }
+    }
+    il[e] = v;
+}
+
+cudaError_t launch_prepare_index(const int64_t* offs64, int nl, int32_t* offs32, const uint8_t* codes,
+                                 int64_t n, int cb, int W, uint32_t* codes_il, cudaStream_t s) {
+    offsets_to_i32_kernel<<<(nl + 1 + 255) / 256, 256, 0, s>>>(offs64, nl, offs32);
+    int64_t tiles = (n + 31) / 32;
+    int64_t total = tiles * W * 32;
+    int64_t grid = (total + 255) / 256;
+    interleave_codes_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, n, cb, W, codes_il, total);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// partitioning: centroid scores and top-L leaves
+// ---------------------------------------------------------------------------
+
+constexpr int kGemmBM = 64, kGemmBN = 64, kGemmBK = 16;
+
+// S[q][c] = sum_t Q[q][t] * C[c][t]  (fp32, SIMT; 64x64 tile, 4x4 per thread)
+__global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __restrict__ Q, const float* __restrict__ C,
+                                                              float* __restrict__ S, int nq, int nl, int d) {
+    __shared__ float As[kGemmBK][kGemmBM + 4];
+    __shared__ float Bs[kGemmBK][kGemmBN + 4];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+    for (int k0 = 0; k0 < d; k0 += kGemmBK) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            int e = threadIdx.x + 256 * r;
+            int row = e >> 4, col = e & 15;
+            int gk = k0 + col;
+            int gm = m0 + row, gn = n0 + row;
+            As[col][row] = (gm < nq && gk < d) ? Q[static_cast<int64_t>(gm) * d + gk] : 0.0f;
+            Bs[col][row] = (gn < nl && gk < d) ? C[static_cast<int64_t>(gn) * d + gk] : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kGemmBK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int gm = m0 + ty + 16 * i;
+        if (gm >= nq) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int gn = n0 + tx + 16 * j;
+            if (gn < nl) S[static_cast<int64_t>(gm) * nl + gn] = acc[i][j];
+        }
+    }
+}
+
+cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    dim3 grid((ix.nl + kGemmBN - 1) / kGemmBN, (a.nq + kGemmBM - 1) / kGemmBM);
+    centroid_scores_kernel<<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+    return cudaGetLastError();
+}
+
+constexpr int kSelThreads = 256;
+
+// One CTA per query: best L leaves by (score desc, leaf id asc); counts the
+// queries per leaf and the points the query will scan.
+__global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ SelectScratch scr;
+    __shared__ long long s_scanned;
+    const int q = blockIdx.x;
+    const int L = a.L, nl = ix.nl;
+    const int P2 = next_pow2(L);
+    uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
+    const float* grow = b.cscore + static_cast<int64_t>(q) * nl;
+    const float* row = grow;
+    if (a.topl_row_smem) {                    // stage the score row once; the selection reads it several times
+        float* srow = reinterpret_cast<float*>(keys + P2);
+        for (int i = threadIdx.x; i < nl; i += kSelThreads) srow[i] = grow[i];
+        __syncthreads();
+        row = srow;
+    }
+    auto get = [&](int i) { return make_key(float_key(row[i]), i); };
+    auto pay = [&](int i) { return i; };
+    if (threadIdx.x == 0) s_scanned = 0;
+    block_topk<kSelThreads>(get, pay, nl, L, scr, keys, nullptr, b.err);
+    long long local = 0;
+    for (int i = threadIdx.x; i < L; i += kSelThreads) {
+        uint64_t key = keys[i];
+        int leaf = key_id(key);
+        b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
+        b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
+        atomicAdd(&b.qcount[leaf], 1);
+        local += ix.offs[leaf + 1] - ix.offs[leaf];
+    }
+    atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
+    __syncthreads();
+    if (threadIdx.x == 0) b.scanned[q] = s_scanned;
+}
+
+cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+    size_t smem = static_cast<size_t>(next_pow2(a.L)) * sizeof(uint64_t);
+    const size_t row = static_cast<size_t>(ix.nl) * sizeof(float);
+    a.topl_row_smem = (row <= 64 * 1024) ? 1 : 0;
+    if (a.topl_row_smem) smem += row;
+    cudaError_t e = cudaFuncSetAttribute(top_leaves_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    top_leaves_kernel<<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// inversion: leaf -> query lists and the scan work items
+// ---------------------------------------------------------------------------
+
+constexpr int kScanBlock = 1024;
+
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_sums[lane];
+        int xs = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            int y = __shfl_up_sync(0xFFFFFFFFu, xs, off);
+            if (lane >= off) xs += y;
+        }
+        warp_sums[lane] = xs - w;   // exclusive prefix of warps
+        if (lane == 31) *total = xs;
+    }
+    __syncthreads();
+    int r = warp_sums[warp] + x - v;
+    __syncthreads();
+    return r;
+}
+
+// Single CTA: qoff = exclusive scan of queries per leaf; item_off = exclusive
+// scan of work items per leaf (query groups x slot chunks).
+__global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex ix, SearchBuffers b, int group, int chunk) {
+    __shared__ int warp_sums[32];
+    __shared__ int total_q, total_i;
+    int carry_q = 0, carry_i = 0;
+    for (int base = 0; base < ix.nl; base += kScanBlock) {
+        int c = base + threadIdx.x;
+        int qc = 0, it = 0;
+        if (c < ix.nl) {
+            qc = b.qcount[c];
+            int sz = ix.offs[c + 1] - ix.offs[c];
+            it = (qc > 0 && sz > 0) ? ((qc + group - 1) / group) * ((sz + chunk - 1) / chunk) : 0;
+        }
+        int eq = block_exclusive_scan_1024(qc, warp_sums, &total_q);
+        int ei = block_exclusive_scan_1024(it, warp_sums, &total_i);
+        if (c < ix.nl) {
+            b.qoff[c] = carry_q + eq;
+            b.item_off[c] = carry_i + ei;
+        }
+        carry_q += total_q;
+        carry_i += total_i;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        b.qoff[ix.nl] = carry_q;
+        b.item_off[ix.nl] = carry_i;
+    }
+}
+
+__global__ void invert_scatter_kernel(SearchArgs a, SearchBuffers b) {
+    int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    int64_t total = static_cast<int64_t>(a.nq) * a.L;
+    if (e >= total) return;
+    int q = static_cast<int>(e / a.L);
+    int leaf = b.leaves[e];
+    int pos = atomicAdd(&b.qcursor[leaf], 1);
+    b.qlist[b.qoff[leaf] + pos] = q;
+}
+
+cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    invert_offsets_kernel<<<1, kScanBlock, 0, s>>>(ix, b, scan_group(a.lut_mode), a.chunk);
+    int64_t total = static_cast<int64_t>(a.nq) * a.L;
+    invert_scatter_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(a, b);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// lookup tables
+// ---------------------------------------------------------------------------
+
+// lut[q][b][j] = q[b*dpb] * c[0], then fmaf(q[b*dpb+t], c[t], lut) for t >= 1.
+__device__ __forceinline__ float lut_entry(const float* __restrict__ q, const float* __restrict__ c, int dpb) {
+    float v = __fmul_rn(q[0], c[0]);
+    for (int t = 1; t < dpb; ++t) v = fmaf(q[t], c[t], v);
+    return v;
+}
+
+__global__ void lut_f32_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int per_q = ix.B * kCenters;
+    if (e >= static_cast<int64_t>(a.nq) * per_q) return;
+    int q = static_cast<int>(e / per_q);
+    int r = static_cast<int>(e - static_cast<int64_t>(q) * per_q);
+    int blk = r >> 4;
+    b.lut_f32[e] = lut_entry(a.queries + static_cast<int64_t>(q) * ix.d + blk * ix.dpb,
+                             ix.codebook + static_cast<int64_t>(r) * ix.dpb, ix.dpb);
+}
+
+// One CTA per query: the uint8 table, delta and bias, all in fp32 with
+// round-to-nearest operations in a fixed order.
+__global__ void __launch_bounds__(256) lut_u8_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    float* lut = reinterpret_cast<float*>(smem);          // [B*16]
+    float* mins = lut + ix.B * kCenters;                  // [B]
+    __shared__ unsigned int s_range_bits;
+    const int q = blockIdx.x;
+    const int per_q = ix.B * kCenters;
+    const float* qv = a.queries + static_cast<int64_t>(q) * ix.d;
+    if (threadIdx.x == 0) s_range_bits = 0u;
+    for (int r = threadIdx.x; r < per_q; r += blockDim.x)
+        lut[r] = lut_entry(qv + (r >> 4) * ix.dpb, ix.codebook + static_cast<int64_t>(r) * ix.dpb, ix.dpb);
+    __syncthreads();
+    for (int blk = threadIdx.x; blk < ix.B; blk += blockDim.x) {
+        float lo = lut[blk * kCenters], hi = lo;
+        for (int j = 1; j < kCenters; ++j) {
+            lo = fminf(lo, lut[blk * kCenters + j]);
+            hi = fmaxf(hi, lut[blk * kCenters + j]);
+        }
+        mins[blk] = lo;
+        float range = __fsub_rn(hi, lo);                  // >= 0: bits order as floats
+        atomicMax(&s_range_bits, __float_as_uint(range));
+    }
+    __syncthreads();
+    float delta = __fdiv_rn(__uint_as_float(s_range_bits), 255.0f);
+    if (delta == 0.0f) delta = 1.0f;
+    uint8_t* out = b.lut_u8 + static_cast<int64_t>(q) * per_q;
+    for (int r = threadIdx.x; r < per_q; r += blockDim.x) {
+        float v = rintf(__fdiv_rn(__fsub_rn(lut[r], mins[r >> 4]), delta));
+        out[r] = static_cast<uint8_t>(fminf(v, 255.0f));
+    }
+    if (threadIdx.x == 0) {
+        float bias = 0.0f;
+        for (int blk = 0; blk < ix.B; ++blk) bias = __fadd_rn(bias, mins[blk]);
+        b.lut_delta[q] = delta;
+        b.lut_bias[q] = bias;
+    }
+}
+
+cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    if (a.lut_mode == 0) {
+        int64_t total = static_cast<int64_t>(a.nq) * ix.B * kCenters;
+        lut_f32_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(ix, a, b);
+    } else {
+        size_t smem = (static_cast<size_t>(ix.B) * kCenters + ix.B) * sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(lut_u8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        lut_u8_kernel<<<a.nq, 256, smem, s>>>(ix, a, b);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// per-slot approximate score (query-major kernels): sum over blocks in order
+// ---------------------------------------------------------------------------
+
+// fp32: table in shared memory as [B][16] floats; returns the score key.
+// uint8: table as [B][16] bytes; returns the integer sum.
+template <int MODE>
+__device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int B,
+                                               const unsigned char* lut, int32_t slot) {
+    const uint32_t* cw = codes_il + (static_cast<int64_t>(slot >> 5) * W) * 32 + (slot & 31);
+    if (MODE == 0) {
+        const float* lf = reinterpret_cast<const float*>(lut);
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) {
+            uint32_t c = cw[w * 32];
+            int nb = min(8, B - 8 * w);
+            for (int i = 0; i < nb; ++i) acc = __fadd_rn(acc, lf[(8 * w + i) * kCenters + ((c >> (4 * i)) & 15u)]);
+        }
+        return float_key(acc);
+    } else {
+        uint32_t acc = 0;
+        for (int w = 0; w < W; ++w) {
+            uint32_t c = cw[w * 32];
+            int nb = min(8, B - 8 * w);
+            for (int i = 0; i < nb; ++i) acc += lut[(8 * w + i) * kCenters + ((c >> (4 * i)) & 15u)];
+        }
+        return acc;
+    }
+}
+
+// Four slots at once (independent chains for latency hiding); each slot's sum
+// still runs over blocks in order, identical to slot_value.
+template <int MODE>
+__device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int B,
+                                             const unsigned char* lut, const int32_t* slot, const bool* valid,
+                                             uint32_t* out) {
+    const uint32_t* cw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int32_t sl = valid[u] ? slot[u] : 0;
+        cw[u] = codes_il + (static_cast<int64_t>(sl >> 5) * W) * 32 + (sl & 31);
+    }
+    if (MODE == 0) {
+        const float* lf = reinterpret_cast<const float*>(lut);
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int w = 0; w < W; ++w) {
+            uint32_t c[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) c[u] = cw[u][w * 32];
+            const int nb = min(8, B - 8 * w);
+            const float* base = lf + 8 * w * kCenters;
+            if (nb == 8) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u] >> (4 * i)) & 15u)]);
+            } else {
+                for (int i = 0; i < nb; ++i)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u] >> (4 * i)) & 15u)]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) out[u] = float_key(acc[u]);
+    } else {
+        uint32_t acc[4] = {0u, 0u, 0u, 0u};
+        for (int w = 0; w < W; ++w) {
+            uint32_t c[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) c[u] = cw[u][w * 32];
+            const int nb = min(8, B - 8 * w);
+            const unsigned char* base = lut + 8 * w * kCenters;
+            for (int i = 0; i < nb; ++i)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u] += base[i * kCenters + ((c[u] >> (4 * i)) & 15u)];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) out[u] = acc[u];
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void load_query_table(const DeviceIndex& ix, const SearchBuffers& b, int q, unsigned char* lut) {
+    const int per_q = ix.B * kCenters;
+    if (MODE == 0) {
+        float* lf = reinterpret_cast<float*>(lut);
+        const float* src = b.lut_f32 + static_cast<int64_t>(q) * per_q;
+        for (int r = threadIdx.x; r < per_q; r += blockDim.x) lf[r] = src[r];
+    } else {
+        const uint8_t* src = b.lut_u8 + static_cast<int64_t>(q) * per_q;
+        for (int r = threadIdx.x; r < per_q; r += blockDim.x) lut[r] = src[r];
+    }
+}
+
+__host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
+    return B * kCenters * (mode == 0 ? 4 : 1);
+}
+
+// ---------------------------------------------------------------------------
+// threshold: R-th best approximate score over a prefix of the best leaves
+// ---------------------------------------------------------------------------
+
+// One CTA per query.  Scores the first M = min(points, max(R, 1024)) slots of
+// the query's leaves in rank order; the R-th largest (score, id) key among them
+// is a lower bound on the R-th largest over all its leaves (a subset's R-th
+// best can only be lower), so every point of the final top R has a key >= it.
+// With fewer than R points in total the bound is 0 (keep everything).
+template <int MODE>
+__global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ SelectScratch scr;
+    const int q = blockIdx.x;
+    const int R = a.R;
+    unsigned char* lut = smem;
+    uint64_t* vals = reinterpret_cast<uint64_t*>(smem + ((table_bytes(MODE, ix.B) + 15) & ~15));
+    uint64_t* top = vals + kMaxThresholdSample;
+    load_query_table<MODE>(ix, b, q, lut);
+    __syncthreads();
+    const int M = min(kMaxThresholdSample, max(R, 1024));
+    int taken = 0;
+    for (int i = 0; i < a.L && taken < M; ++i) {
+        int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
+        int s0 = ix.offs[leaf], sz = ix.offs[leaf + 1] - s0;
+        int m = min(sz, M - taken);
+        for (int t0 = 0; t0 < m; t0 += 4 * kSelThreads) {
+            int32_t sl[4];
+            bool ok[4];
+            uint32_t v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + u * kSelThreads + threadIdx.x;
+                ok[u] = t < m;
+                sl[u] = s0 + t;
+            }
+            slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, sl, ok, v);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + u * kSelThreads + threadIdx.x;
+                if (ok[u]) vals[taken + t] = make_key(v[u], ix.slot_ids[sl[u]]);
+            }
+        }
+        taken += m;
+    }
+    __syncthreads();
+    uint64_t tau = 0ull;
+    if (taken >= R) {
+        auto get = [&](int i) { return vals[i]; };
+        auto pay = [&](int i) { return i; };
+        block_topk<kSelThreads>(get, pay, taken, R, scr, top, nullptr, b.err);
+        tau = top[R - 1];
+    }
+    if (threadIdx.x == 0) b.tau[q] = tau;
+}
+
+cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + kMaxThresholdSample * sizeof(uint64_t) +
+                  static_cast<size_t>(next_pow2(a.R)) * sizeof(uint64_t);
+    cudaError_t e;
+    if (a.lut_mode == 0) {
+        e = cudaFuncSetAttribute(threshold_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        threshold_kernel<0><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+    } else {
+        e = cudaFuncSetAttribute(threshold_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        threshold_kernel<1><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// the code scan (leaf-major)
+// ---------------------------------------------------------------------------
+
+// Does (value, id of slot) reach the bound (th, tl)?  The id is only read for
+// an exact tie on the score part.
+__device__ __forceinline__ bool reaches(uint32_t v, uint32_t th, uint32_t tl, const int32_t* __restrict__ slot_ids,
+                                        int32_t slot) {
+    if (v != th) return v > th;
+    return (0xFFFFFFFFu - static_cast<uint32_t>(slot_ids[slot])) >= tl;
+}
+
+// Warp-aggregated append of the lanes with `pass` set to query q's buffer, as
+// full (score key, id) keys.  Entries past the capacity are counted, not stored.
+__device__ __forceinline__ void append_candidates(bool pass, uint32_t key, int32_t slot, int q, const DeviceIndex& ix,
+                                                  const SearchBuffers& b) {
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, pass);
+    if (m == 0u) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(&b.count[q], __popc(m));
+    base = __shfl_sync(0xFFFFFFFFu, base, leader);
+    if (pass) {
+        int pos = base + __popc(m & ((1u << lane) - 1u));
+        if (pos < b.cap) {
+            const int64_t o = static_cast<int64_t>(q) * b.cap + pos;
+            b.ckey[o] = make_key(key, ix.slot_ids[slot]);
+            b.cslot[o] = slot;
+        }
+    }
+}
+
+// Persistent CTAs take work items (leaf, query group of G, chunk of slots) from
+// an atomic counter.  Per item the group's tables are staged in shared memory:
+//   fp32: [b][G/2][16][2] floats: one 8-byte load fetches query pair
+//         (2p, 2p+1)'s entries for center j; a (block, pair) table is 128 B.
+//   u8:   [b][G/4][16][4] bytes: one 4-byte load fetches 4 queries' entries.
+// Each lane owns one slot of a 32-slot tile and walks its code words; per
+// nibble it issues G/2 (fp32) or G/4 (u8) shared loads.  Sums run over blocks
+// in order 0..B-1 with IEEE fp32 adds (two lanes per packed f32x2 add), the
+// same order as the query-major kernels, so a slot's score is bit-identical
+// in every kernel.
+template <int G, int MODE>
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_item, s_leaf;
+    __shared__ int s_q[G];
+    __shared__ uint32_t s_th[G], s_tl[G];
+    const int B = ix.B, W = ix.W;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int NW = kScanThreads / 32;
+    const int total_items = b.item_off[ix.nl];
+    const int blk_bytes = (MODE == 0) ? G * 64 : G * 16;     // one block's tables for the group
+    // work-item offsets per leaf, copied once per CTA when they fit
+    const size_t lut_bytes = static_cast<size_t>(B) * blk_bytes;
+    int* s_item_off = reinterpret_cast<int*>(smem + lut_bytes);
+    const bool off_in_smem = a.scan_item_off_smem != 0;
+    if (off_in_smem)
+        for (int i = threadIdx.x; i <= ix.nl; i += kScanThreads) s_item_off[i] = b.item_off[i];
+    const int* item_off = off_in_smem ? s_item_off : b.item_off;
+
+    for (;;) {
+        __syncthreads();   // previous item's tables are no longer read
+        if (threadIdx.x == 0) {
+            int item = atomicAdd(&b.counters[0], 1);
+            s_item = item;
+            if (item < total_items) {
+                int lo = 0, hi = ix.nl;
+                while (lo < hi) {
+                    int mid = (lo + hi + 1) >> 1;
+                    if (item_off[mid] <= item) lo = mid; else hi = mid - 1;
+                }
+                s_leaf = lo;
+            }
+        }
+        __syncthreads();
+        const int item = s_item;
+        if (item >= total_items) break;
+        const int leaf = s_leaf;
+        const int off0 = ix.offs[leaf], nslots = ix.offs[leaf + 1] - off0;
+        const int npc = (nslots + a.chunk - 1) / a.chunk;
+        const int local = item - item_off[leaf];
+        const int g = local / npc, c = local - g * npc;
+        const int qcnt = b.qcount[leaf];
+        const int gsize = min(G, qcnt - g * G);
+        const int s0 = off0 + c * a.chunk;
+        const int s1 = min(off0 + nslots, s0 + a.chunk);
+        if (threadIdx.x < G) {
+            int qq = (threadIdx.x < gsize) ? b.qlist[b.qoff[leaf] + g * G + threadIdx.x] : -1;
+            s_q[threadIdx.x] = qq;
+            uint64_t t = (qq >= 0) ? b.tau[qq] : ~0ull;
+            s_th[threadIdx.x] = static_cast<uint32_t>(t >> 32);
+            s_tl[threadIdx.x] = static_cast<uint32_t>(t);
+        }
+        __syncthreads();
+        // stage the group's tables
+        const int per_q = B * kCenters;
+        if (MODE == 0) {
+            float* lf = reinterpret_cast<float*>(smem);
+            for (int e = threadIdx.x; e < G * per_q; e += kScanThreads) {
+                int qi = e / per_q, r = e - qi * per_q;
+                int blk = r >> 4, j = r & 15;
+                int qq = s_q[qi];
+                float v = (qq >= 0) ? b.lut_f32[static_cast<int64_t>(qq) * per_q + r] : 0.0f;
+                lf[((blk * (G / 2) + (qi >> 1)) * kCenters + j) * 2 + (qi & 1)] = v;
+            }
+        } else {
+            for (int e = threadIdx.x; e < G * per_q; e += kScanThreads) {
+                int qi = e / per_q, r = e - qi * per_q;
+                int blk = r >> 4, j = r & 15;
+                int qq = s_q[qi];
+                uint8_t v = (qq >= 0) ? b.lut_u8[static_cast<int64_t>(qq) * per_q + r] : 0;
+                smem[((blk * (G / 4) + (qi >> 2)) * kCenters + j) * 4 + (qi & 3)] = v;
+            }
+        }
+        __syncthreads();
+
+        const int t0 = s0 >> 5, t1 = (s1 - 1) >> 5;
+        for (int t = t0 + warp; t <= t1; t += NW) {
+            const int slot = t * 32 + lane;
+            const bool valid = (slot >= s0) && (slot < s1);
+            const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
+            if (MODE == 0) {
+                unsigned long long acc[G / 2];
+#pragma unroll
+                for (int p = 0; p < G / 2; ++p) acc[p] = 0ull;
+                for (int w0 = 0; w0 < W; w0 += 8) {
+                    uint32_t cw[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) cw[u] = (w0 + u < W) ? cwp[(w0 + u) * 32] : 0u;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int wi = w0 + u;
+                        if (wi >= W) break;
+                        const int nb = min(8, B - 8 * wi);
+                        const unsigned char* pb = smem + static_cast<size_t>(8 * wi) * blk_bytes;
+#pragma unroll
+                        for (int nib = 0; nib < 8; ++nib) {
+                            if (nib < nb) {
+                                const uint32_t j = (cw[u] >> (4 * nib)) & 15u;
+                                const unsigned long long* p =
+                                    reinterpret_cast<const unsigned long long*>(pb + nib * blk_bytes) + j;
+#pragma unroll
+                                for (int pr = 0; pr < G / 2; ++pr) acc[pr] = add_f32x2(acc[pr], p[pr * kCenters]);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int qi = 0; qi < G; ++qi) {
+                    if (qi >= gsize) break;
+                    const float sc = (qi & 1) ? hi_f32(acc[qi >> 1]) : lo_f32(acc[qi >> 1]);
+                    const uint32_t key = float_key(sc);
+                    append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot,
+                                      s_q[qi], ix, b);
+                }
+            } else {
+                uint32_t sums[G];
+#pragma unroll
+                for (int qi = 0; qi < G; ++qi) sums[qi] = 0u;
+                for (int w0 = 0; w0 < W; w0 += 8) {
+                    uint32_t cw[8];
+                    uint32_t ae[G / 4], ao[G / 4];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) cw[u] = (w0 + u < W) ? cwp[(w0 + u) * 32] : 0u;
+#pragma unroll
+                    for (int p = 0; p < G / 4; ++p) { ae[p] = 0u; ao[p] = 0u; }
+                    // 8 words = 64 blocks: 16-bit lanes hold at most 64 * 255
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int wi = w0 + u;
+                        if (wi >= W) break;
+                        const int nb = min(8, B - 8 * wi);
+                        const unsigned char* pb = smem + static_cast<size_t>(8 * wi) * blk_bytes;
+#pragma unroll
+                        for (int nib = 0; nib < 8; ++nib) {
+                            if (nib < nb) {
+                                const uint32_t j = (cw[u] >> (4 * nib)) & 15u;
+                                const uint32_t* p = reinterpret_cast<const uint32_t*>(pb + nib * blk_bytes) + j;
+#pragma unroll
+                                for (int qd = 0; qd < G / 4; ++qd) {
+                                    const uint32_t v = p[qd * kCenters];
+                                    ae[qd] += v & 0x00FF00FFu;
+                                    ao[qd] += __byte_perm(v, 0u, 0x4341);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int qd = 0; qd < G / 4; ++qd) {
+                        sums[4 * qd + 0] += ae[qd] & 0xFFFFu;
+                        sums[4 * qd + 2] += ae[qd] >> 16;
+                        sums[4 * qd + 1] += ao[qd] & 0xFFFFu;
+                        sums[4 * qd + 3] += ao[qd] >> 16;
+                    }
+                }
+#pragma unroll
+                for (int qi = 0; qi < G; ++qi) {
+                    if (qi >= gsize) break;
+                    append_candidates(valid && reaches(sums[qi], s_th[qi], s_tl[qi], ix.slot_ids, slot), sums[qi],
+                                      slot, s_q[qi], ix, b);
+                }
+            }
+        }
+    }
+}
+
+int scan_group(int lut_mode) { return lut_mode == 0 ? kGroupF32 : kGroupU8; }
+
+template <int G, int MODE>
+static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
+                                 cudaStream_t s) {
+    size_t smem = static_cast<size_t>(ix.B) * G * kCenters * (MODE == 0 ? 4 : 1);
+    const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
+    a.scan_item_off_smem = (smem + off_bytes <= 200 * 1024 && off_bytes <= 64 * 1024) ? 1 : 0;
+    if (a.scan_item_off_smem) smem += off_bytes;
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<G, MODE>, kScanThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    scan_kernel<G, MODE><<<num_sms * per_sm, kScanThreads, smem, s>>>(ix, a, b);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s) {
+    if (a.lut_mode == 0) return launch_scan_t<kGroupF32, 0>(ix, a, b, num_sms, s);
+    return launch_scan_t<kGroupU8, 1>(ix, a, b, num_sms, s);
+}
+
+// ---------------------------------------------------------------------------
+// redo scan (query-major, rare): rescan a query's leaves with its tighter bound
+// ---------------------------------------------------------------------------
+
+// Persistent CTAs take (redo query, leaf rank) pairs from a counter; each pair
+// rescans one leaf for one query with the query's tighter bound.  With no query
+// to redo every CTA exits after one atomic.
+template <int MODE>
+__global__ void __launch_bounds__(kSelThreads) redo_scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_item;
+    const int* list = b.redo + static_cast<int64_t>(round - 1) * a.nq;
+    const int total = b.counters[round] * a.L;
+    int loaded_q = -1;
+    for (;;) {
+        __syncthreads();
+        if (threadIdx.x == 0) s_item = atomicAdd(&b.counters[2 + round], 1);
+        __syncthreads();
+        const int item = s_item;
+        if (item >= total) break;
+        const int r = item / a.L, i = item - r * a.L;
+        const int q = list[r];
+        if (q != loaded_q) {
+            load_query_table<MODE>(ix, b, q, smem);
+            loaded_q = q;
+            __syncthreads();
+        }
+        const uint64_t tau = b.tau[q];
+        const uint32_t th = static_cast<uint32_t>(tau >> 32), tl = static_cast<uint32_t>(tau);
+        const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
+        const int s0 = ix.offs[leaf], s1 = ix.offs[leaf + 1];
+        for (int base = s0; base < s1; base += kSelThreads) {
+            const int slot = base + threadIdx.x;
+            const bool in = slot < s1;
+            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot) : 0u;
+            append_candidates(in && reaches(v, th, tl, ix.slot_ids, slot), v, slot, q, ix, b);
+        }
+    }
+}
+
+cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round,
+                             int num_sms, cudaStream_t s) {
+    size_t smem = table_bytes(a.lut_mode, ix.B);
+    cudaError_t e;
+    const int grid = num_sms * 2;
+    if (a.lut_mode == 0) {
+        e = cudaFuncSetAttribute(redo_scan_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        redo_scan_kernel<0><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
+    } else {
+        e = cudaFuncSetAttribute(redo_scan_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        redo_scan_kernel<1><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// select best R, exact reorder, best k
+// ---------------------------------------------------------------------------
+
+size_t select_smem_bytes(int R) {
+    return static_cast<size_t>(next_pow2(R)) * (sizeof(uint64_t) + sizeof(int32_t));
+}
+
+// One CTA per query (round 0) or per entry of the previous round's redo list.
+// Keeps the best R of the query's buffer (by (approximate score, id) key).
+// A query whose buffer overflowed instead gets a tighter bound (the R-th best
+// stored key: stored entries are real candidates, so this is still a lower
+// bound on its R-th best) and is queued for a rescan; on the last round an
+// overflow is reported through the error word and the stored subset is used.
+// Without reorder the best k of the R are the result.
+template <int MODE>
+__global__ void __launch_bounds__(kSelThreads) select_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ SelectScratch scr;
+    int q;
+    if (round == 0) {
+        q = blockIdx.x;
+    } else {
+        if (static_cast<int>(blockIdx.x) >= b.counters[round]) return;
+        q = b.redo[static_cast<int64_t>(round - 1) * a.nq + blockIdx.x];
+    }
+    const int cap = b.cap, R = a.R, k = a.k;
+    const int P2 = next_pow2(R);
+    uint64_t* okeys = reinterpret_cast<uint64_t*>(smem);                 // [P2]
+    int32_t* oslots = reinterpret_cast<int32_t*>(okeys + P2);            // [P2]
+    const uint64_t* ck = b.ckey + static_cast<int64_t>(q) * cap;
+    const int32_t* cs = b.cslot + static_cast<int64_t>(q) * cap;
+    int cnt = b.count[q];
+    if (round == 0 && a.tr_passed && threadIdx.x == 0) a.tr_passed[q] = cnt;
+    if (cnt > cap) {
+        if (round < 2) {
+            auto get = [&](int i) { return ck[i]; };
+            auto pay = [&](int i) { return i; };
+            block_topk<kSelThreads>(get, pay, cap, R, scr, okeys, nullptr, b.err);
+            if (threadIdx.x == 0) {
+                b.tau[q] = okeys[R - 1];
+                b.count[q] = 0;
+                int pos = atomicAdd(&b.counters[round + 1], 1);
+                b.redo[static_cast<int64_t>(round) * a.nq + pos] = q;
+            }
+            return;
+        }
+        if (threadIdx.x == 0) raise_error(b.err, kDevCandOverflow);
+        cnt = cap;
+    }
+    auto get = [&](int i) { return ck[i]; };
+    auto pay = [&](int i) { return cs[i]; };
+    const int K = block_topk<kSelThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+    const float delta = (MODE == 1) ? b.lut_delta[q] : 0.0f;
+    const float bias = (MODE == 1) ? b.lut_bias[q] : 0.0f;
+    auto approx_score = [&](uint32_t sk) {
+        return (MODE == 0) ? key_float(sk) : fmaf(delta, static_cast<float>(sk), bias);
+    };
+    const int64_t ro = static_cast<int64_t>(q) * R;
+    for (int i = threadIdx.x; i < R; i += kSelThreads) {
+        const bool have = i < K;
+        b.rkey[ro + i] = have ? okeys[i] : 0ull;
+        b.rslot[ro + i] = have ? oslots[i] : -1;
+        if (a.tr_cand_ids) a.tr_cand_ids[ro + i] = have ? key_id(okeys[i]) : -1;
+        if (a.tr_cand_scores) a.tr_cand_scores[ro + i] = have ? approx_score(key_score(okeys[i])) : -INFINITY;
+        if (a.tr_cand_sums) a.tr_cand_sums[ro + i] = (have && MODE == 1) ? key_score(okeys[i]) : 0u;
+    }
+    if (threadIdx.x == 0) {
+        b.rcount[q] = K;
+        if (a.tr_ncand) a.tr_ncand[q] = K;
+    }
+    if (a.reorder_num == 0) {
+        const int64_t oo = static_cast<int64_t>(q) * k;
+        for (int i = threadIdx.x; i < k; i += kSelThreads) {
+            const bool have = i < K;
+            a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
+            a.out_scores[oo + i] = have ? approx_score(key_score(okeys[i])) : -INFINITY;
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    return v;
+}
+
+constexpr int kReorderThreads = 256;
+
+// Reordering: one warp per (query, kept candidate) computes the exact fp32 dot
+// product with the stored vector (float, or bfloat16 upcast), lanes striding
+// over d, then a butterfly sum.  Writes the (exact score, id) key.
+__global__ void __launch_bounds__(kReorderThreads) reorder_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    const int lane = threadIdx.x & 31;
+    const int64_t p = static_cast<int64_t>(blockIdx.x) * (kReorderThreads / 32) + (threadIdx.x >> 5);
+    const int R = a.R, d = ix.d;
+    if (p >= static_cast<int64_t>(a.nq) * R) return;
+    const int q = static_cast<int>(p / R), i = static_cast<int>(p - static_cast<int64_t>(q) * R);
+    if (i >= b.rcount[q]) {
+        if (lane == 0) b.ekey[p] = 0ull;
+        return;
+    }
+    const int64_t slot = b.rslot[p];
+    const float* qv = a.queries + static_cast<int64_t>(q) * d;
+    float acc = 0.0f;
+    if (ix.reorder_bf16) {
+        const uint16_t* v = reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d;
+        for (int t = lane; t < d; t += 32) acc = fmaf(qv[t], __uint_as_float(static_cast<uint32_t>(v[t]) << 16), acc);
+    } else {
+        const float* v = reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d;
+        for (int t = lane; t < d; t += 32) acc = fmaf(qv[t], v[t], acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) b.ekey[p] = make_key(float_key(acc), key_id(b.rkey[p]));
+}
+
+constexpr int kFinalThreads = 128;
+
+// One CTA per query: the best k of its rescored candidates.
+__global__ void __launch_bounds__(kFinalThreads) final_kernel(SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ SelectScratch scr;
+    const int q = blockIdx.x;
+    const int R = a.R, k = a.k;
+    uint64_t* okeys = reinterpret_cast<uint64_t*>(smem);
+    const uint64_t* ek = b.ekey + static_cast<int64_t>(q) * R;
+    auto get = [&](int i) { return ek[i]; };
+    auto pay = [&](int i) { return i; };
+    const int K = block_topk<kFinalThreads>(get, pay, b.rcount[q], k, scr, okeys, nullptr, b.err);
+    const int64_t oo = static_cast<int64_t>(q) * k;
+    for (int i = threadIdx.x; i < k; i += kFinalThreads) {
+        const bool have = i < K;
+        a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
+        a.out_scores[oo + i] = have ? key_float(key_score(okeys[i])) : -INFINITY;
+    }
+}
+
+cudaError_t launch_select(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, cudaStream_t s) {
+    size_t smem = select_smem_bytes(a.R);
+    cudaError_t e;
+    if (a.lut_mode == 0) {
+        e = cudaFuncSetAttribute(select_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        select_kernel<0><<<a.nq, kSelThreads, smem, s>>>(ix, a, b, round);
+    } else {
+        e = cudaFuncSetAttribute(select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        select_kernel<1><<<a.nq, kSelThreads, smem, s>>>(ix, a, b, round);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reorder(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    const int64_t pairs = static_cast<int64_t>(a.nq) * a.R;
+    const int64_t grid = (pairs + kReorderThreads / 32 - 1) / (kReorderThreads / 32);
+    reorder_kernel<<<static_cast<unsigned>(grid), kReorderThreads, 0, s>>>(ix, a, b);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    size_t smem = static_cast<size_t>(next_pow2(a.k)) * sizeof(uint64_t);
+    e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    final_kernel<<<a.nq, kFinalThreads, smem, s>>>(a, b);
+    return cudaGetLastError();
+}
+
+}  // namespace ah

@@ -1,0 +1,99 @@
+// Host-side launchers of the search kernels (implemented in kernels.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ah {
+
+// Queries per scan work item (leaf, query group, slot chunk).
+constexpr int kGroupF32 = 8;
+constexpr int kGroupU8 = 16;
+constexpr int kScanThreads = 256;
+constexpr int kMaxThresholdSample = 4096;   // slots scored per query for the threshold
+
+struct DeviceIndex {
+    int64_t n;
+    int d, nl, dpb, B, W;                 // W: 32-bit code words per point
+    const float* centroids;               // [NL][d]
+    const int32_t* offs;                  // [NL+1] int32 leaf offsets (owned copy)
+    const int32_t* slot_ids;              // [n]
+    const uint32_t* codes_il;             // [ceil(n/32)][W][32] (owned)
+    const float* codebook;                // [B][16][dpb]
+    const void* reorder_vecs;             // [n][d]
+    int reorder_bf16;
+};
+
+struct SearchBuffers {
+    // per query
+    float* cscore;          // [nq][NL]
+    int32_t* leaves;        // [nq][L]
+    float* leaf_scores;     // [nq][L]
+    int64_t* scanned;       // [nq]
+    float* lut_f32;         // [nq][B][16]
+    uint8_t* lut_u8;        // [nq][B][16]
+    float* lut_delta;       // [nq]
+    float* lut_bias;        // [nq]
+    uint64_t* tau;          // [nq] lower bound on the R-th best (score key, id) key
+    uint64_t* ckey;         // [nq][cap] kept candidates: (score key, id) keys
+    int32_t* cslot;         // [nq][cap] and their slots
+    int32_t* count;         // [nq]          (zeroed per search)
+    uint64_t* rkey;         // [nq][R] best R (approximate score, id) keys, descending
+    int32_t* rslot;         // [nq][R] their slots
+    int32_t* rcount;        // [nq]    how many (<= R)
+    uint64_t* ekey;         // [nq][R] (exact score, id) keys after reordering
+    int32_t* redo;          // [2][nq]       queries to rescan after rounds 0 and 1
+    int32_t* counters;      // [8]           (zeroed per search): 0 scan work, 1..2 redo list sizes,
+                            //               3..4 rescan work of rounds 1..2
+    // per leaf
+    int32_t* qcount;        // [NL]          (zeroed per search)
+    int32_t* qcursor;       // [NL]          (zeroed per search)
+    int32_t* qoff;          // [NL+1]
+    int32_t* item_off;      // [NL+1]
+    int32_t* qlist;         // [nq*L]
+    int* err;               // device error word
+    int cap;                // candidate capacity per query
+};
+
+struct SearchArgs {
+    const float* queries;
+    int nq, k, L, reorder_num, R, lut_mode, chunk;
+    int32_t* out_ids;
+    float* out_scores;
+    // optional trace outputs
+    int32_t* tr_leaf_ids;
+    float* tr_leaf_scores;
+    int32_t* tr_cand_ids;
+    float* tr_cand_scores;
+    uint32_t* tr_cand_sums;
+    int32_t* tr_ncand;
+    int64_t* tr_scanned;
+    int32_t* tr_passed;
+    int32_t* tr_rescans;
+    int scan_item_off_smem;     // set by the scan launcher
+    int topl_row_smem;          // set by the top-leaves launcher
+};
+
+// Build-time: int32 offsets and the tiled code copy.
+cudaError_t launch_prepare_index(const int64_t* offs64, int nl, int32_t* offs32, const uint8_t* codes,
+                                 int64_t n, int cb, int W, uint32_t* codes_il, cudaStream_t s);
+
+cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s);
+// round 0: all queries; rounds 1..2: the redo list of the previous round
+cudaError_t launch_select(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, cudaStream_t s);
+// exact rescoring of the kept candidates, then the best k (reorder_num > 0)
+cudaError_t launch_reorder(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round,
+                             int num_sms, cudaStream_t s);
+
+int scan_group(int lut_mode);
+size_t select_smem_bytes(int R);
+
+}  // namespace ah

@@ -1,0 +1,198 @@
+// CTA-wide selection of the K largest 64-bit keys (radix select, MSB first,
+// 8 bits per pass) and a bitonic sort of the selected keys.  Used for every
+// "keep the best N" step of the search: leaves, candidates, final neighbours.
+// Keys are distinct by construction (the low 32 bits encode the id), so the
+// K-th largest key is unique and exactly K keys are selected.
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace ah {
+
+// Shared scratch for block_select_threshold: 256 histogram bins + bookkeeping.
+struct SelectScratch {
+    int hist[256];
+    int bucket;
+    int above;
+    int count;
+    unsigned long long kand;
+    unsigned long long kor;
+};
+
+// Among the warp's 256 bins (lane l owns bins 8l..8l+7), find the bucket b where
+// the count of keys in bins above b is < need <= count in bins >= b.  Lane 0
+// writes the bucket and the count strictly above it.
+__device__ __forceinline__ void find_bucket_warp(SelectScratch& s, int need) {
+    const int lane = threadIdx.x & 31;
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) local += s.hist[lane * 8 + i];
+    // suffix sum over lanes: sum of lanes >= lane
+    int suf = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        int v = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+        if (lane + off < 32) suf += v;
+    }
+    const int above_lane = suf - local;   // keys in lanes above this one
+    const bool here = (above_lane < need) && (suf >= need);
+    if (here) {
+        int acc = above_lane;
+        for (int i = 7; i >= 0; --i) {
+            int h = s.hist[lane * 8 + i];
+            if (acc + h >= need) {
+                s.bucket = lane * 8 + i;
+                s.above = acc;
+                break;
+            }
+            acc += h;
+        }
+    }
+}
+
+// Radix select over n keys given by get(i).  On return (*prefix, *mask) define
+// the selection: key selected  <=>  (key & mask) >= prefix, which holds for
+// exactly K keys when keys are distinct.  Requires 1 <= K <= n.  All threads
+// of the block must call it; NT must be a multiple of 32.
+template <int NT, class GetKey>
+__device__ void block_select_threshold(GetKey get, int n, int K, SelectScratch& s,
+                                       uint64_t* prefix_out, uint64_t* mask_out) {
+    // Bytes every key shares carry no information: find the first byte (from
+    // the top) where keys differ with a block AND/OR reduction and start there.
+    uint64_t kand = ~0ull, kor = 0ull;
+    for (int i = threadIdx.x; i < n; i += NT) {
+        const uint64_t k = get(i);
+        kand &= k;
+        kor |= k;
+    }
+    const unsigned a_hi = __reduce_and_sync(0xFFFFFFFFu, static_cast<unsigned>(kand >> 32));
+    const unsigned a_lo = __reduce_and_sync(0xFFFFFFFFu, static_cast<unsigned>(kand));
+    const unsigned o_hi = __reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(kor >> 32));
+    const unsigned o_lo = __reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(kor));
+    if (threadIdx.x == 0) {
+        s.kand = ~0ull;
+        s.kor = 0ull;
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) {
+        atomicAnd(&s.kand, (static_cast<unsigned long long>(a_hi) << 32) | a_lo);
+        atomicOr(&s.kor, (static_cast<unsigned long long>(o_hi) << 32) | o_lo);
+    }
+    __syncthreads();
+    const uint64_t diff = s.kand ^ s.kor;
+    int shift = 56;
+    uint64_t prefix = 0, mask = 0;
+    if (diff != 0ull) {
+        const int top = 63 - __clzll(static_cast<long long>(diff));   // highest differing bit
+        shift = (top / 8) * 8;
+        mask = (shift >= 56) ? 0ull : (~0ull << (shift + 8));
+        prefix = s.kand & mask;
+    }
+    int need = K;
+    for (; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += NT) s.hist[i] = 0;
+        if (threadIdx.x == 0) {
+            s.bucket = 0;
+            s.above = 0;
+        }
+        __syncthreads();
+        // histogram; lanes of a warp that hit the same bin add once (keys of
+        // close scores share their top bits, so one bin is typically hot)
+        const int lane = threadIdx.x & 31;
+        for (int base = 0; base < n; base += NT) {
+            const int i = base + threadIdx.x;
+            bool take = false;
+            int bin = 256 + lane;                       // unique dummy for idle lanes
+            if (i < n) {
+                uint64_t k = get(i);
+                take = (k & mask) == prefix;
+                if (take) bin = static_cast<int>((k >> shift) & 255);
+            }
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (take && lane == __ffs(peers) - 1) atomicAdd(&s.hist[bin], __popc(peers));
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) find_bucket_warp(s, need);
+        __syncthreads();
+        const int b = s.bucket;
+        const int cnt_b = s.hist[b];
+        need -= s.above;
+        prefix |= static_cast<uint64_t>(b) << shift;
+        mask |= 0xFFull << shift;
+        __syncthreads();   // everyone has read bucket/above/hist before the next pass clears them
+        if (cnt_b == need) break;
+    }
+    *prefix_out = prefix;
+    *mask_out = mask;
+}
+
+// Bitonic sort (descending) of keys[0..P2) with int payloads, P2 a power of two.
+template <int NT>
+__device__ void block_sort_desc(uint64_t* keys, int32_t* vals, int P2) {
+    for (int size = 2; size <= P2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            __syncthreads();
+            for (int t = threadIdx.x; t < (P2 >> 1); t += NT) {
+                int i = 2 * t - (t & (stride - 1));
+                int j = i + stride;
+                bool desc = ((i & size) == 0);
+                uint64_t a = keys[i], b = keys[j];
+                bool swap = desc ? (a < b) : (a > b);
+                if (swap) {
+                    keys[i] = b;
+                    keys[j] = a;
+                    if (vals) {
+                        int32_t t2 = vals[i];
+                        vals[i] = vals[j];
+                        vals[j] = t2;
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+}
+
+__host__ __device__ __forceinline__ int next_pow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+// Select the K = min(K, n) largest keys of get(i) (payload pay(i)) into
+// out_keys/out_vals (shared, capacity >= next_pow2(K)), sorted descending.
+// Returns K.  Slots K..next_pow2(K)-1 hold key 0.  err is raised if more than
+// K keys qualify (duplicate keys).
+template <int NT, class GetKey, class GetVal>
+__device__ int block_topk(GetKey get, GetVal pay, int n, int K, SelectScratch& s,
+                          uint64_t* out_keys, int32_t* out_vals, int* err) {
+    if (K > n) K = n;
+    if (K <= 0) return 0;
+    uint64_t prefix = 0, mask = 0;
+    if (K < n) block_select_threshold<NT>(get, n, K, s, &prefix, &mask);
+    const int P2 = next_pow2(K);
+    for (int i = threadIdx.x; i < P2; i += NT) {
+        out_keys[i] = 0ull;
+        if (out_vals) out_vals[i] = -1;
+    }
+    if (threadIdx.x == 0) s.count = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += NT) {
+        uint64_t k = get(i);
+        if ((k & mask) >= prefix) {
+            int pos = atomicAdd(&s.count, 1);
+            if (pos < K) {
+                out_keys[pos] = k;
+                if (out_vals) out_vals[pos] = pay(i);
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && s.count != K && err) raise_error(err, kDevSelectSize);
+    block_sort_desc<NT>(out_keys, out_vals, P2);
+    return K;
+}
+
+}  // namespace ah

@@ -1,0 +1,243 @@
+"""Python binding of the C ABI in ``include/ah.h`` (ctypes; marshalling only).
+
+Every step of a search runs in the CUDA library ``_build/libah.so``; this module
+only passes device pointers, sizes and the current torch stream, and allocates
+output tensors.  There is no fallback: without the library, or without a CUDA
+device, constructing an ``Index`` raises ``AhError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_build", "libah.so")
+
+AH_OK = 0
+_STATUS = {0: "AH_OK", 1: "AH_ERR_INVALID_ARG", 2: "AH_ERR_UNSUPPORTED", 3: "AH_ERR_OOM",
+           4: "AH_ERR_CUDA", 5: "AH_ERR_DEVICE", 6: "AH_ERR_TIMEOUT"}
+AH_F32, AH_BF16 = 0, 1
+
+_lib = None
+
+
+class AhError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Views(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int64),
+        ("d", ctypes.c_int32),
+        ("num_leaves", ctypes.c_int32),
+        ("dims_per_block", ctypes.c_int32),
+        ("centroids", ctypes.c_void_p),
+        ("leaf_offsets", ctypes.c_void_p),
+        ("slot_ids", ctypes.c_void_p),
+        ("codes", ctypes.c_void_p),
+        ("codebook", ctypes.c_void_p),
+        ("reorder_vecs", ctypes.c_void_p),
+        ("reorder_dtype", ctypes.c_int32),
+    ]
+
+
+class Trace(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("leaf_ids", "leaf_scores", "cand_ids", "cand_scores", "cand_sums", "ncand", "scanned",
+                 "passed", "rescans")]
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load ``libah.so`` and declare the prototypes of ``include/ah.h``."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise AhError(4, f"CUDA library not built: {p} (run python -m mips_ivf_centroid_b200.build)")
+    lib = ctypes.CDLL(p)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    sig = {
+        "ah_build_index_views": (I32, [P, P, ctypes.POINTER(P)]),
+        "ah_search": (I32, [P, P, I32, I32, I32, I32, I32, P, P, P]),
+        "ah_search_traced": (I32, [P, P, I32, I32, I32, I32, I32, P, P, P, P]),
+        "ah_search_host": (I32, [P, P, I32, I32, I32, I32, I32, P, P, P]),
+        "ah_reserve": (I32, [P, I32, I32, I32, I32, I32]),
+        "ah_sync_status": (I32, [P, P]),
+        "ah_set_profiling": (I32, [P, I32]),
+        "ah_stage_times": (I32, [P, P, I32, P]),
+        "ah_stage_name": (ctypes.c_char_p, [I32]),
+        "ah_last_search_info": (I32, [P, P, P]),
+        "ah_index_memory": (I32, [P, P]),
+        "ah_destroy": (None, [P]),
+        "ah_status_string": (ctypes.c_char_p, [I32]),
+        "ah_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(lib, st: int):
+    if st != AH_OK:
+        raise AhError(st, lib.ah_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Index:
+    """A searchable index over borrowed device arrays.
+
+    ``arrays`` is a ``datagen.IndexArrays`` (or any object with the same
+    attributes) whose tensors live on one CUDA device; the index keeps a
+    reference to them for its lifetime.
+    """
+
+    def __init__(self, arrays, stream=None):
+        self._lib = load_library()
+        if not torch.cuda.is_available():
+            raise AhError(4, "no CUDA device")
+        self.arrays = arrays
+        c = arrays.centroids
+        dev = c.device
+        if dev.type != "cuda":
+            raise AhError(1, "index arrays must be CUDA tensors")
+        req = dict(centroids=torch.float32, leaf_offsets=torch.int64, slot_ids=torch.int32,
+                   codes=torch.uint8, codebook=torch.float32)
+        for k, dt in req.items():
+            t = getattr(arrays, k)
+            if t.dtype != dt or not t.is_contiguous() or t.device != dev:
+                raise AhError(1, f"{k}: need contiguous {dt} on {dev}")
+        rv = arrays.reorder_vecs
+        if rv is not None and (not rv.is_contiguous() or rv.device != dev or rv.dtype not in (torch.float32, torch.bfloat16)):
+            raise AhError(1, "reorder_vecs: need contiguous float32/bfloat16 on the index device")
+        self.device = dev
+        self.n = arrays.slot_ids.shape[0]
+        self.d = c.shape[1]
+        self.num_leaves = c.shape[0]
+        self.dims_per_block = arrays.codebook.shape[2]
+        v = Views(self.n, self.d, self.num_leaves, self.dims_per_block, c.data_ptr(),
+                  arrays.leaf_offsets.data_ptr(), arrays.slot_ids.data_ptr(), arrays.codes.data_ptr(),
+                  arrays.codebook.data_ptr(), rv.data_ptr() if rv is not None else None,
+                  AH_BF16 if (rv is not None and rv.dtype == torch.bfloat16) else AH_F32)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(self._lib, self._lib.ah_build_index_views(ctypes.byref(v), _stream(stream), ctypes.byref(h)))
+        self._h = h
+
+    # -- search ---------------------------------------------------------------
+    def search(self, queries: torch.Tensor, k: int, num_leaves_to_search: int, reorder_num: int,
+               lut_mode: int = 0, stream=None, trace: bool = False):
+        """(ids int32 [nq,k], scores float32 [nq,k]) on the index device.
+
+        With ``trace`` a third element holds the intermediate results (leaf ids
+        and scores, best-R candidates, points scanned per query).
+        """
+        q = queries
+        if q.device != self.device or q.dtype != torch.float32 or not q.is_contiguous() or q.dim() != 2 \
+                or q.shape[1] != self.d:
+            raise AhError(1, f"queries: need contiguous float32 [nq, {self.d}] on {self.device}")
+        nq = q.shape[0]
+        ids = torch.empty((nq, k), dtype=torch.int32, device=self.device)
+        scores = torch.empty((nq, k), dtype=torch.float32, device=self.device)
+        with torch.cuda.device(self.device):
+            s = _stream(stream)
+            if not trace:
+                _check(self._lib, self._lib.ah_search(self._h, _ptr(q), nq, k, num_leaves_to_search, reorder_num,
+                                                      lut_mode, _ptr(ids), _ptr(scores), s))
+                return ids, scores
+            R = max(reorder_num, k)
+            L = num_leaves_to_search
+            t = dict(leaf_ids=torch.empty((nq, L), dtype=torch.int32, device=self.device),
+                     leaf_scores=torch.empty((nq, L), dtype=torch.float32, device=self.device),
+                     cand_ids=torch.empty((nq, R), dtype=torch.int32, device=self.device),
+                     cand_scores=torch.empty((nq, R), dtype=torch.float32, device=self.device),
+                     cand_sums=torch.empty((nq, R), dtype=torch.int32, device=self.device),
+                     ncand=torch.empty((nq,), dtype=torch.int32, device=self.device),
+                     scanned=torch.empty((nq,), dtype=torch.int64, device=self.device),
+                     passed=torch.empty((nq,), dtype=torch.int32, device=self.device),
+                     rescans=torch.zeros((1,), dtype=torch.int32, device=self.device))
+            tr = Trace(*[t[n].data_ptr() for n, _ in Trace._fields_])
+            _check(self._lib, self._lib.ah_search_traced(self._h, _ptr(q), nq, k, num_leaves_to_search, reorder_num,
+                                                         lut_mode, _ptr(ids), _ptr(scores), ctypes.byref(tr), s))
+            return ids, scores, t
+
+    def search_host(self, queries, k: int, num_leaves_to_search: int, reorder_num: int, lut_mode: int = 0,
+                    out_ids=None, out_scores=None, stream=None):
+        """Search host queries (numpy or CPU tensor, ideally pinned); returns
+        host (ids, scores).  The copies in and out happen inside the call."""
+        if isinstance(queries, np.ndarray):
+            queries = torch.from_numpy(np.ascontiguousarray(queries, dtype=np.float32))
+        if queries.device.type != "cpu" or queries.dtype != torch.float32 or not queries.is_contiguous():
+            raise AhError(1, "queries: need a contiguous float32 host tensor")
+        nq = queries.shape[0]
+        if out_ids is None:
+            out_ids = torch.empty((nq, k), dtype=torch.int32, pin_memory=queries.is_pinned())
+        if out_scores is None:
+            out_scores = torch.empty((nq, k), dtype=torch.float32, pin_memory=queries.is_pinned())
+        with torch.cuda.device(self.device):
+            _check(self._lib, self._lib.ah_search_host(self._h, _ptr(queries), nq, k, num_leaves_to_search,
+                                                       reorder_num, lut_mode, _ptr(out_ids), _ptr(out_scores),
+                                                       _stream(stream)))
+        return out_ids, out_scores
+
+    def reserve(self, max_nq: int, k: int, num_leaves_to_search: int, reorder_num: int, lut_mode: int = 0):
+        with torch.cuda.device(self.device):
+            _check(self._lib, self._lib.ah_reserve(self._h, max_nq, k, num_leaves_to_search, reorder_num, lut_mode))
+
+    def sync_status(self, stream=None):
+        with torch.cuda.device(self.device):
+            _check(self._lib, self._lib.ah_sync_status(self._h, _stream(stream)))
+
+    # -- instrumentation ------------------------------------------------------
+    def set_profiling(self, on: bool = True):
+        _check(self._lib, self._lib.ah_set_profiling(self._h, 1 if on else 0))
+
+    def stage_times(self) -> dict:
+        ms = (ctypes.c_float * 16)()
+        n = ctypes.c_int32()
+        _check(self._lib, self._lib.ah_stage_times(self._h, ms, 16, ctypes.byref(n)))
+        return {self._lib.ah_stage_name(i).decode(): float(ms[i]) for i in range(n.value)}
+
+    def last_search_info(self, points_scanned: bool = False) -> dict:
+        launches = ctypes.c_int32()
+        pts = ctypes.c_int64()
+        _check(self._lib, self._lib.ah_last_search_info(self._h, ctypes.byref(launches),
+                                                        ctypes.byref(pts) if points_scanned else None))
+        out = {"launches": launches.value}
+        if points_scanned:
+            out["points_scanned"] = pts.value
+        return out
+
+    def memory_bytes(self) -> int:
+        b = ctypes.c_int64()
+        _check(self._lib, self._lib.ah_index_memory(self._h, ctypes.byref(b)))
+        return b.value
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.ah_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
