@@ -217,6 +217,34 @@ AH_API ah_status ah_last_search_info(ah_index *ix, int32_t *launches, int64_t *p
 /* Device bytes owned by the index (derived state + workspace). */
 AH_API ah_status ah_index_memory(ah_index *ix, int64_t *bytes);
 
+/*
+ * Partition stage without any device allocation (no counterpart in the
+ * paper: it exists for callers that cannot allocate).  Some callers must not
+ * allocate device memory on the call path: a serving process whose device
+ * memory is reserved up front by another allocator, or a latency-critical
+ * loop that cannot afford cudaMalloc's implicit device synchronisation.  For
+ * them this call scores the queries against every centroid and keeps the best
+ * num_leaves_to_search leaves, the first stage of ah_search, using a scratch
+ * area that lives in the library itself: a device array of
+ * AH_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits.
+ *   queries          float [nq][d], device
+ *   out_leaf_ids     int32 [nq][num_leaves_to_search], device
+ *   out_leaf_scores  float [nq][num_leaves_to_search], device (fp32 q . c)
+ * The scratch must hold nq * num_leaves scores plus small counters; larger
+ * batches are rejected with AH_ERR_UNSUPPORTED before anything is enqueued
+ * (split the batch).  The index's device must be current.  The first call on
+ * a device looks up the scratch array's device address (a runtime query, no
+ * allocation); make that first call before any stream capture.  All calls
+ * share the one scratch area: calls whose work overlaps on the GPU (different
+ * streams, or different indexes on one device) race and must be serialised by
+ * the caller.  Results equal the leaves ah_search_traced reports.
+ */
+#define AH_NOALLOC_SCRATCH_BYTES (8u << 20)
+AH_API ah_status ah_search_leaves_noalloc(ah_index *ix, const float *queries, int32_t nq,
+                                          int32_t num_leaves_to_search, int32_t *out_leaf_ids,
+                                          float *out_leaf_scores, void *cuda_stream);
+
 /* Release everything the index owns.  Does not touch the borrowed views. */
 AH_API void ah_destroy(ah_index *ix);
 

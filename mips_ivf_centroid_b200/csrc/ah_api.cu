@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -488,6 +489,78 @@ void ah_destroy(ah_index* ix) {
     if (ix->ev_ready)
         for (int i = 0; i <= kStages; ++i) cudaEventDestroy(ix->ev[i]);
     delete ix;
+}
+
+// Scratch of ah_search_leaves_noalloc: the centroid score matrix and the
+// per-leaf counters of the partition stage, in a file-scope device array so
+// that the call never allocates.  Host code must not take this symbol's
+// address directly (on the host it is only a stand-in); the device address is
+// looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[AH_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (first call per
+// device does the lookup).
+ah_status noalloc_scratch(int device, void** out) {
+    if (device < 0 || device >= kMaxDevices) return fail(AH_ERR_UNSUPPORTED, "device ordinal beyond the scratch table");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_dev_ptr[device]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "scratch address lookup");
+        g_noalloc_dev_ptr[device] = p;
+    }
+    *out = g_noalloc_dev_ptr[device];
+    return AH_OK;
+}
+}  // namespace
+
+ah_status ah_search_leaves_noalloc(ah_index* ix, const float* queries, int32_t nq, int32_t L,
+                                   int32_t* out_leaf_ids, float* out_leaf_scores, void* cuda_stream) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    if (nq < 0) return fail(AH_ERR_INVALID_ARG, "nq < 0");
+    if (L < 1 || L > ix->dix.nl) return fail(AH_ERR_INVALID_ARG, "num_leaves_to_search outside [1, num_leaves]");
+    if (L > AH_MAX_LEAVES_SEARCHED) return fail(AH_ERR_UNSUPPORTED, "num_leaves_to_search above AH_MAX_LEAVES_SEARCHED");
+    if (nq == 0) return AH_OK;
+    if (!queries || !out_leaf_ids || !out_leaf_scores) return fail(AH_ERR_INVALID_ARG, "NULL queries or outputs");
+    const int NL = ix->dix.nl;
+    const size_t score_bytes = align_up(sizeof(float) * (size_t)nq * NL, 256);
+    const size_t count_bytes = align_up(sizeof(int32_t) * (size_t)NL, 256);
+    const size_t scanned_bytes = align_up(sizeof(int64_t) * (size_t)nq, 256);
+    if (score_bytes + count_bytes + scanned_bytes > AH_NOALLOC_SCRATCH_BYTES)
+        return fail(AH_ERR_UNSUPPORTED, "nq * num_leaves scores exceed the library's fixed scratch "
+                                        "(AH_NOALLOC_SCRATCH_BYTES); split the batch");
+    int device = -1;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (device != ix->device) return fail(AH_ERR_INVALID_ARG, "the index's device is not current");
+    void* base = nullptr;
+    ah_status st = noalloc_scratch(device, &base);
+    if (st != AH_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    char* p = static_cast<char*>(base);
+    ah::SearchBuffers b{};
+    b.cscore = reinterpret_cast<float*>(p);
+    b.qcount = reinterpret_cast<int32_t*>(p + score_bytes);
+    b.scanned = reinterpret_cast<int64_t*>(p + score_bytes + count_bytes);
+    b.leaves = out_leaf_ids;
+    b.leaf_scores = out_leaf_scores;
+    b.err = ix->err;
+    ah::SearchArgs a{};
+    a.queries = queries;
+    a.nq = nq;
+    a.L = L;
+    a.k = 1;
+    a.R = 1;
+    // the per-leaf counters are accumulated by the top-L kernel: start them at zero
+    if ((e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)NL, s)) != cudaSuccess) return cuda_fail(e, "memset");
+    if ((e = ah::launch_centroid_scores(ix->dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "centroid scores");
+    if ((e = ah::launch_top_leaves(ix->dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
+    return AH_OK;
 }
 
 }  // extern "C"

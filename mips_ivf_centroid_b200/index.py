@@ -78,6 +78,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_destroy": (None, [P]),
         "ah_status_string": (ctypes.c_char_p, [I32]),
         "ah_last_error": (ctypes.c_char_p, []),
+        "ah_search_leaves_noalloc": (I32, [P, P, I32, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -230,6 +231,16 @@ class Index:
         b = ctypes.c_int64()
         _check(self._lib, self._lib.ah_index_memory(self._h, ctypes.byref(b)))
         return b.value
+
+    def search_leaves_noalloc(self, queries: torch.Tensor, num_leaves_to_search: int, out_leaf_ids: torch.Tensor,
+                              out_leaf_scores: torch.Tensor, stream=None):
+        """Partition stage into caller-provided outputs, with no device
+        allocation anywhere on the call path (see ah_search_leaves_noalloc in
+        include/ah.h for the scratch limit and the sharing rules)."""
+        with torch.cuda.device(self.device):
+            _check(self._lib, self._lib.ah_search_leaves_noalloc(
+                self._h, _ptr(queries), queries.shape[0], num_leaves_to_search, _ptr(out_leaf_ids),
+                _ptr(out_leaf_scores), _stream(stream)))
 
     def close(self):
         if getattr(self, "_h", None):
