@@ -31,9 +31,9 @@ ah_status cuda_fail(cudaError_t e, const char* what) {
     return e == cudaErrorMemoryAllocation ? AH_ERR_OOM : AH_ERR_CUDA;
 }
 
-constexpr int kStages = 9;
+constexpr int kStages = 8;
 const char* kStageNames[kStages] = {"centroid_scores", "top_leaves", "invert", "lut",
-                                    "threshold", "scan", "select", "rescan", "reorder"};
+                                    "threshold", "scan", "finish", "rescan"};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -60,6 +60,7 @@ struct ah_index {
     int device = 0;
     int num_sms = 0;
     int32_t* offs32 = nullptr;
+    int32_t* ptile = nullptr;
     uint32_t* codes_il = nullptr;
     int* err = nullptr;
     size_t owned_bytes = 0;
@@ -108,10 +109,6 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     add(stage ? sizeof(int32_t) * (size_t)cnq * ck : 0);        // 16 dids
     add(stage ? sizeof(float) * (size_t)cnq * ck : 0);          // 17 dscores
     add(sizeof(int32_t) * (size_t)cnq * cap);                   // 18 candidate slots
-    add(sizeof(uint64_t) * (size_t)cnq * cR);                   // 19 rkey
-    add(sizeof(int32_t) * (size_t)cnq * cR);                    // 20 rslot
-    add(sizeof(int32_t) * (size_t)cnq);                         // 21 rcount
-    add(sizeof(uint64_t) * (size_t)cnq * cR);                   // 22 ekey
     size_t total = 0;
     for (int i = 0; i < n; ++i) total += sz[i];
     if (w.base) {
@@ -146,10 +143,6 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     b.tau = reinterpret_cast<uint64_t*>(part[8]);
     b.ckey = reinterpret_cast<uint64_t*>(part[9]);
     b.cslot = reinterpret_cast<int32_t*>(part[18]);
-    b.rkey = reinterpret_cast<uint64_t*>(part[19]);
-    b.rslot = reinterpret_cast<int32_t*>(part[20]);
-    b.rcount = reinterpret_cast<int32_t*>(part[21]);
-    b.ekey = reinterpret_cast<uint64_t*>(part[22]);
     int32_t* zr = reinterpret_cast<int32_t*>(part[10]);
     b.qcount = zr;
     b.qcursor = zr + NL;
@@ -207,7 +200,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     a.reorder_num = reorder_num;
     a.R = R;
     a.lut_mode = lut_mode;
-    a.chunk = nq >= 64 ? 1024 : 256;
+    a.chunk = nq >= 64 ? 32 : 8;          // code tiles per scan work item
     a.out_ids = out_ids;
     a.out_scores = out_scores;
     if (tr) {
@@ -249,20 +242,15 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
     launches += 1;
     mark(6);
-    if ((e = ah::launch_select(dix, a, b, 0, s)) != cudaSuccess) return cuda_fail(e, "select");
+    if ((e = ah::launch_finish(dix, a, b, 0, s)) != cudaSuccess) return cuda_fail(e, "finish");
     launches += 1;
     mark(7);
     for (int round = 1; round <= 2; ++round) {
         if ((e = ah::launch_redo_scan(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "rescan");
-        if ((e = ah::launch_select(dix, a, b, round, s)) != cudaSuccess) return cuda_fail(e, "select after rescan");
+        if ((e = ah::launch_finish(dix, a, b, round, s)) != cudaSuccess) return cuda_fail(e, "finish after rescan");
         launches += 2;
     }
     mark(8);
-    if (reorder_num > 0) {
-        if ((e = ah::launch_reorder(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "reorder");
-        launches += 2;
-    }
-    mark(9);
     if (prof) ix->ev_recorded = true;
     if (tr) {
         const size_t nL = (size_t)nq * L;
@@ -327,19 +315,47 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
     const int B = v->d / v->dims_per_block;
     const int cb = B / 2;
     const int W = (cb + 3) / 4;
-    const int64_t tiles = (v->n + 31) / 32;
-    const size_t il_bytes = (size_t)tiles * W * 32 * sizeof(uint32_t);
-    const size_t offs_bytes = sizeof(int32_t) * (size_t)(v->num_leaves + 1);
+    const int NL = v->num_leaves;
+    // leaf offsets: validated on the host, then int32 offsets and the first
+    // code tile of each leaf in the leaf-padded code copy
+    std::vector<int64_t> o64(NL + 1);
+    if ((e = cudaMemcpy(o64.data(), v->leaf_offsets, sizeof(int64_t) * (NL + 1), cudaMemcpyDeviceToHost)) != cudaSuccess) {
+        delete ix;
+        return cuda_fail(e, "leaf offsets read");
+    }
+    std::vector<int32_t> o32(NL + 1), pt(NL + 1);
+    if (o64[0] != 0 || o64[NL] != v->n) {
+        delete ix;
+        return fail(AH_ERR_INVALID_ARG, "leaf_offsets must start at 0 and end at n");
+    }
+    int64_t tiles = 0;
+    for (int c = 0; c <= NL; ++c) {
+        if (c < NL && o64[c + 1] < o64[c]) {
+            delete ix;
+            return fail(AH_ERR_INVALID_ARG, "leaf_offsets must be non-decreasing");
+        }
+        o32[c] = static_cast<int32_t>(o64[c]);
+        pt[c] = static_cast<int32_t>(tiles);
+        if (c < NL) tiles += (o64[c + 1] - o64[c] + 31) / 32;
+    }
+    if (tiles * 32 >= (int64_t(1) << 31)) {
+        delete ix;
+        return fail(AH_ERR_UNSUPPORTED, "padded code copy beyond 2^31 slots");
+    }
+    const size_t il_bytes = (size_t)std::max<int64_t>(tiles, 1) * W * 32 * sizeof(uint32_t);
+    const size_t offs_bytes = sizeof(int32_t) * (size_t)(NL + 1);
     if ((e = cudaMalloc(&ix->codes_il, il_bytes)) != cudaSuccess ||
         (e = cudaMalloc(&ix->offs32, offs_bytes)) != cudaSuccess ||
+        (e = cudaMalloc(&ix->ptile, offs_bytes)) != cudaSuccess ||
         (e = cudaMalloc(&ix->err, sizeof(int))) != cudaSuccess) {
         ah_destroy(ix);
         return cuda_fail(e, "index allocation");
     }
-    ix->owned_bytes = il_bytes + offs_bytes + sizeof(int);
-    if ((e = cudaMemsetAsync(ix->err, 0, sizeof(int), s)) != cudaSuccess ||
-        (e = ah::launch_prepare_index(v->leaf_offsets, v->num_leaves, ix->offs32, v->codes, v->n, cb, W, ix->codes_il, s)) !=
-            cudaSuccess ||
+    ix->owned_bytes = il_bytes + 2 * offs_bytes + sizeof(int);
+    if ((e = cudaMemcpy(ix->offs32, o32.data(), offs_bytes, cudaMemcpyHostToDevice)) != cudaSuccess ||
+        (e = cudaMemcpy(ix->ptile, pt.data(), offs_bytes, cudaMemcpyHostToDevice)) != cudaSuccess ||
+        (e = cudaMemsetAsync(ix->err, 0, sizeof(int), s)) != cudaSuccess ||
+        (e = ah::launch_prepare_index(ix->offs32, ix->ptile, NL, v->codes, cb, W, tiles, ix->codes_il, s)) != cudaSuccess ||
         (e = cudaStreamSynchronize(s)) != cudaSuccess) {
         ah_destroy(ix);
         return cuda_fail(e, "index preparation");
@@ -353,6 +369,7 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
     d.W = W;
     d.centroids = v->centroids;
     d.offs = ix->offs32;
+    d.ptile = ix->ptile;
     d.slot_ids = v->slot_ids;
     d.codes_il = ix->codes_il;
     d.codebook = v->codebook;
@@ -485,6 +502,7 @@ void ah_destroy(ah_index* ix) {
     if (ix->ws.base) cudaFree(ix->ws.base);
     if (ix->codes_il) cudaFree(ix->codes_il);
     if (ix->offs32) cudaFree(ix->offs32);
+    if (ix->ptile) cudaFree(ix->ptile);
     if (ix->err) cudaFree(ix->err);
     if (ix->ev_ready)
         for (int i = 0; i <= kStages; ++i) cudaEventDestroy(ix->ev[i]);

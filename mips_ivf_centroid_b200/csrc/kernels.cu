@@ -30,24 +30,27 @@ namespace ah {
 // index preparation
 // ---------------------------------------------------------------------------
 
-__global__ void offsets_to_i32_kernel(const int64_t* __restrict__ o64, int nl, int32_t* __restrict__ o32) {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i <= nl) o32[i] = static_cast<int32_t>(o64[i]);
-}
-
-// codes [n][cb] bytes -> il[tile][w][lane] 32-bit words (slot = 32*tile + lane,
-// word w holds code bytes 4w..4w+3; bytes past cb and slots past n are 0).
-__global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, int64_t n, int cb, int W,
+// codes [n][cb] bytes -> il[tile][w][lane] 32-bit words.  Tiles are padded
+// per leaf: leaf c owns tiles ptile[c] .. ptile[c+1]-1, and lane l of its tile
+// t holds slot offs[c] + 32 (t - ptile[c]) + l (zero codes past the leaf's
+// end).  Word w holds code bytes 4w..4w+3.
+__global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, const int32_t* __restrict__ offs,
+                                        const int32_t* __restrict__ ptile, int nl, int cb, int W,
                                         uint32_t* __restrict__ il, int64_t total_words) {
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e >= total_words) return;
-    int lane = static_cast<int>(e & 31);
-    int64_t tw = e >> 5;                 // tile*W + w
-    int w = static_cast<int>(tw % W);
-    int64_t tile = tw / W;
-    int64_t slot = tile * 32 + lane;
+    const int lane = static_cast<int>(e & 31);
+    const int64_t tw = e >> 5;                 // tile*W + w
+    const int w = static_cast<int>(tw % W);
+    const int tile = static_cast<int>(tw / W);
+    int lo = 0, hi = nl - 1;                   // leaf owning the tile: last c with ptile[c] <= tile
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (ptile[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int64_t slot = static_cast<int64_t>(offs[lo]) + 32ll * (tile - ptile[lo]) + lane;
     uint32_t v = 0;
-    if (slot < n) {
+    if (slot < offs[lo + 1]) {
         const uint8_t* row = codes + slot * cb;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -58,13 +61,12 @@ __global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, int64
     il[e] = v;
 }
 
-cudaError_t launch_prepare_index(const int64_t* offs64, int nl, int32_t* offs32, const uint8_t* codes,
-                                 int64_t n, int cb, int W, uint32_t* codes_il, cudaStream_t s) {
-    offsets_to_i32_kernel<<<(nl + 1 + 255) / 256, 256, 0, s>>>(offs64, nl, offs32);
-    int64_t tiles = (n + 31) / 32;
-    int64_t total = tiles * W * 32;
-    int64_t grid = (total + 255) / 256;
-    interleave_codes_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, n, cb, W, codes_il, total);
+cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, int nl, const uint8_t* codes, int cb,
+                                 int W, int64_t ntiles, uint32_t* codes_il, cudaStream_t s) {
+    const int64_t total = ntiles * W * 32;
+    if (total == 0) return cudaSuccess;
+    const int64_t grid = (total + 255) / 256;
+    interleave_codes_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, offs32, ptile, nl, cb, W, codes_il, total);
     return cudaGetLastError();
 }
 
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix,
     if (threadIdx.x == 0) b.scanned[q] = s_scanned;
 }
 
-cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+static cudaError_t launch_top_leaves_block(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
     size_t smem = static_cast<size_t>(next_pow2(a.L)) * sizeof(uint64_t);
     const size_t row = static_cast<size_t>(ix.nl) * sizeof(float);
     a.topl_row_smem = (row <= 64 * 1024) ? 1 : 0;
@@ -176,6 +178,12 @@ cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchB
     if (e != cudaSuccess) return e;
     top_leaves_kernel<<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
     return cudaGetLastError();
+}
+
+constexpr int kWarpMaxK = 256;          // warp-cooperative selection up to this K
+
+cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+    return launch_top_leaves_block(ix, a, b, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -212,7 +220,7 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, 
 }
 
 // Single CTA: qoff = exclusive scan of queries per leaf; item_off = exclusive
-// scan of work items per leaf (query groups x slot chunks).
+// scan of work items per leaf (query groups x chunks of `chunk` code tiles).
 __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex ix, SearchBuffers b, int group, int chunk) {
     __shared__ int warp_sums[32];
     __shared__ int total_q, total_i;
@@ -222,8 +230,8 @@ __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex 
         int qc = 0, it = 0;
         if (c < ix.nl) {
             qc = b.qcount[c];
-            int sz = ix.offs[c + 1] - ix.offs[c];
-            it = (qc > 0 && sz > 0) ? ((qc + group - 1) / group) * ((sz + chunk - 1) / chunk) : 0;
+            int tiles = ix.ptile[c + 1] - ix.ptile[c];
+            it = (qc > 0 && tiles > 0) ? ((qc + group - 1) / group) * ((tiles + chunk - 1) / chunk) : 0;
         }
         int eq = block_exclusive_scan_1024(qc, warp_sums, &total_q);
         int ei = block_exclusive_scan_1024(it, warp_sums, &total_i);
@@ -339,10 +347,11 @@ cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchB
 
 // fp32: table in shared memory as [B][16] floats; returns the score key.
 // uint8: table as [B][16] bytes; returns the integer sum.
+// `pos` is the slot's position in the leaf-padded code copy.
 template <int MODE>
 __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int B,
-                                               const unsigned char* lut, int32_t slot) {
-    const uint32_t* cw = codes_il + (static_cast<int64_t>(slot >> 5) * W) * 32 + (slot & 31);
+                                               const unsigned char* lut, int32_t pos) {
+    const uint32_t* cw = codes_il + (static_cast<int64_t>(pos >> 5) * W) * 32 + (pos & 31);
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
         float acc = 0.0f;
@@ -367,12 +376,12 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
 // still runs over blocks in order, identical to slot_value.
 template <int MODE>
 __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int B,
-                                             const unsigned char* lut, const int32_t* slot, const bool* valid,
+                                             const unsigned char* lut, const int32_t* pos, const bool* valid,
                                              uint32_t* out) {
     const uint32_t* cw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        const int32_t sl = valid[u] ? slot[u] : 0;
+        const int32_t sl = valid[u] ? pos[u] : 0;
         cw[u] = codes_il + (static_cast<int64_t>(sl >> 5) * W) * 32 + (sl & 31);
     }
     if (MODE == 0) {
@@ -435,6 +444,11 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 // threshold: R-th best approximate score over a prefix of the best leaves
 // ---------------------------------------------------------------------------
 
+// Slots sampled per query for the bound.
+__host__ __device__ __forceinline__ int threshold_sample(int R) {
+    return min(kMaxThresholdSample, max(R, 1024));
+}
+
 // One CTA per query.  Scores the first M = min(points, max(R, 1024)) slots of
 // the query's leaves in rank order; the R-th largest (score, id) key among them
 // is a lower bound on the R-th largest over all its leaves (a subset's R-th
@@ -448,30 +462,31 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, 
     const int R = a.R;
     unsigned char* lut = smem;
     uint64_t* vals = reinterpret_cast<uint64_t*>(smem + ((table_bytes(MODE, ix.B) + 15) & ~15));
-    uint64_t* top = vals + kMaxThresholdSample;
+    uint64_t* top = nullptr;
     load_query_table<MODE>(ix, b, q, lut);
     __syncthreads();
-    const int M = min(kMaxThresholdSample, max(R, 1024));
+    const int M = threshold_sample(R);
     int taken = 0;
     for (int i = 0; i < a.L && taken < M; ++i) {
         int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
         int s0 = ix.offs[leaf], sz = ix.offs[leaf + 1] - s0;
+        int p0 = ix.ptile[leaf] * 32;
         int m = min(sz, M - taken);
         for (int t0 = 0; t0 < m; t0 += 4 * kSelThreads) {
-            int32_t sl[4];
+            int32_t ps[4];
             bool ok[4];
             uint32_t v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int t = t0 + u * kSelThreads + threadIdx.x;
                 ok[u] = t < m;
-                sl[u] = s0 + t;
+                ps[u] = p0 + t;
             }
-            slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, sl, ok, v);
+            slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, v);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int t = t0 + u * kSelThreads + threadIdx.x;
-                if (ok[u]) vals[taken + t] = make_key(v[u], ix.slot_ids[sl[u]]);
+                if (ok[u]) vals[taken + t] = make_key(v[u], ix.slot_ids[s0 + t]);
             }
         }
         taken += m;
@@ -480,17 +495,15 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, 
     uint64_t tau = 0ull;
     if (taken >= R) {
         auto get = [&](int i) { return vals[i]; };
-        auto pay = [&](int i) { return i; };
-        block_topk<kSelThreads>(get, pay, taken, R, scr, top, nullptr, b.err);
-        tau = top[R - 1];
+        tau = block_kth_largest<kSelThreads>(get, taken, R, scr);
     }
     if (threadIdx.x == 0) b.tau[q] = tau;
+    (void)top;
 }
 
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
-    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + kMaxThresholdSample * sizeof(uint64_t) +
-                  static_cast<size_t>(next_pow2(a.R)) * sizeof(uint64_t);
     cudaError_t e;
+    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + static_cast<size_t>(threshold_sample(a.R)) * sizeof(uint64_t);
     if (a.lut_mode == 0) {
         e = cudaFuncSetAttribute(threshold_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
@@ -536,29 +549,178 @@ __device__ __forceinline__ void append_candidates(bool pass, uint32_t key, int32
     }
 }
 
-// Persistent CTAs take work items (leaf, query group of G, chunk of slots) from
-// an atomic counter.  Per item the group's tables are staged in shared memory:
-//   fp32: [b][G/2][16][2] floats: one 8-byte load fetches query pair
-//         (2p, 2p+1)'s entries for center j; a (block, pair) table is 128 B.
-//   u8:   [b][G/4][16][4] bytes: one 4-byte load fetches 4 queries' entries.
-// Each lane owns one slot of a 32-slot tile and walks its code words; per
-// nibble it issues G/2 (fp32) or G/4 (u8) shared loads.  Sums run over blocks
-// in order 0..B-1 with IEEE fp32 adds (two lanes per packed f32x2 add), the
-// same order as the query-major kernels, so a slot's score is bit-identical
-// in every kernel.
-template <int G, int MODE>
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+// One code word (8 blocks) for a group of G queries, fp32 tables staged as
+// [b][G/2][16] float2: per nibble one 8-byte shared load per query pair, one
+// packed add.  `base` points at block 8w's tables.
+template <int G>
+__device__ __forceinline__ void f32_word(uint32_t c, const float2* __restrict__ base, float2 (&acc)[G / 2]) {
+    constexpr int BS = (G / 2) * kCenters;   // float2 per block
+#pragma unroll
+    for (int nib = 0; nib < 8; ++nib) {
+        const float2* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
+#pragma unroll
+        for (int pr = 0; pr < G / 2; ++pr) acc[pr] = __fadd2_rn(acc[pr], p[pr * kCenters]);
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void f32_tail(uint32_t c, int nb, const float2* __restrict__ base, float2 (&acc)[G / 2]) {
+    constexpr int BS = (G / 2) * kCenters;
+    for (int nib = 0; nib < nb; ++nib) {
+        const float2* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
+#pragma unroll
+        for (int pr = 0; pr < G / 2; ++pr) acc[pr] = __fadd2_rn(acc[pr], p[pr * kCenters]);
+    }
+}
+
+// uint8 tables staged as [b][G/4][16] words (4 queries' bytes per word); two
+// 16-bit lanes per accumulator (queries 4d+0/4d+2 in ae, 4d+1/4d+3 in ao).
+template <int G>
+__device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, const uint32_t* __restrict__ base, uint32_t (&ae)[G / 4],
+                                           uint32_t (&ao)[G / 4]) {
+    constexpr int BS = (G / 4) * kCenters;   // words per block
+#pragma unroll
+    for (int nib = 0; nib < 8; ++nib) {
+        if (nib < nb) {
+            const uint32_t* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
+#pragma unroll
+            for (int qd = 0; qd < G / 4; ++qd) {
+                const uint32_t v = p[qd * kCenters];
+                ae[qd] += v & 0x00FF00FFu;
+                ao[qd] += __byte_perm(v, 0u, 0x4341);
+            }
+        }
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void u8_flush(uint32_t (&sums)[G], uint32_t (&ae)[G / 4], uint32_t (&ao)[G / 4]) {
+#pragma unroll
+    for (int qd = 0; qd < G / 4; ++qd) {
+        sums[4 * qd + 0] += ae[qd] & 0xFFFFu;
+        sums[4 * qd + 2] += ae[qd] >> 16;
+        sums[4 * qd + 1] += ao[qd] & 0xFFFFu;
+        sums[4 * qd + 3] += ao[qd] >> 16;
+        ae[qd] = 0u;
+        ao[qd] = 0u;
+    }
+}
+
+struct TileJob {
+    int t0, t1;          // code tiles [t0, t1) of one leaf
+    int slot_base;       // slot of lane 0 of tile t is slot_base + 32 t
+    int send;            // first slot past the leaf
+    int gsize;           // real queries in the group (<= G)
+};
+
+// The warps of a CTA split the item's tiles; a lane owns one slot.  Blocks are
+// summed in order 0..B-1 with IEEE fp32 adds (two queries per packed add), the
+// order every kernel that scores a slot uses.
+template <int G>
+__device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
+                                               const TileJob& job, const int* s_q, const uint32_t* s_th,
+                                               const uint32_t* s_tl) {
+    constexpr int BS = (G / 2) * kCenters;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
+    const float2* lut2 = reinterpret_cast<const float2*>(smem);
+    for (int t = job.t0 + warp; t < job.t1; t += kScanThreads / 32) {
+        const int slot = job.slot_base + 32 * t + lane;
+        const bool valid = slot < job.send;
+        const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
+        float2 acc[G / 2];
+#pragma unroll
+        for (int pr = 0; pr < G / 2; ++pr) acc[pr] = make_float2(0.0f, 0.0f);
+        int w = 0;
+        for (; w + 4 <= Wf; w += 4) {
+            const uint32_t c0 = cwp[(w + 0) * 32], c1 = cwp[(w + 1) * 32];
+            const uint32_t c2 = cwp[(w + 2) * 32], c3 = cwp[(w + 3) * 32];
+            f32_word<G>(c0, lut2 + (8 * w + 0) * BS, acc);
+            f32_word<G>(c1, lut2 + (8 * w + 8) * BS, acc);
+            f32_word<G>(c2, lut2 + (8 * w + 16) * BS, acc);
+            f32_word<G>(c3, lut2 + (8 * w + 24) * BS, acc);
+        }
+        for (; w < Wf; ++w) f32_word<G>(cwp[w * 32], lut2 + 8 * w * BS, acc);
+        if (tail) f32_tail<G>(cwp[Wf * 32], tail, lut2 + 8 * Wf * BS, acc);
+#pragma unroll
+        for (int qi = 0; qi < G; ++qi) {
+            if (qi < job.gsize) {
+                const float sc = (qi & 1) ? acc[qi >> 1].y : acc[qi >> 1].x;
+                const uint32_t key = float_key(sc);
+                append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot, s_q[qi], ix, b);
+            }
+        }
+    }
+}
+
+template <int G>
+__device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
+                                              const TileJob& job, const int* s_q, const uint32_t* s_th,
+                                              const uint32_t* s_tl) {
+    constexpr int BS = (G / 4) * kCenters;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
+    const uint32_t* lutw = reinterpret_cast<const uint32_t*>(smem);
+    for (int t = job.t0 + warp; t < job.t1; t += kScanThreads / 32) {
+        const int slot = job.slot_base + 32 * t + lane;
+        const bool valid = slot < job.send;
+        const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
+        uint32_t sums[G];
+        uint32_t ae[G / 4], ao[G / 4];
+#pragma unroll
+        for (int qi = 0; qi < G; ++qi) sums[qi] = 0u;
+#pragma unroll
+        for (int qd = 0; qd < G / 4; ++qd) { ae[qd] = 0u; ao[qd] = 0u; }
+        // 16-bit lanes hold 256 blocks of 255: flush every 32 words
+        for (int w0 = 0; w0 < Wf; w0 += 32) {
+            const int wend = min(Wf, w0 + 32);
+            int w = w0;
+            for (; w + 4 <= wend; w += 4) {
+                const uint32_t c0 = cwp[(w + 0) * 32], c1 = cwp[(w + 1) * 32];
+                const uint32_t c2 = cwp[(w + 2) * 32], c3 = cwp[(w + 3) * 32];
+                u8_nibbles<G>(c0, 8, lutw + (8 * w + 0) * BS, ae, ao);
+                u8_nibbles<G>(c1, 8, lutw + (8 * w + 8) * BS, ae, ao);
+                u8_nibbles<G>(c2, 8, lutw + (8 * w + 16) * BS, ae, ao);
+                u8_nibbles<G>(c3, 8, lutw + (8 * w + 24) * BS, ae, ao);
+            }
+            for (; w < wend; ++w) u8_nibbles<G>(cwp[w * 32], 8, lutw + 8 * w * BS, ae, ao);
+            u8_flush<G>(sums, ae, ao);
+        }
+        if (tail) {
+            u8_nibbles<G>(cwp[Wf * 32], tail, lutw + 8 * Wf * BS, ae, ao);
+            u8_flush<G>(sums, ae, ao);
+        }
+#pragma unroll
+        for (int qi = 0; qi < G; ++qi) {
+            if (qi < job.gsize)
+                append_candidates(valid && reaches(sums[qi], s_th[qi], s_tl[qi], ix.slot_ids, slot), sums[qi], slot,
+                                  s_q[qi], ix, b);
+        }
+    }
+}
+
+// Persistent CTAs take work items (leaf, query group, chunk of code tiles) from
+// an atomic counter.  A leaf's m queries form groups of GMAX, then one group of
+// the remainder rounded up to GSTEP, so at most GSTEP-1 table slots of a leaf
+// are padding.  Per item the group's tables are staged in shared memory
+// (fp32 pair-interleaved, uint8 quad-interleaved) and the warps scan the
+// chunk's tiles.  Only a leaf's last tile is partial (leaf-padded code copy).
+#ifndef AH_SCAN_MIN_BLOCKS
+#define AH_SCAN_MIN_BLOCKS 6
+#endif
+
+template <int MODE>
+__global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(DeviceIndex ix, SearchArgs a,
+                                                                                 SearchBuffers b) {
+    constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
+    constexpr int GSTEP = (MODE == 0) ? 2 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_item, s_leaf;
-    __shared__ int s_q[G];
-    __shared__ uint32_t s_th[G], s_tl[G];
-    const int B = ix.B, W = ix.W;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int NW = kScanThreads / 32;
+    __shared__ int s_q[GMAX];
+    __shared__ uint32_t s_th[GMAX], s_tl[GMAX];
+    const int B = ix.B;
     const int total_items = b.item_off[ix.nl];
-    const int blk_bytes = (MODE == 0) ? G * 64 : G * 16;     // one block's tables for the group
-    // work-item offsets per leaf, copied once per CTA when they fit
-    const size_t lut_bytes = static_cast<size_t>(B) * blk_bytes;
+    const size_t lut_bytes = static_cast<size_t>(B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
     int* s_item_off = reinterpret_cast<int*>(smem + lut_bytes);
     const bool off_in_smem = a.scan_item_off_smem != 0;
     if (off_in_smem)
@@ -583,16 +745,20 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(DeviceIndex ix, Sear
         const int item = s_item;
         if (item >= total_items) break;
         const int leaf = s_leaf;
-        const int off0 = ix.offs[leaf], nslots = ix.offs[leaf + 1] - off0;
-        const int npc = (nslots + a.chunk - 1) / a.chunk;
+        const int pt0 = ix.ptile[leaf], ntile = ix.ptile[leaf + 1] - pt0;
+        const int npc = (ntile + a.chunk - 1) / a.chunk;
         const int local = item - item_off[leaf];
         const int g = local / npc, c = local - g * npc;
         const int qcnt = b.qcount[leaf];
-        const int gsize = min(G, qcnt - g * G);
-        const int s0 = off0 + c * a.chunk;
-        const int s1 = min(off0 + nslots, s0 + a.chunk);
-        if (threadIdx.x < G) {
-            int qq = (threadIdx.x < gsize) ? b.qlist[b.qoff[leaf] + g * G + threadIdx.x] : -1;
+        TileJob job;
+        job.gsize = min(GMAX, qcnt - g * GMAX);
+        const int G = ((job.gsize + GSTEP - 1) / GSTEP) * GSTEP;   // table width of this group
+        job.t0 = pt0 + c * a.chunk;
+        job.t1 = min(pt0 + ntile, job.t0 + a.chunk);
+        job.slot_base = ix.offs[leaf] - 32 * pt0;
+        job.send = ix.offs[leaf + 1];
+        if (threadIdx.x < GMAX) {
+            int qq = (threadIdx.x < job.gsize) ? b.qlist[b.qoff[leaf] + g * GMAX + threadIdx.x] : -1;
             s_q[threadIdx.x] = qq;
             uint64_t t = (qq >= 0) ? b.tau[qq] : ~0ull;
             s_th[threadIdx.x] = static_cast<uint32_t>(t >> 32);
@@ -602,110 +768,55 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(DeviceIndex ix, Sear
         // stage the group's tables
         const int per_q = B * kCenters;
         if (MODE == 0) {
-            float* lf = reinterpret_cast<float*>(smem);
-            for (int e = threadIdx.x; e < G * per_q; e += kScanThreads) {
-                int qi = e / per_q, r = e - qi * per_q;
-                int blk = r >> 4, j = r & 15;
-                int qq = s_q[qi];
-                float v = (qq >= 0) ? b.lut_f32[static_cast<int64_t>(qq) * per_q + r] : 0.0f;
-                lf[((blk * (G / 2) + (qi >> 1)) * kCenters + j) * 2 + (qi & 1)] = v;
+            // one 8-byte store per (block, center) of each query pair
+            float2* lf = reinterpret_cast<float2*>(smem);
+            const int half = G / 2;
+            for (int pr = 0; pr < half; ++pr) {
+                const int qa = s_q[2 * pr], qb = s_q[2 * pr + 1];
+                const float* la = b.lut_f32 + static_cast<int64_t>(qa < 0 ? 0 : qa) * per_q;
+                const float* lb = b.lut_f32 + static_cast<int64_t>(qb < 0 ? 0 : qb) * per_q;
+                for (int r = threadIdx.x; r < per_q; r += kScanThreads) {
+                    const float va = (qa >= 0) ? la[r] : 0.0f;
+                    const float vb = (qb >= 0) ? lb[r] : 0.0f;
+                    lf[((r >> 4) * half + pr) * kCenters + (r & 15)] = make_float2(va, vb);
+                }
             }
         } else {
-            for (int e = threadIdx.x; e < G * per_q; e += kScanThreads) {
-                int qi = e / per_q, r = e - qi * per_q;
-                int blk = r >> 4, j = r & 15;
-                int qq = s_q[qi];
-                uint8_t v = (qq >= 0) ? b.lut_u8[static_cast<int64_t>(qq) * per_q + r] : 0;
-                smem[((blk * (G / 4) + (qi >> 2)) * kCenters + j) * 4 + (qi & 3)] = v;
+            // one 4-byte store per (block, center) of each query quad
+            uint32_t* lw = reinterpret_cast<uint32_t*>(smem);
+            const int quads = G / 4;
+            for (int qd = 0; qd < quads; ++qd) {
+                const uint8_t* src[4];
+                bool ok[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int qq = s_q[4 * qd + u];
+                    ok[u] = qq >= 0;
+                    src[u] = b.lut_u8 + static_cast<int64_t>(ok[u] ? qq : 0) * per_q;
+                }
+                for (int r = threadIdx.x; r < per_q; r += kScanThreads) {
+                    uint32_t v = 0u;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (ok[u]) v |= static_cast<uint32_t>(src[u][r]) << (8 * u);
+                    lw[((r >> 4) * quads + qd) * kCenters + (r & 15)] = v;
+                }
             }
         }
         __syncthreads();
-
-        const int t0 = s0 >> 5, t1 = (s1 - 1) >> 5;
-        for (int t = t0 + warp; t <= t1; t += NW) {
-            const int slot = t * 32 + lane;
-            const bool valid = (slot >= s0) && (slot < s1);
-            const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
-            if (MODE == 0) {
-                unsigned long long acc[G / 2];
-#pragma unroll
-                for (int p = 0; p < G / 2; ++p) acc[p] = 0ull;
-                for (int w0 = 0; w0 < W; w0 += 8) {
-                    uint32_t cw[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) cw[u] = (w0 + u < W) ? cwp[(w0 + u) * 32] : 0u;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int wi = w0 + u;
-                        if (wi >= W) break;
-                        const int nb = min(8, B - 8 * wi);
-                        const unsigned char* pb = smem + static_cast<size_t>(8 * wi) * blk_bytes;
-#pragma unroll
-                        for (int nib = 0; nib < 8; ++nib) {
-                            if (nib < nb) {
-                                const uint32_t j = (cw[u] >> (4 * nib)) & 15u;
-                                const unsigned long long* p =
-                                    reinterpret_cast<const unsigned long long*>(pb + nib * blk_bytes) + j;
-#pragma unroll
-                                for (int pr = 0; pr < G / 2; ++pr) acc[pr] = add_f32x2(acc[pr], p[pr * kCenters]);
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int qi = 0; qi < G; ++qi) {
-                    if (qi >= gsize) break;
-                    const float sc = (qi & 1) ? hi_f32(acc[qi >> 1]) : lo_f32(acc[qi >> 1]);
-                    const uint32_t key = float_key(sc);
-                    append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot,
-                                      s_q[qi], ix, b);
-                }
-            } else {
-                uint32_t sums[G];
-#pragma unroll
-                for (int qi = 0; qi < G; ++qi) sums[qi] = 0u;
-                for (int w0 = 0; w0 < W; w0 += 8) {
-                    uint32_t cw[8];
-                    uint32_t ae[G / 4], ao[G / 4];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) cw[u] = (w0 + u < W) ? cwp[(w0 + u) * 32] : 0u;
-#pragma unroll
-                    for (int p = 0; p < G / 4; ++p) { ae[p] = 0u; ao[p] = 0u; }
-                    // 8 words = 64 blocks: 16-bit lanes hold at most 64 * 255
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int wi = w0 + u;
-                        if (wi >= W) break;
-                        const int nb = min(8, B - 8 * wi);
-                        const unsigned char* pb = smem + static_cast<size_t>(8 * wi) * blk_bytes;
-#pragma unroll
-                        for (int nib = 0; nib < 8; ++nib) {
-                            if (nib < nb) {
-                                const uint32_t j = (cw[u] >> (4 * nib)) & 15u;
-                                const uint32_t* p = reinterpret_cast<const uint32_t*>(pb + nib * blk_bytes) + j;
-#pragma unroll
-                                for (int qd = 0; qd < G / 4; ++qd) {
-                                    const uint32_t v = p[qd * kCenters];
-                                    ae[qd] += v & 0x00FF00FFu;
-                                    ao[qd] += __byte_perm(v, 0u, 0x4341);
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int qd = 0; qd < G / 4; ++qd) {
-                        sums[4 * qd + 0] += ae[qd] & 0xFFFFu;
-                        sums[4 * qd + 2] += ae[qd] >> 16;
-                        sums[4 * qd + 1] += ao[qd] & 0xFFFFu;
-                        sums[4 * qd + 3] += ao[qd] >> 16;
-                    }
-                }
-#pragma unroll
-                for (int qi = 0; qi < G; ++qi) {
-                    if (qi >= gsize) break;
-                    append_candidates(valid && reaches(sums[qi], s_th[qi], s_tl[qi], ix.slot_ids, slot), sums[qi],
-                                      slot, s_q[qi], ix, b);
-                }
+        if (MODE == 0) {
+            switch (G) {
+                case 8: scan_tiles_f32<8>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 6: scan_tiles_f32<6>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 4: scan_tiles_f32<4>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                default: scan_tiles_f32<2>(ix, b, smem, job, s_q, s_th, s_tl); break;
+            }
+        } else {
+            switch (G) {
+                case 16: scan_tiles_u8<16>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 12: scan_tiles_u8<12>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 8: scan_tiles_u8<8>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                default: scan_tiles_u8<4>(ix, b, smem, job, s_q, s_th, s_tl); break;
             }
         }
     }
@@ -713,26 +824,27 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(DeviceIndex ix, Sear
 
 int scan_group(int lut_mode) { return lut_mode == 0 ? kGroupF32 : kGroupU8; }
 
-template <int G, int MODE>
+template <int MODE>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
-    size_t smem = static_cast<size_t>(ix.B) * G * kCenters * (MODE == 0 ? 4 : 1);
+    constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
+    size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
     a.scan_item_off_smem = (smem + off_bytes <= 200 * 1024 && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = cudaFuncSetAttribute(scan_kernel<G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<G, MODE>, kScanThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE>, kScanThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    scan_kernel<G, MODE><<<num_sms * per_sm, kScanThreads, smem, s>>>(ix, a, b);
+    scan_kernel<MODE><<<num_sms * per_sm, kScanThreads, smem, s>>>(ix, a, b);
     return cudaGetLastError();
 }
 
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s) {
-    if (a.lut_mode == 0) return launch_scan_t<kGroupF32, 0>(ix, a, b, num_sms, s);
-    return launch_scan_t<kGroupU8, 1>(ix, a, b, num_sms, s);
+    if (a.lut_mode == 0) return launch_scan_t<0>(ix, a, b, num_sms, s);
+    return launch_scan_t<1>(ix, a, b, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -766,10 +878,11 @@ __global__ void __launch_bounds__(kSelThreads) redo_scan_kernel(DeviceIndex ix, 
         const uint32_t th = static_cast<uint32_t>(tau >> 32), tl = static_cast<uint32_t>(tau);
         const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
         const int s0 = ix.offs[leaf], s1 = ix.offs[leaf + 1];
+        const int p0 = ix.ptile[leaf] * 32 - s0;            // padded position = slot + p0
         for (int base = s0; base < s1; base += kSelThreads) {
             const int slot = base + threadIdx.x;
             const bool in = slot < s1;
-            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot) : 0u;
+            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot + p0) : 0u;
             append_candidates(in && reaches(v, th, tl, ix.slot_ids, slot), v, slot, q, ix, b);
         }
     }
@@ -793,22 +906,32 @@ cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const S
 }
 
 // ---------------------------------------------------------------------------
-// select best R, exact reorder, best k
+// finish: best R, exact reorder, best k (one CTA per query)
 // ---------------------------------------------------------------------------
 
-size_t select_smem_bytes(int R) {
-    return static_cast<size_t>(next_pow2(R)) * (sizeof(uint64_t) + sizeof(int32_t));
+constexpr int kFinishThreads = 256;
+constexpr int kStageCap = 2048;          // candidate keys staged in shared memory up to this count
+
+size_t finish_smem_bytes(int R, int d) {
+    const size_t p2 = static_cast<size_t>(next_pow2(R));
+    return static_cast<size_t>(kStageCap) * (sizeof(uint64_t) + sizeof(int32_t)) +   // staged keys, slots
+           p2 * (2 * sizeof(uint64_t) + sizeof(int32_t)) +                            // best R keys, slots; exact keys
+           256 * sizeof(int) + static_cast<size_t>(d) * sizeof(float) + 64;            // warp histogram; query
 }
 
 // One CTA per query (round 0) or per entry of the previous round's redo list.
-// Keeps the best R of the query's buffer (by (approximate score, id) key).
-// A query whose buffer overflowed instead gets a tighter bound (the R-th best
-// stored key: stored entries are real candidates, so this is still a lower
-// bound on its R-th best) and is queued for a rescan; on the last round an
-// overflow is reported through the error word and the stored subset is used.
-// Without reorder the best k of the R are the result.
+//  1. The best R of the query's kept candidates by (approximate score, id) key.
+//     A query whose buffer overflowed instead gets a tighter bound (the R-th
+//     best stored key: stored entries are real candidates, so it is still a
+//     lower bound on the R-th best) and is queued for a rescan; on the last
+//     round an overflow is reported through the error word and the stored
+//     subset is used.
+//  2. Without reorder, the best k of those are the result.  With reorder,
+//     8-lane groups compute the exact fp32 dot product of each candidate's
+//     stored vector (float, or bfloat16 upcast) with the query, and one warp
+//     keeps the best k by (exact score, id).
 template <int MODE>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+__global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     int q;
@@ -818,10 +941,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DeviceIndex ix, Sea
         if (static_cast<int>(blockIdx.x) >= b.counters[round]) return;
         q = b.redo[static_cast<int64_t>(round - 1) * a.nq + blockIdx.x];
     }
-    const int cap = b.cap, R = a.R, k = a.k;
+    const int cap = b.cap, R = a.R, k = a.k, d = ix.d;
     const int P2 = next_pow2(R);
-    uint64_t* okeys = reinterpret_cast<uint64_t*>(smem);                 // [P2]
-    int32_t* oslots = reinterpret_cast<int32_t*>(okeys + P2);            // [P2]
+    uint64_t* skeys = reinterpret_cast<uint64_t*>(smem);            // [kStageCap]
+    uint64_t* okeys = skeys + kStageCap;                            // [P2]
+    uint64_t* ekeys = okeys + P2;                                   // [P2]
+    int32_t* sslots = reinterpret_cast<int32_t*>(ekeys + P2);       // [kStageCap]
+    int32_t* oslots = sslots + kStageCap;                           // [P2]
+    int* whist = oslots + P2;                                       // [256]
+    float* qv = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(whist + 256) + 15) & ~uintptr_t(15));  // [d], 16-B aligned
     const uint64_t* ck = b.ckey + static_cast<int64_t>(q) * cap;
     const int32_t* cs = b.cslot + static_cast<int64_t>(q) * cap;
     int cnt = b.count[q];
@@ -829,10 +957,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DeviceIndex ix, Sea
     if (cnt > cap) {
         if (round < 2) {
             auto get = [&](int i) { return ck[i]; };
-            auto pay = [&](int i) { return i; };
-            block_topk<kSelThreads>(get, pay, cap, R, scr, okeys, nullptr, b.err);
+            const uint64_t tau = block_kth_largest<kFinishThreads>(get, cap, R, scr);
             if (threadIdx.x == 0) {
-                b.tau[q] = okeys[R - 1];
+                b.tau[q] = tau;
                 b.count[q] = 0;
                 int pos = atomicAdd(&b.counters[round + 1], 1);
                 b.redo[static_cast<int64_t>(round) * a.nq + pos] = q;
@@ -842,118 +969,126 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(DeviceIndex ix, Sea
         if (threadIdx.x == 0) raise_error(b.err, kDevCandOverflow);
         cnt = cap;
     }
-    auto get = [&](int i) { return ck[i]; };
-    auto pay = [&](int i) { return cs[i]; };
-    const int K = block_topk<kSelThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+    int K;
+    if (cnt <= kStageCap) {
+        for (int i = threadIdx.x; i < cnt; i += kFinishThreads) {
+            skeys[i] = ck[i];
+            sslots[i] = cs[i];
+        }
+        __syncthreads();
+        auto get = [&](int i) { return skeys[i]; };
+        auto pay = [&](int i) { return sslots[i]; };
+        K = block_topk<kFinishThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+    } else {
+        auto get = [&](int i) { return ck[i]; };
+        auto pay = [&](int i) { return cs[i]; };
+        K = block_topk<kFinishThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+    }
     const float delta = (MODE == 1) ? b.lut_delta[q] : 0.0f;
     const float bias = (MODE == 1) ? b.lut_bias[q] : 0.0f;
     auto approx_score = [&](uint32_t sk) {
         return (MODE == 0) ? key_float(sk) : fmaf(delta, static_cast<float>(sk), bias);
     };
     const int64_t ro = static_cast<int64_t>(q) * R;
-    for (int i = threadIdx.x; i < R; i += kSelThreads) {
-        const bool have = i < K;
-        b.rkey[ro + i] = have ? okeys[i] : 0ull;
-        b.rslot[ro + i] = have ? oslots[i] : -1;
-        if (a.tr_cand_ids) a.tr_cand_ids[ro + i] = have ? key_id(okeys[i]) : -1;
-        if (a.tr_cand_scores) a.tr_cand_scores[ro + i] = have ? approx_score(key_score(okeys[i])) : -INFINITY;
-        if (a.tr_cand_sums) a.tr_cand_sums[ro + i] = (have && MODE == 1) ? key_score(okeys[i]) : 0u;
+    if (a.tr_cand_ids || a.tr_cand_scores || a.tr_cand_sums) {
+        for (int i = threadIdx.x; i < R; i += kFinishThreads) {
+            const bool have = i < K;
+            if (a.tr_cand_ids) a.tr_cand_ids[ro + i] = have ? key_id(okeys[i]) : -1;
+            if (a.tr_cand_scores) a.tr_cand_scores[ro + i] = have ? approx_score(key_score(okeys[i])) : -INFINITY;
+            if (a.tr_cand_sums) a.tr_cand_sums[ro + i] = (have && MODE == 1) ? key_score(okeys[i]) : 0u;
+        }
     }
-    if (threadIdx.x == 0) {
-        b.rcount[q] = K;
-        if (a.tr_ncand) a.tr_ncand[q] = K;
-    }
+    if (a.tr_ncand && threadIdx.x == 0) a.tr_ncand[q] = K;
+    const int64_t oo = static_cast<int64_t>(q) * k;
     if (a.reorder_num == 0) {
-        const int64_t oo = static_cast<int64_t>(q) * k;
-        for (int i = threadIdx.x; i < k; i += kSelThreads) {
+        for (int i = threadIdx.x; i < k; i += kFinishThreads) {
             const bool have = i < K;
             a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
             a.out_scores[oo + i] = have ? approx_score(key_score(okeys[i])) : -INFINITY;
         }
-    }
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    return v;
-}
-
-constexpr int kReorderThreads = 256;
-
-// Reordering: one warp per (query, kept candidate) computes the exact fp32 dot
-// product with the stored vector (float, or bfloat16 upcast), lanes striding
-// over d, then a butterfly sum.  Writes the (exact score, id) key.
-__global__ void __launch_bounds__(kReorderThreads) reorder_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
-    const int lane = threadIdx.x & 31;
-    const int64_t p = static_cast<int64_t>(blockIdx.x) * (kReorderThreads / 32) + (threadIdx.x >> 5);
-    const int R = a.R, d = ix.d;
-    if (p >= static_cast<int64_t>(a.nq) * R) return;
-    const int q = static_cast<int>(p / R), i = static_cast<int>(p - static_cast<int64_t>(q) * R);
-    if (i >= b.rcount[q]) {
-        if (lane == 0) b.ekey[p] = 0ull;
         return;
     }
-    const int64_t slot = b.rslot[p];
-    const float* qv = a.queries + static_cast<int64_t>(q) * d;
-    float acc = 0.0f;
-    if (ix.reorder_bf16) {
-        const uint16_t* v = reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d;
-        for (int t = lane; t < d; t += 32) acc = fmaf(qv[t], __uint_as_float(static_cast<uint32_t>(v[t]) << 16), acc);
+    // exact reorder: 32 groups of 8 lanes, one candidate per group per round
+    for (int t = threadIdx.x; t < d; t += kFinishThreads) qv[t] = a.queries[static_cast<int64_t>(q) * d + t];
+    __syncthreads();
+    const int grp = threadIdx.x >> 3, gl = threadIdx.x & 7;
+    for (int base = 0; base < K; base += kFinishThreads / 8) {
+        const int i = base + grp;
+        float acc = 0.0f;
+        if (i < K) {
+            const int64_t slot = oslots[i];
+            if (a.reorder_vec4) {        // d % 4 == 0 and 16-byte aligned rows (checked on the host)
+                const float4* q4 = reinterpret_cast<const float4*>(qv);
+                if (ix.reorder_bf16) {
+                    const uint2* v = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d);
+                    for (int t = gl; t < d / 4; t += 8) {
+                        const uint2 h = v[t];
+                        const float4 x = q4[t];
+                        acc = fmaf(x.x, __uint_as_float(h.x << 16), acc);
+                        acc = fmaf(x.y, __uint_as_float(h.x & 0xFFFF0000u), acc);
+                        acc = fmaf(x.z, __uint_as_float(h.y << 16), acc);
+                        acc = fmaf(x.w, __uint_as_float(h.y & 0xFFFF0000u), acc);
+                    }
+                } else {
+                    const float4* v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d);
+                    for (int t = gl; t < d / 4; t += 8) {
+                        const float4 h = v[t];
+                        const float4 x = q4[t];
+                        acc = fmaf(x.x, h.x, acc);
+                        acc = fmaf(x.y, h.y, acc);
+                        acc = fmaf(x.z, h.z, acc);
+                        acc = fmaf(x.w, h.w, acc);
+                    }
+                }
+            } else if (ix.reorder_bf16) {
+                const uint16_t* v = reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d;
+                for (int t = gl; t < d; t += 8) acc = fmaf(qv[t], __uint_as_float(static_cast<uint32_t>(v[t]) << 16), acc);
+            } else {
+                const float* v = reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d;
+                for (int t = gl; t < d; t += 8) acc = fmaf(qv[t], v[t], acc);
+            }
+        }
+        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
+        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
+        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+        if (i < K && gl == 0) ekeys[i] = make_key(float_key(acc), key_id(okeys[i]));
+    }
+    __syncthreads();
+    auto eget = [&](int i) { return ekeys[i]; };
+    auto epay = [&](int i) { return i; };
+    if (k <= kWarpMaxK) {
+        if (threadIdx.x < 32) {
+            const int Kk = warp_topk(eget, epay, K, k, whist, okeys, nullptr);
+            for (int i = threadIdx.x; i < k; i += 32) {
+                const bool have = i < Kk;
+                a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
+                a.out_scores[oo + i] = have ? key_float(key_score(okeys[i])) : -INFINITY;
+            }
+        }
     } else {
-        const float* v = reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d;
-        for (int t = lane; t < d; t += 32) acc = fmaf(qv[t], v[t], acc);
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) b.ekey[p] = make_key(float_key(acc), key_id(b.rkey[p]));
-}
-
-constexpr int kFinalThreads = 128;
-
-// One CTA per query: the best k of its rescored candidates.
-__global__ void __launch_bounds__(kFinalThreads) final_kernel(SearchArgs a, SearchBuffers b) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ SelectScratch scr;
-    const int q = blockIdx.x;
-    const int R = a.R, k = a.k;
-    uint64_t* okeys = reinterpret_cast<uint64_t*>(smem);
-    const uint64_t* ek = b.ekey + static_cast<int64_t>(q) * R;
-    auto get = [&](int i) { return ek[i]; };
-    auto pay = [&](int i) { return i; };
-    const int K = block_topk<kFinalThreads>(get, pay, b.rcount[q], k, scr, okeys, nullptr, b.err);
-    const int64_t oo = static_cast<int64_t>(q) * k;
-    for (int i = threadIdx.x; i < k; i += kFinalThreads) {
-        const bool have = i < K;
-        a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
-        a.out_scores[oo + i] = have ? key_float(key_score(okeys[i])) : -INFINITY;
+        const int Kk = block_topk<kFinishThreads>(eget, epay, K, k, scr, okeys, nullptr, b.err);
+        for (int i = threadIdx.x; i < k; i += kFinishThreads) {
+            const bool have = i < Kk;
+            a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
+            a.out_scores[oo + i] = have ? key_float(key_score(okeys[i])) : -INFINITY;
+        }
     }
 }
 
-cudaError_t launch_select(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, cudaStream_t s) {
-    size_t smem = select_smem_bytes(a.R);
+cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, cudaStream_t s) {
+    const uintptr_t qa = reinterpret_cast<uintptr_t>(a.queries), va = reinterpret_cast<uintptr_t>(ix.reorder_vecs);
+    a.reorder_vec4 = (ix.d % 4 == 0 && qa % 16 == 0 && va % 16 == 0) ? 1 : 0;
+    const size_t smem = finish_smem_bytes(a.R, ix.d);
     cudaError_t e;
     if (a.lut_mode == 0) {
-        e = cudaFuncSetAttribute(select_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = cudaFuncSetAttribute(finish_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        select_kernel<0><<<a.nq, kSelThreads, smem, s>>>(ix, a, b, round);
+        finish_kernel<0><<<a.nq, kFinishThreads, smem, s>>>(ix, a, b, round);
     } else {
-        e = cudaFuncSetAttribute(select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = cudaFuncSetAttribute(finish_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        select_kernel<1><<<a.nq, kSelThreads, smem, s>>>(ix, a, b, round);
+        finish_kernel<1><<<a.nq, kFinishThreads, smem, s>>>(ix, a, b, round);
     }
-    return cudaGetLastError();
-}
-
-cudaError_t launch_reorder(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
-    const int64_t pairs = static_cast<int64_t>(a.nq) * a.R;
-    const int64_t grid = (pairs + kReorderThreads / 32 - 1) / (kReorderThreads / 32);
-    reorder_kernel<<<static_cast<unsigned>(grid), kReorderThreads, 0, s>>>(ix, a, b);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    size_t smem = static_cast<size_t>(next_pow2(a.k)) * sizeof(uint64_t);
-    e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    final_kernel<<<a.nq, kFinalThreads, smem, s>>>(a, b);
     return cudaGetLastError();
 }
 

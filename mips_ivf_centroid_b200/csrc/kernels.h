@@ -19,8 +19,9 @@ struct DeviceIndex {
     int d, nl, dpb, B, W;                 // W: 32-bit code words per point
     const float* centroids;               // [NL][d]
     const int32_t* offs;                  // [NL+1] int32 leaf offsets (owned copy)
+    const int32_t* ptile;                 // [NL+1] first code tile of each leaf (leaf-padded copy)
     const int32_t* slot_ids;              // [n]
-    const uint32_t* codes_il;             // [ceil(n/32)][W][32] (owned)
+    const uint32_t* codes_il;             // [ptile[NL]][W][32] leaf-padded tiles (owned)
     const float* codebook;                // [B][16][dpb]
     const void* reorder_vecs;             // [n][d]
     int reorder_bf16;
@@ -40,10 +41,6 @@ struct SearchBuffers {
     uint64_t* ckey;         // [nq][cap] kept candidates: (score key, id) keys
     int32_t* cslot;         // [nq][cap] and their slots
     int32_t* count;         // [nq]          (zeroed per search)
-    uint64_t* rkey;         // [nq][R] best R (approximate score, id) keys, descending
-    int32_t* rslot;         // [nq][R] their slots
-    int32_t* rcount;        // [nq]    how many (<= R)
-    uint64_t* ekey;         // [nq][R] (exact score, id) keys after reordering
     int32_t* redo;          // [2][nq]       queries to rescan after rounds 0 and 1
     int32_t* counters;      // [8]           (zeroed per search): 0 scan work, 1..2 redo list sizes,
                             //               3..4 rescan work of rounds 1..2
@@ -59,7 +56,8 @@ struct SearchBuffers {
 
 struct SearchArgs {
     const float* queries;
-    int nq, k, L, reorder_num, R, lut_mode, chunk;
+    int nq, k, L, reorder_num, R, lut_mode;
+    int chunk;                  // code tiles (32 slots each) per scan work item
     int32_t* out_ids;
     float* out_scores;
     // optional trace outputs
@@ -74,11 +72,12 @@ struct SearchArgs {
     int32_t* tr_rescans;
     int scan_item_off_smem;     // set by the scan launcher
     int topl_row_smem;          // set by the top-leaves launcher
+    int reorder_vec4;           // set by the reorder launcher: 16-byte vector loads allowed
 };
 
-// Build-time: int32 offsets and the tiled code copy.
-cudaError_t launch_prepare_index(const int64_t* offs64, int nl, int32_t* offs32, const uint8_t* codes,
-                                 int64_t n, int cb, int W, uint32_t* codes_il, cudaStream_t s);
+// Build-time: the leaf-padded tiled code copy.
+cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, int nl, const uint8_t* codes, int cb,
+                                 int W, int64_t ntiles, uint32_t* codes_il, cudaStream_t s);
 
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s);
@@ -86,14 +85,13 @@ cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const Sear
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s);
-// round 0: all queries; rounds 1..2: the redo list of the previous round
-cudaError_t launch_select(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, cudaStream_t s);
-// exact rescoring of the kept candidates, then the best k (reorder_num > 0)
-cudaError_t launch_reorder(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+// best R, exact reorder, best k.  round 0: all queries; rounds 1..2: the
+// redo list of the previous round
+cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, cudaStream_t s);
 cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round,
                              int num_sms, cudaStream_t s);
 
 int scan_group(int lut_mode);
-size_t select_smem_bytes(int R);
+size_t finish_smem_bytes(int R, int d);
 
 }  // namespace ah

@@ -196,3 +196,195 @@ __device__ int block_topk(GetKey get, GetVal pay, int n, int K, SelectScratch& s
 }
 
 }  // namespace ah
+
+// ---------------------------------------------------------------------------
+// Warp-cooperative versions: one warp selects for one query with no block
+// barrier.  `hist` is this warp's 256-int shared histogram; outputs are this
+// warp's shared arrays of capacity next_pow2(K).
+// ---------------------------------------------------------------------------
+namespace ah {
+
+__device__ __forceinline__ uint64_t warp_and64(uint64_t v) {
+    const unsigned hi = __reduce_and_sync(0xFFFFFFFFu, static_cast<unsigned>(v >> 32));
+    const unsigned lo = __reduce_and_sync(0xFFFFFFFFu, static_cast<unsigned>(v));
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t warp_or64(uint64_t v) {
+    const unsigned hi = __reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(v >> 32));
+    const unsigned lo = __reduce_or_sync(0xFFFFFFFFu, static_cast<unsigned>(v));
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Same selection rule as block_select_threshold: (key & mask) >= prefix holds
+// for exactly K of n distinct keys.  Requires 1 <= K < n.
+template <class GetKey>
+__device__ void warp_select_threshold(GetKey get, int n, int K, int* hist, uint64_t* prefix_out, uint64_t* mask_out) {
+    const int lane = threadIdx.x & 31;
+    uint64_t kand = ~0ull, kor = 0ull;
+    for (int i = lane; i < n; i += 32) {
+        const uint64_t k = get(i);
+        kand &= k;
+        kor |= k;
+    }
+    kand = warp_and64(kand);
+    kor = warp_or64(kor);
+    const uint64_t diff = kand ^ kor;
+    int shift = 56;
+    uint64_t prefix = 0ull, mask = 0ull;
+    if (diff != 0ull) {
+        const int top = 63 - __clzll(static_cast<long long>(diff));
+        shift = (top / 8) * 8;
+        mask = (shift >= 56) ? 0ull : (~0ull << (shift + 8));
+        prefix = kand & mask;
+    }
+    int need = K;
+    for (; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0;
+        __syncwarp();
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            bool take = false;
+            int bin = 256 + lane;
+            if (i < n) {
+                const uint64_t k = get(i);
+                take = (k & mask) == prefix;
+                if (take) bin = static_cast<int>((k >> shift) & 255);
+            }
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
+            if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
+        __syncwarp();
+        int local = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) local += hist[lane * 8 + i];
+        int suf = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_down_sync(0xFFFFFFFFu, suf, off);
+            if (lane + off < 32) suf += v;
+        }
+        const int above_lane = suf - local;
+        const bool here = (above_lane < need) && (suf >= need);
+        int my_bucket = 0, my_above = 0;
+        if (here) {
+            int acc = above_lane;
+            for (int i = 7; i >= 0; --i) {
+                const int h = hist[lane * 8 + i];
+                if (acc + h >= need) {
+                    my_bucket = lane * 8 + i;
+                    my_above = acc;
+                    break;
+                }
+                acc += h;
+            }
+        }
+        const unsigned hb = __ballot_sync(0xFFFFFFFFu, here);
+        const int src = hb ? (__ffs(hb) - 1) : 0;
+        const int bucket = __shfl_sync(0xFFFFFFFFu, my_bucket, src);
+        const int above = __shfl_sync(0xFFFFFFFFu, my_above, src);
+        const int cnt_b = hist[bucket];
+        __syncwarp();
+        need -= above;
+        prefix |= static_cast<uint64_t>(bucket) << shift;
+        mask |= 0xFFull << shift;
+        if (cnt_b == need) break;
+    }
+    *prefix_out = prefix;
+    *mask_out = mask;
+}
+
+__device__ __forceinline__ void warp_sort_desc(uint64_t* keys, int32_t* vals, int P2) {
+    const int lane = threadIdx.x & 31;
+    for (int size = 2; size <= P2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            __syncwarp();
+            for (int t = lane; t < (P2 >> 1); t += 32) {
+                const int i = 2 * t - (t & (stride - 1));
+                const int j = i + stride;
+                const bool desc = ((i & size) == 0);
+                const uint64_t a = keys[i], b = keys[j];
+                if (desc ? (a < b) : (a > b)) {
+                    keys[i] = b;
+                    keys[j] = a;
+                    if (vals) {
+                        const int32_t t2 = vals[i];
+                        vals[i] = vals[j];
+                        vals[j] = t2;
+                    }
+                }
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// The K = min(K, n) largest keys of get(i) (payload pay(i)), sorted
+// descending into out_keys/out_vals; slots K..next_pow2(K)-1 hold key 0.
+// Compaction is by ballot, so the kept set is written in index order before
+// the sort.  Returns K.
+template <class GetKey, class GetVal>
+__device__ int warp_topk(GetKey get, GetVal pay, int n, int K, int* hist, uint64_t* out_keys, int32_t* out_vals) {
+    const int lane = threadIdx.x & 31;
+    if (K > n) K = n;
+    if (K <= 0) return 0;
+    uint64_t prefix = 0ull, mask = 0ull;
+    if (K < n) warp_select_threshold(get, n, K, hist, &prefix, &mask);
+    const int P2 = next_pow2(K);
+    for (int i = lane; i < P2; i += 32) {
+        out_keys[i] = 0ull;
+        if (out_vals) out_vals[i] = -1;
+    }
+    __syncwarp();
+    int base = 0;
+    for (int b0 = 0; b0 < n; b0 += 32) {
+        const int i = b0 + lane;
+        bool sel = false;
+        uint64_t k = 0ull;
+        if (i < n) {
+            k = get(i);
+            sel = (k & mask) >= prefix;
+        }
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            if (pos < K) {
+                out_keys[pos] = k;
+                if (out_vals) out_vals[pos] = pay(i);
+            }
+        }
+        base += __popc(m);
+    }
+    warp_sort_desc(out_keys, out_vals, P2);
+    return K;
+}
+
+}  // namespace ah
+
+namespace ah {
+
+// The K-th largest of n distinct keys (1 <= K <= n) without sorting: the
+// minimum of the selected set.  All threads of the block call it; all get it.
+template <int NT, class GetKey>
+__device__ uint64_t block_kth_largest(GetKey get, int n, int K, SelectScratch& s) {
+    uint64_t prefix = 0ull, mask = 0ull;
+    if (K < n) block_select_threshold<NT>(get, n, K, s, &prefix, &mask);
+    uint64_t mn = ~0ull;
+    for (int i = threadIdx.x; i < n; i += NT) {
+        const uint64_t k = get(i);
+        if ((k & mask) >= prefix && k < mn) mn = k;
+    }
+    // warp min, then across warps through the scratch word
+    const unsigned hi = __reduce_min_sync(0xFFFFFFFFu, static_cast<unsigned>(mn >> 32));
+    const unsigned lo = __reduce_min_sync(0xFFFFFFFFu, (static_cast<unsigned>(mn >> 32) == hi)
+                                                           ? static_cast<unsigned>(mn) : 0xFFFFFFFFu);
+    if (threadIdx.x == 0) s.kand = ~0ull;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) atomicMin(&s.kand, (static_cast<unsigned long long>(hi) << 32) | lo);
+    __syncthreads();
+    const uint64_t r = s.kand;
+    __syncthreads();
+    return r;
+}
+
+}  // namespace ah
