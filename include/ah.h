@@ -192,6 +192,19 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
                      int32_t reorder_num, int32_t lut_mode);
 
 /*
+ * Search tuning knobs (they never change results, only speed).
+ *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves in
+ *                            rank order, to bound its R-th best approximate
+ *                            score before the scan (default 1024; the bound
+ *                            uses max(R, value) points, at most 4096)
+ *   AH_OPT_SCAN_CHUNK_TILES  32-point code tiles per scan work item (0 =
+ *                            automatic, the default)
+ * Errors: AH_ERR_INVALID_ARG for an unknown option or a value out of range.
+ */
+enum { AH_OPT_THRESHOLD_SAMPLE = 1, AH_OPT_SCAN_CHUNK_TILES = 2 };
+AH_API ah_status ah_set_option(ah_index *ix, int32_t option, int64_t value);
+
+/*
  * Synchronise cuda_stream, then report and clear the index's device error
  * word: AH_OK, or AH_ERR_DEVICE with ah_last_error() describing it.
  */

@@ -71,6 +71,8 @@ struct ah_index {
     bool ev_recorded = false;
     int last_launches = 0;
     int last_nq = 0;
+    int opt_threshold_sample = 1024;
+    int opt_chunk_tiles = 0;
 };
 
 namespace {
@@ -200,7 +202,8 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     a.reorder_num = reorder_num;
     a.R = R;
     a.lut_mode = lut_mode;
-    a.chunk = nq >= 64 ? 32 : 8;          // code tiles per scan work item
+    a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : (nq >= 64 ? 32 : 8);   // code tiles per scan item
+    a.threshold_sample = ix->opt_threshold_sample;
     a.out_ids = out_ids;
     a.out_scores = out_scores;
     if (tr) {
@@ -242,12 +245,12 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
     launches += 1;
     mark(6);
-    if ((e = ah::launch_finish(dix, a, b, 0, s)) != cudaSuccess) return cuda_fail(e, "finish");
+    if ((e = ah::launch_finish(dix, a, b, 0, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "finish");
     launches += 1;
     mark(7);
     for (int round = 1; round <= 2; ++round) {
         if ((e = ah::launch_redo_scan(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "rescan");
-        if ((e = ah::launch_finish(dix, a, b, round, s)) != cudaSuccess) return cuda_fail(e, "finish after rescan");
+        if ((e = ah::launch_finish(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "finish after rescan");
         launches += 2;
     }
     mark(8);
@@ -437,6 +440,22 @@ ah_status ah_sync_status(ah_index* ix, void* cuda_stream) {
         case ah::kDevBadLeaf: return fail(AH_ERR_DEVICE, "leaf id out of range");
         case ah::kDevSelectSize: return fail(AH_ERR_DEVICE, "selection size mismatch (duplicate keys)");
         default: return fail(AH_ERR_DEVICE, "device error " + std::to_string(code));
+    }
+}
+
+ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
+    if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    switch (option) {
+        case AH_OPT_THRESHOLD_SAMPLE:
+            if (value < 1 || value > 4096) return fail(AH_ERR_INVALID_ARG, "threshold sample outside [1, 4096]");
+            ix->opt_threshold_sample = static_cast<int>(value);
+            return AH_OK;
+        case AH_OPT_SCAN_CHUNK_TILES:
+            if (value < 0 || value > 1024) return fail(AH_ERR_INVALID_ARG, "scan chunk outside [0, 1024] tiles");
+            ix->opt_chunk_tiles = static_cast<int>(value);
+            return AH_OK;
+        default:
+            return fail(AH_ERR_INVALID_ARG, "unknown option");
     }
 }
 

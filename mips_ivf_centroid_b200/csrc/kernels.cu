@@ -19,12 +19,36 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
 
 namespace ah {
+
+// cudaFuncSetAttribute costs host time on every call; each kernel's dynamic
+// shared-memory limit and carveout are raised once per device and size.
+namespace {
+std::mutex g_attr_mu;
+std::unordered_map<uint64_t, int> g_attr_smem;
+}  // namespace
+
+static cudaError_t ensure_smem(const void* kernel, size_t bytes, bool max_carveout) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t key = (reinterpret_cast<uint64_t>(kernel) << 6) ^ static_cast<uint64_t>(dev);
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    auto it = g_attr_smem.find(key);
+    if (it != g_attr_smem.end() && it->second >= static_cast<int>(bytes)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess && max_carveout)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) g_attr_smem[key] = static_cast<int>(bytes);
+    return e;
+}
 
 // ---------------------------------------------------------------------------
 // index preparation
@@ -174,7 +198,7 @@ static cudaError_t launch_top_leaves_block(const DeviceIndex& ix, SearchArgs a, 
     const size_t row = static_cast<size_t>(ix.nl) * sizeof(float);
     a.topl_row_smem = (row <= 64 * 1024) ? 1 : 0;
     if (a.topl_row_smem) smem += row;
-    cudaError_t e = cudaFuncSetAttribute(top_leaves_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_kernel), smem, true);
     if (e != cudaSuccess) return e;
     top_leaves_kernel<<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
     return cudaGetLastError();
@@ -334,7 +358,7 @@ cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchB
         lut_f32_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(ix, a, b);
     } else {
         size_t smem = (static_cast<size_t>(ix.B) * kCenters + ix.B) * sizeof(float);
-        cudaError_t e = cudaFuncSetAttribute(lut_u8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(lut_u8_kernel), smem, true);
         if (e != cudaSuccess) return e;
         lut_u8_kernel<<<a.nq, 256, smem, s>>>(ix, a, b);
     }
@@ -444,18 +468,19 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 // threshold: R-th best approximate score over a prefix of the best leaves
 // ---------------------------------------------------------------------------
 
-// Slots sampled per query for the bound.
-__host__ __device__ __forceinline__ int threshold_sample(int R) {
-    return min(kMaxThresholdSample, max(R, 1024));
+// Slots sampled per query for the bound: the requested sample, at least R,
+// at most kMaxThresholdSample.
+__host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
+    return min(kMaxThresholdSample, max(R, requested));
 }
 
-// One CTA per query.  Scores the first M = min(points, max(R, 1024)) slots of
+// One CTA per query.  Scores the first M = min(points, threshold_sample) slots of
 // the query's leaves in rank order; the R-th largest (score, id) key among them
 // is a lower bound on the R-th largest over all its leaves (a subset's R-th
 // best can only be lower), so every point of the final top R has a key >= it.
 // With fewer than R points in total the bound is 0 (keep everything).
 template <int MODE>
-__global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+__global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     const int q = blockIdx.x;
@@ -465,7 +490,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, 
     uint64_t* top = nullptr;
     load_query_table<MODE>(ix, b, q, lut);
     __syncthreads();
-    const int M = threshold_sample(R);
+    const int M = threshold_sample(R, a.threshold_sample);
     int taken = 0;
     for (int i = 0; i < a.L && taken < M; ++i) {
         int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
@@ -503,13 +528,13 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(DeviceIndex ix, 
 
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
     cudaError_t e;
-    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + static_cast<size_t>(threshold_sample(a.R)) * sizeof(uint64_t);
+    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + static_cast<size_t>(threshold_sample(a.R, a.threshold_sample)) * sizeof(uint64_t);
     if (a.lut_mode == 0) {
-        e = cudaFuncSetAttribute(threshold_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
         threshold_kernel<0><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
     } else {
-        e = cudaFuncSetAttribute(threshold_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<1>), smem, true);
         if (e != cudaSuccess) return e;
         threshold_kernel<1><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
     }
@@ -832,7 +857,7 @@ static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const Sear
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
     a.scan_item_off_smem = (smem + off_bytes <= 200 * 1024 && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = cudaFuncSetAttribute(scan_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE>), smem, true);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE>, kScanThreads, smem);
@@ -894,11 +919,11 @@ cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const S
     cudaError_t e;
     const int grid = num_sms * 2;
     if (a.lut_mode == 0) {
-        e = cudaFuncSetAttribute(redo_scan_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = ensure_smem(reinterpret_cast<const void*>(redo_scan_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
         redo_scan_kernel<0><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
     } else {
-        e = cudaFuncSetAttribute(redo_scan_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        e = ensure_smem(reinterpret_cast<const void*>(redo_scan_kernel<1>), smem, true);
         if (e != cudaSuccess) return e;
         redo_scan_kernel<1><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
     }
@@ -910,7 +935,7 @@ cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const S
 // ---------------------------------------------------------------------------
 
 constexpr int kFinishThreads = 256;
-constexpr int kStageCap = 2048;          // candidate keys staged in shared memory up to this count
+constexpr int kStageCap = 1024;          // candidate keys staged in shared memory up to this count
 
 size_t finish_smem_bytes(int R, int d) {
     const size_t p2 = static_cast<size_t>(next_pow2(R));
@@ -931,16 +956,8 @@ size_t finish_smem_bytes(int R, int d) {
 //     stored vector (float, or bfloat16 upcast) with the query, and one warp
 //     keeps the best k by (exact score, id).
 template <int MODE>
-__global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ SelectScratch scr;
-    int q;
-    if (round == 0) {
-        q = blockIdx.x;
-    } else {
-        if (static_cast<int>(blockIdx.x) >= b.counters[round]) return;
-        q = b.redo[static_cast<int64_t>(round - 1) * a.nq + blockIdx.x];
-    }
+__device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, int q,
+                             unsigned char* smem, SelectScratch& scr) {
     const int cap = b.cap, R = a.R, k = a.k, d = ix.d;
     const int P2 = next_pow2(R);
     uint64_t* skeys = reinterpret_cast<uint64_t*>(smem);            // [kStageCap]
@@ -969,20 +986,60 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
         if (threadIdx.x == 0) raise_error(b.err, kDevCandOverflow);
         cnt = cap;
     }
+    // the best R need an order only when they are reported (trace) or are the
+    // result (no reorder); the reorder path reads them as a set
+    const bool sorted = a.reorder_num == 0 || a.tr_cand_ids || a.tr_cand_scores || a.tr_cand_sums;
     int K;
+    int staged = -1;                  // keys staged in shared memory, or -1: read from global
     if (cnt <= kStageCap) {
         for (int i = threadIdx.x; i < cnt; i += kFinishThreads) {
             skeys[i] = ck[i];
             sslots[i] = cs[i];
         }
+        staged = cnt;
         __syncthreads();
+    } else if (R < kStageCap) {
+        // Many kept candidates: the R-th best of the first kStageCap is a lower
+        // bound on the R-th best of all (a subset's), so one batched pass keeps
+        // only the keys that reach it.
+        for (int i = threadIdx.x; i < kStageCap; i += kFinishThreads) skeys[i] = ck[i];
+        __syncthreads();
+        auto sget = [&](int i) { return skeys[i]; };
+        const uint64_t bound = block_kth_largest<kFinishThreads>(sget, kStageCap, R, scr);
+        if (threadIdx.x == 0) scr.count = 0;
+        __syncthreads();
+        constexpr int U = 4;
+        for (int i0 = 0; i0 < cnt; i0 += U * kFinishThreads) {
+            uint64_t kk[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kFinishThreads + threadIdx.x;
+                kk[u] = (i < cnt) ? ck[i] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u * kFinishThreads + threadIdx.x;
+                if (i < cnt && kk[u] >= bound) {
+                    const int pos = atomicAdd(&scr.count, 1);
+                    if (pos < kStageCap) {
+                        skeys[pos] = kk[u];
+                        sslots[pos] = cs[i];
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (scr.count <= kStageCap) staged = scr.count;
+        __syncthreads();
+    }
+    if (staged >= 0) {
         auto get = [&](int i) { return skeys[i]; };
         auto pay = [&](int i) { return sslots[i]; };
-        K = block_topk<kFinishThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+        K = block_topk<kFinishThreads>(get, pay, staged, R, scr, okeys, oslots, b.err, sorted);
     } else {
         auto get = [&](int i) { return ck[i]; };
         auto pay = [&](int i) { return cs[i]; };
-        K = block_topk<kFinishThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err);
+        K = block_topk<kFinishThreads>(get, pay, cnt, R, scr, okeys, oslots, b.err, sorted);
     }
     const float delta = (MODE == 1) ? b.lut_delta[q] : 0.0f;
     const float bias = (MODE == 1) ? b.lut_bias[q] : 0.0f;
@@ -1008,11 +1065,13 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
         }
         return;
     }
-    // exact reorder: 32 groups of 8 lanes, one candidate per group per round
+    // exact reorder: groups of `lpc` lanes, one candidate per group per round
     for (int t = threadIdx.x; t < d; t += kFinishThreads) qv[t] = a.queries[static_cast<int64_t>(q) * d + t];
     __syncthreads();
-    const int grp = threadIdx.x >> 3, gl = threadIdx.x & 7;
-    for (int base = 0; base < K; base += kFinishThreads / 8) {
+    const int lpc = a.reorder_lanes;                  // power of two in [2, 32]
+    const int groups = kFinishThreads / lpc;
+    const int grp = threadIdx.x / lpc, gl = threadIdx.x & (lpc - 1);
+    for (int base = 0; base < K; base += groups) {
         const int i = base + grp;
         float acc = 0.0f;
         if (i < K) {
@@ -1021,7 +1080,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
                 const float4* q4 = reinterpret_cast<const float4*>(qv);
                 if (ix.reorder_bf16) {
                     const uint2* v = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d);
-                    for (int t = gl; t < d / 4; t += 8) {
+                    for (int t = gl; t < d / 4; t += lpc) {
                         const uint2 h = v[t];
                         const float4 x = q4[t];
                         acc = fmaf(x.x, __uint_as_float(h.x << 16), acc);
@@ -1031,7 +1090,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
                     }
                 } else {
                     const float4* v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d);
-                    for (int t = gl; t < d / 4; t += 8) {
+                    for (int t = gl; t < d / 4; t += lpc) {
                         const float4 h = v[t];
                         const float4 x = q4[t];
                         acc = fmaf(x.x, h.x, acc);
@@ -1042,15 +1101,13 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
                 }
             } else if (ix.reorder_bf16) {
                 const uint16_t* v = reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d;
-                for (int t = gl; t < d; t += 8) acc = fmaf(qv[t], __uint_as_float(static_cast<uint32_t>(v[t]) << 16), acc);
+                for (int t = gl; t < d; t += lpc) acc = fmaf(qv[t], __uint_as_float(static_cast<uint32_t>(v[t]) << 16), acc);
             } else {
                 const float* v = reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d;
-                for (int t = gl; t < d; t += 8) acc = fmaf(qv[t], v[t], acc);
+                for (int t = gl; t < d; t += lpc) acc = fmaf(qv[t], v[t], acc);
             }
         }
-        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 4);
-        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 2);
-        acc += __shfl_xor_sync(0xFFFFFFFFu, acc, 1);
+        for (int off = lpc >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
         if (i < K && gl == 0) ekeys[i] = make_key(float_key(acc), key_id(okeys[i]));
     }
     __syncthreads();
@@ -1075,19 +1132,48 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(DeviceIndex ix, 
     }
 }
 
-cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, cudaStream_t s) {
+template <int MODE>
+__global__ void __launch_bounds__(kFinishThreads, 6) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ SelectScratch scr;
+    if (round == 0) {
+        finish_query<MODE>(ix, a, b, 0, blockIdx.x, smem, scr);
+        return;
+    }
+    // rescan rounds: a small grid walks the previous round's redo list
+    const int n = b.counters[round];
+    for (int e = blockIdx.x; e < n; e += gridDim.x) {
+        finish_query<MODE>(ix, a, b, round, b.redo[static_cast<int64_t>(round - 1) * a.nq + e], smem, scr);
+        __syncthreads();
+    }
+}
+
+static int lanes_per_candidate(int d) {
+    const int vec = (d + 3) / 4;                 // 4-element loads per row
+    int lpc = 2;
+    while (lpc < 32 && lpc * 8 < vec) lpc <<= 1;  // about 8 loads per lane
+    return lpc;
+}
+
+template <class Kernel>
+static cudaError_t prefer_shared(Kernel k, size_t smem) {
+    return ensure_smem(reinterpret_cast<const void*>(k), smem, true);
+}
+
+cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, int num_sms,
+                          cudaStream_t s) {
     const uintptr_t qa = reinterpret_cast<uintptr_t>(a.queries), va = reinterpret_cast<uintptr_t>(ix.reorder_vecs);
     a.reorder_vec4 = (ix.d % 4 == 0 && qa % 16 == 0 && va % 16 == 0) ? 1 : 0;
+    a.reorder_lanes = lanes_per_candidate(ix.d);
     const size_t smem = finish_smem_bytes(a.R, ix.d);
+    const unsigned grid = (round == 0) ? static_cast<unsigned>(a.nq) : static_cast<unsigned>(std::min(a.nq, 2 * num_sms));
     cudaError_t e;
     if (a.lut_mode == 0) {
-        e = cudaFuncSetAttribute(finish_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        finish_kernel<0><<<a.nq, kFinishThreads, smem, s>>>(ix, a, b, round);
+        if ((e = prefer_shared(finish_kernel<0>, smem)) != cudaSuccess) return e;
+        finish_kernel<0><<<grid, kFinishThreads, smem, s>>>(ix, a, b, round);
     } else {
-        e = cudaFuncSetAttribute(finish_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        finish_kernel<1><<<a.nq, kFinishThreads, smem, s>>>(ix, a, b, round);
+        if ((e = prefer_shared(finish_kernel<1>, smem)) != cudaSuccess) return e;
+        finish_kernel<1><<<grid, kFinishThreads, smem, s>>>(ix, a, b, round);
     }
     return cudaGetLastError();
 }

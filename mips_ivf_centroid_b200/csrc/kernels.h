@@ -72,7 +72,9 @@ struct SearchArgs {
     int32_t* tr_rescans;
     int scan_item_off_smem;     // set by the scan launcher
     int topl_row_smem;          // set by the top-leaves launcher
-    int reorder_vec4;           // set by the reorder launcher: 16-byte vector loads allowed
+    int reorder_vec4;           // set by the finish launcher: 16-byte vector loads allowed
+    int reorder_lanes;          // set by the finish launcher: lanes per rescored candidate
+    int threshold_sample;       // slots sampled per query for the filter bound (requested)
 };
 
 // Build-time: the leaf-padded tiled code copy.
@@ -87,7 +89,8 @@ cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const S
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s);
 // best R, exact reorder, best k.  round 0: all queries; rounds 1..2: the
 // redo list of the previous round
-cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, cudaStream_t s);
+cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, int num_sms,
+                          cudaStream_t s);
 cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round,
                              int num_sms, cudaStream_t s);
 

@@ -162,12 +162,13 @@ __host__ __device__ __forceinline__ int next_pow2(int x) {
 }
 
 // Select the K = min(K, n) largest keys of get(i) (payload pay(i)) into
-// out_keys/out_vals (shared, capacity >= next_pow2(K)), sorted descending.
+// out_keys/out_vals (shared, capacity >= next_pow2(K)), sorted descending
+// (unless `sort` is false: then in no particular order).
 // Returns K.  Slots K..next_pow2(K)-1 hold key 0.  err is raised if more than
 // K keys qualify (duplicate keys).
 template <int NT, class GetKey, class GetVal>
 __device__ int block_topk(GetKey get, GetVal pay, int n, int K, SelectScratch& s,
-                          uint64_t* out_keys, int32_t* out_vals, int* err) {
+                          uint64_t* out_keys, int32_t* out_vals, int* err, bool sort = true) {
     if (K > n) K = n;
     if (K <= 0) return 0;
     uint64_t prefix = 0, mask = 0;
@@ -191,7 +192,7 @@ __device__ int block_topk(GetKey get, GetVal pay, int n, int K, SelectScratch& s
     }
     __syncthreads();
     if (threadIdx.x == 0 && s.count != K && err) raise_error(err, kDevSelectSize);
-    block_sort_desc<NT>(out_keys, out_vals, P2);
+    if (sort) block_sort_desc<NT>(out_keys, out_vals, P2);
     return K;
 }
 
@@ -324,7 +325,8 @@ __device__ __forceinline__ void warp_sort_desc(uint64_t* keys, int32_t* vals, in
 // Compaction is by ballot, so the kept set is written in index order before
 // the sort.  Returns K.
 template <class GetKey, class GetVal>
-__device__ int warp_topk(GetKey get, GetVal pay, int n, int K, int* hist, uint64_t* out_keys, int32_t* out_vals) {
+__device__ int warp_topk(GetKey get, GetVal pay, int n, int K, int* hist, uint64_t* out_keys, int32_t* out_vals,
+                         bool sort = true) {
     const int lane = threadIdx.x & 31;
     if (K > n) K = n;
     if (K <= 0) return 0;
@@ -355,7 +357,8 @@ __device__ int warp_topk(GetKey get, GetVal pay, int n, int K, int* hist, uint64
         }
         base += __popc(m);
     }
-    warp_sort_desc(out_keys, out_vals, P2);
+    if (sort) warp_sort_desc(out_keys, out_vals, P2);
+    else __syncwarp();
     return K;
 }
 
@@ -385,6 +388,27 @@ __device__ uint64_t block_kth_largest(GetKey get, int n, int K, SelectScratch& s
     const uint64_t r = s.kand;
     __syncthreads();
     return r;
+}
+
+}  // namespace ah
+
+namespace ah {
+
+// The K-th largest of n distinct keys (1 <= K <= n), computed by one warp
+// without sorting; all lanes return it.
+template <class GetKey>
+__device__ uint64_t warp_kth_largest(GetKey get, int n, int K, int* hist) {
+    uint64_t prefix = 0ull, mask = 0ull;
+    if (K < n) warp_select_threshold(get, n, K, hist, &prefix, &mask);
+    uint64_t mn = ~0ull;
+    for (int i = threadIdx.x & 31; i < n; i += 32) {
+        const uint64_t k = get(i);
+        if ((k & mask) >= prefix && k < mn) mn = k;
+    }
+    const unsigned hi = __reduce_min_sync(0xFFFFFFFFu, static_cast<unsigned>(mn >> 32));
+    const unsigned lo = __reduce_min_sync(0xFFFFFFFFu, (static_cast<unsigned>(mn >> 32) == hi)
+                                                           ? static_cast<unsigned>(mn) : 0xFFFFFFFFu);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
 }  // namespace ah

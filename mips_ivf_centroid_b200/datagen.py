@@ -269,19 +269,19 @@ def _train_codebook(w: Workload, X: torch.Tensor) -> torch.Tensor:
         return cb
     Sb = S.view(S.shape[0], B, dpb).transpose(0, 1).contiguous()        # [B, m, dpb]
     m = Sb.shape[1]
-    bstep = max(1, _ELEM_BUDGET // (m * NUM_CENTERS * dpb))
+    bstep = max(1, _ELEM_BUDGET // (m * NUM_CENTERS * max(dpb, 2)))
     for _ in range(w.lloyd_iters):
         new = cb.clone()
         for b0 in range(0, B, bstep):
             sb, cbb = Sb[b0:b0 + bstep], cb[b0:b0 + bstep]
             dist = (sb[:, :, None, :] - cbb[:, None, :, :]).pow(2).sum(-1)  # [b, m, 16]
             a = torch.argmin(dist, dim=2)                                  # [b, m]
-            sums = torch.zeros_like(cbb)
-            sums.scatter_add_(1, a[:, :, None].expand(-1, -1, dpb), sb)
-            cnt = torch.zeros(cbb.shape[:2], dtype=torch.float32, device=dev)
-            cnt.scatter_add_(1, a, torch.ones_like(a, dtype=torch.float32))
+            # member sums as a one-hot product (deterministic, unlike atomic scatter-adds)
+            onehot = torch.nn.functional.one_hot(a, NUM_CENTERS).to(torch.float64)   # [b, m, 16]
+            sums = torch.bmm(onehot.transpose(1, 2), sb.double())                    # [b, 16, dpb]
+            cnt = onehot.sum(1)                                                      # [b, 16]
             new[b0:b0 + bstep] = torch.where((cnt > 0)[:, :, None],
-                                             sums / cnt.clamp(min=1)[:, :, None], cbb)
+                                             (sums / cnt.clamp(min=1)[:, :, None]).float(), cbb)
         cb = new
     return cb
 

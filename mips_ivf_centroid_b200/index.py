@@ -79,6 +79,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_status_string": (ctypes.c_char_p, [I32]),
         "ah_last_error": (ctypes.c_char_p, []),
         "ah_search_leaves_noalloc": (I32, [P, P, I32, I32, P, P, P]),
+        "ah_set_option": (I32, [P, I32, I64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -206,6 +207,13 @@ class Index:
     def sync_status(self, stream=None):
         with torch.cuda.device(self.device):
             _check(self._lib, self._lib.ah_sync_status(self._h, _stream(stream)))
+
+    OPT_THRESHOLD_SAMPLE = 1
+    OPT_SCAN_CHUNK_TILES = 2
+
+    def set_option(self, option: int, value: int):
+        """Tuning knob (ah_set_option): results are unchanged, only speed."""
+        _check(self._lib, self._lib.ah_set_option(self._h, option, value))
 
     # -- instrumentation ------------------------------------------------------
     def set_profiling(self, on: bool = True):
