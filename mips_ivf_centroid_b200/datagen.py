@@ -18,7 +18,9 @@ query against centroids, never builds a query lookup table, never scans codes
 and never selects or reorders candidates.  The CPU oracle and the CUDA library
 both consume its arrays unchanged.
 
-Random draws use ``numpy.random.default_rng(seed)`` (PCG64).  Heavy index-build
+Random draws use ``numpy.random.default_rng`` (PCG64): the component means
+and labels from the workload's seed, the noise of each 1M-row chunk from a
+generator seeded with (seed-derived key, chunk index).  Heavy index-build
 arithmetic (nearest-centroid assignment, Lloyd iterations, code assignment) runs
 in torch on whatever device is given, so the large workloads build in seconds on
 a GPU; the results are inputs, so the device used does not affect parity.
@@ -26,7 +28,8 @@ a GPU; the results are inputs, so the device used does not affect parity.
 from __future__ import annotations
 
 import dataclasses
-import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -125,7 +128,12 @@ SWEEP_BATCHES = (1, 16, 256, 4_096, 16_384)
 SWEEP_LEAVES = (16, 64, 256)
 
 _CHUNK_ROWS = 1_000_000
-_ELEM_BUDGET = 1 << 27   # elements per temporary in the index-build steps
+_ELEM_BUDGET = 1 << 27   # elements per temporary in the index-build steps (CPU)
+_ELEM_BUDGET_CUDA = 1 << 29
+
+
+def _budget(device) -> int:
+    return _ELEM_BUDGET_CUDA if torch.device(device).type == "cuda" else _ELEM_BUDGET
 
 
 # --------------------------------------------------------------------------
@@ -147,30 +155,44 @@ def _draw_means(w: Workload, rng: np.random.Generator) -> np.ndarray:
     return rng.standard_normal((w.n_means, w.d), dtype=np.float32)
 
 
-def _mixture_rows(w: Workload, means: np.ndarray, rng: np.random.Generator, n: int) -> np.ndarray:
-    """Draw order: component labels (uniform), then noise in 1M-row chunks."""
+def _mixture_rows(w: Workload, means: np.ndarray, rng: np.random.Generator, n: int, stream_key: int) -> np.ndarray:
+    """Mixture draws: component labels (uniform) from ``rng``; then, per chunk
+    of 1M rows, noise from the chunk's own generator seeded with
+    (``stream_key``, chunk index), so chunks can be drawn in parallel and the
+    result does not depend on the thread count."""
     labels = rng.integers(0, means.shape[0], size=n)
     out = np.empty((n, w.d), dtype=np.float32)
     sig = np.float32(w.sigma)
-    for s in range(0, n, _CHUNK_ROWS):
+
+    def work(c: int) -> None:
+        s = c * _CHUNK_ROWS
         e = min(n, s + _CHUNK_ROWS)
-        noise = rng.standard_normal((e - s, w.d), dtype=np.float32)
+        g = np.random.default_rng([stream_key, c])
+        noise = g.standard_normal((e - s, w.d), dtype=np.float32)
         noise *= sig
         noise += means[labels[s:e]]
         if w.data_kind == "int255_mixture":
             np.clip(noise, 0.0, 255.0, out=noise)
             np.rint(noise, out=noise)
+        else:
+            _normalise_rows(noise)
         out[s:e] = noise
-    if w.data_kind == "unit_mixture":
-        _normalise_rows(out)
+
+    chunks = (n + _CHUNK_ROWS - 1) // _CHUNK_ROWS
+    if chunks == 1:
+        work(0)
+    else:
+        with ThreadPoolExecutor(max_workers=min(chunks, os.cpu_count() or 1)) as ex:
+            list(ex.map(work, range(chunks)))
     return out
 
 
 def make_data(w: Workload) -> np.ndarray:
-    """Datapoints X [n, d] float32 (seed ``w.data_seed``: means, labels, noise)."""
+    """Datapoints X [n, d] float32 (seed ``w.data_seed``: means, labels; noise
+    per chunk from (data_seed, chunk))."""
     rng = np.random.default_rng(w.data_seed)
     means = _draw_means(w, rng)
-    return _mixture_rows(w, means, rng, w.n)
+    return _mixture_rows(w, means, rng, w.n, 1_000_003 * w.data_seed + 11)
 
 
 def make_queries(w: Workload, nq: Optional[int] = None) -> np.ndarray:
@@ -187,7 +209,7 @@ def make_queries(w: Workload, nq: Optional[int] = None) -> np.ndarray:
         _normalise_rows(q)
         return q
     means = _draw_means(w, np.random.default_rng(w.data_seed))
-    return _mixture_rows(w, means, rng, nq)
+    return _mixture_rows(w, means, rng, nq, 1_000_003 * w.query_seed + 17)
 
 
 # --------------------------------------------------------------------------
@@ -233,8 +255,9 @@ class IndexArrays:
         return out
 
 
-def _nearest_rows(x: torch.Tensor, c: torch.Tensor, chunk: int = 262_144) -> torch.Tensor:
+def _nearest_rows(x: torch.Tensor, c: torch.Tensor) -> torch.Tensor:
     """argmin_j ||x_i - c_j||^2 by chunks; ties go to the lower j (first minimum)."""
+    chunk = max(1024, _budget(x.device) // max(1, c.shape[0]))
     cn = (c.double() * c.double()).sum(1).float()
     out = torch.empty(x.shape[0], dtype=torch.int64, device=x.device)
     for s in range(0, x.shape[0], chunk):
@@ -269,7 +292,7 @@ def _train_codebook(w: Workload, X: torch.Tensor) -> torch.Tensor:
         return cb
     Sb = S.view(S.shape[0], B, dpb).transpose(0, 1).contiguous()        # [B, m, dpb]
     m = Sb.shape[1]
-    bstep = max(1, _ELEM_BUDGET // (m * NUM_CENTERS * max(dpb, 2)))
+    bstep = max(1, _budget(dev) // (m * NUM_CENTERS * max(dpb, 2)))
     for _ in range(w.lloyd_iters):
         new = cb.clone()
         for b0 in range(0, B, bstep):
@@ -290,7 +313,7 @@ def _l2_codes(X: torch.Tensor, cb: torch.Tensor) -> torch.Tensor:
     """Per block nearest of 16 centers by squared L2 (ties -> lower j). [n, B] int64."""
     n = X.shape[0]
     B, _, dpb = cb.shape
-    chunk = max(1024, _ELEM_BUDGET // (B * NUM_CENTERS * dpb))
+    chunk = max(1024, _budget(X.device) // (B * NUM_CENTERS * dpb))
     codes = torch.empty((n, B), dtype=torch.int64, device=X.device)
     for s in range(0, n, chunk):
         xb = X[s:s + chunk].view(-1, B, dpb)
@@ -317,7 +340,7 @@ def _anisotropic_codes(X: torch.Tensor, cb: torch.Tensor, codes: torch.Tensor,
     cbd = cb.double()
     out = codes.clone()
     e1 = float(eta) - 1.0
-    chunk = max(1024, _ELEM_BUDGET // (4 * B * dpb))
+    chunk = max(1024, _budget(X.device) // (4 * B * dpb))
     for s in range(0, n, chunk):
         x = X[s:s + chunk].double()
         m = x.shape[0]

@@ -58,3 +58,74 @@ def same_set(a, b):
     a = np.asarray(a)
     b = np.asarray(b)
     return np.array_equal(np.sort(a[a >= 0]), np.sort(b[b >= 0]))
+
+
+def compare_search(index, arr, Q, k, L, reorder_num, lut_mode, qsel=None, max_leaf_mismatch=0.02,
+                   max_cand_mismatch=0.05, orc=None):
+    """Search all of Q on the GPU (one batch, as the benchmark launches it),
+    then check the rows ``qsel`` stage by stage against the oracle.
+
+    Returns a dict with the mismatch counts and the GPU/oracle outputs of the
+    checked rows."""
+    import torch
+    from oracle import OracleIndex
+
+    qsel = np.arange(Q.shape[0]) if qsel is None else np.asarray(qsel)
+    qg = torch.from_numpy(np.ascontiguousarray(Q)).to(index.device)
+    ids, scores, tr = index.search(qg, k, L, reorder_num, lut_mode, trace=True)
+    index.sync_status()
+    ids = ids.cpu().numpy()[qsel]
+    scores = scores.cpu().numpy()[qsel]
+    tr = {kk: v.cpu().numpy() for kk, v in tr.items()}
+    tr = {kk: (v[qsel] if v.ndim >= 1 and v.shape[0] == Q.shape[0] else v) for kk, v in tr.items()}
+    orc = orc or OracleIndex(arr)
+    Qs = np.ascontiguousarray(Q[qsel])
+    o = orc.search(Qs, k, L, reorder_num, lut_mode)
+    n = arr["slot_ids"].shape[0]
+    inv = np.empty(n, np.int64)
+    inv[arr["slot_ids"]] = np.arange(n)
+    leaf_mis = cand_mis = 0
+    for i in range(Qs.shape[0]):
+        q = Qs[i]
+        cs = orc.centroid_scores(q)
+        ranked_match(tr["leaf_ids"][i], tr["leaf_scores"][i], o["leaves"][i], o["leaf_scores"][i],
+                     lambda g: cs[g], f"q{qsel[i]} leaves")
+        if not same_set(tr["leaf_ids"][i], o["leaves"][i]):
+            leaf_mis += 1
+            continue
+        assert tr["scanned"][i] == o["scanned"][i], f"q{qsel[i]} scanned"
+        assert tr["ncand"][i] == o["ncand"][i], f"q{qsel[i]} ncand"
+        gc = tr["cand_ids"][i]
+        if lut_mode == 1:
+            np.testing.assert_array_equal(gc, o["cand_ids"][i], err_msg=f"q{qsel[i]} u8 candidates")
+            np.testing.assert_array_equal(tr["cand_sums"][i].astype(np.uint32), o["cand_sums"][i])
+            np.testing.assert_array_equal(tr["cand_scores"][i], o["cand_scores"][i].astype(np.float32))
+        else:
+            ranked_match(gc, tr["cand_scores"][i], o["cand_ids"][i], o["cand_scores"][i],
+                         lambda g: orc.point_scores(q, inv[g])[0], f"q{qsel[i]} candidates")
+        if reorder_num > 0:
+            exact_of = lambda g: orc.point_scores(q, inv[g])[1]
+        elif lut_mode == 0:
+            exact_of = lambda g: orc.point_scores(q, inv[g])[0]
+        else:
+            exact_of = None
+        if not same_set(gc, o["cand_ids"][i]):
+            cand_mis += 1
+            nc = int((gc >= 0).sum())
+            if exact_of is None:
+                continue
+            ex = exact_of(gc[:nc])
+            order = np.lexsort((gc[:nc], -ex))[:k]
+            ranked_match(ids[i], scores[i], np.pad(gc[:nc][order], (0, k - len(order)), constant_values=-1),
+                         np.pad(ex[order], (0, k - len(order)), constant_values=-np.inf), exact_of,
+                         f"q{qsel[i]} final*")
+            continue
+        if exact_of is None:
+            np.testing.assert_array_equal(ids[i], o["ids"][i])
+            np.testing.assert_array_equal(scores[i], o["scores"][i].astype(np.float32))
+        else:
+            ranked_match(ids[i], scores[i], o["ids"][i], o["scores"][i], exact_of, f"q{qsel[i]} final")
+    nq = Qs.shape[0]
+    assert leaf_mis <= max(1, max_leaf_mismatch * nq), f"{leaf_mis} queries with a different leaf set"
+    assert cand_mis <= max(1, max_cand_mismatch * nq), f"{cand_mis} queries with a different candidate set"
+    return dict(leaf_mismatch=leaf_mis, cand_mismatch=cand_mis, ids=ids, scores=scores, oracle=o, trace=tr)
