@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--e2e-steps", type=int, default=100)
+    p.add_argument("--sweep", action="store_true",
+                   help="sweep workload: one JSON line per (batch, leaves) point instead of the single line")
     return p.parse_args()
 
 
@@ -291,7 +293,7 @@ def run_ours(args):
 
     if rank == 0:
         med = {kname: statistics.median(v) for kname, v in stage_ms.items()}
-        scan_ms = med.get("scan", float("nan"))
+        scan_ms = med.get("scan", float("nan")) + med.get("scan_rest", 0.0)
         clocks = clk.summary()
         lookups = scanned * w.blocks
         bytes_per_lookup = 4 if mode == 0 else 1
@@ -337,10 +339,76 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_sweep(args):
+    """Queries/s and scan rates over the sweep grid (batch x leaves searched)."""
+    import torch
+    from mips_ivf_centroid_b200 import Index, build as ahbuild, datagen
+    ahbuild.build()
+    w = datagen.WORKLOADS["sweep"]
+    dev = torch.device("cuda", 0)
+    X = datagen.make_data(w)
+    Q = datagen.make_queries(w)
+    ix = datagen.build_index(w, X, dev)
+    del X
+    torch.cuda.empty_cache()
+    index = Index(ix)
+    offs = ix.leaf_offsets.cpu().numpy()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for L in datagen.SWEEP_LEAVES:
+        for nq in datagen.SWEEP_BATCHES:
+            qg = torch.from_numpy(Q[:nq]).to(dev)
+            index.reserve(nq, w.k, L, w.reorder_num, args.lut_mode)
+            for _ in range(3):
+                index.search(qg, w.k, L, w.reorder_num, args.lut_mode)
+            _, _, tr = index.search(qg, w.k, L, w.reorder_num, args.lut_mode, trace=True)
+            scanned = int(tr["scanned"].sum().item())
+            touched = np.unique(tr["leaf_ids"].cpu().numpy())
+            unique_bytes = int((offs[touched + 1] - offs[touched]).sum()) * w.code_bytes
+            index.sync_status()
+            # about 1 s of timed work per point, at least 5 steps
+            t0 = time.perf_counter()
+            index.search(qg, w.k, L, w.reorder_num, args.lut_mode)
+            torch.cuda.synchronize()
+            est = time.perf_counter() - t0
+            steps = int(min(200, max(5, 1.0 / max(est, 1e-4))))
+            index.set_profiling(True)
+            ms, scan, stages = [], [], {}
+            for _ in range(steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                index.search(qg, w.k, L, w.reorder_num, args.lut_mode)
+                e1.record(stream)
+                st = index.stage_times()
+                ms.append(e0.elapsed_time(e1))
+                scan.append(st["scan"] + st.get("scan_rest", 0.0))
+                for kname, v in st.items():
+                    stages.setdefault(kname, []).append(v)
+            index.set_profiling(False)
+            index.sync_status()
+            m = statistics.median(ms)
+            sc = statistics.median(scan)
+            lookups = scanned * w.blocks
+            line = {"sweep_point": {"nq": nq, "num_leaves_to_search": L}, "metric": METRIC, "unit": "queries/s",
+                    "value": nq / (m * 1e-3), "ms_per_step": m, "steps": steps,
+                    "scan_ms": sc, "scan_lookups_per_s": lookups / (sc * 1e-3),
+                    "scan_smem_gbs": lookups * (4 if args.lut_mode == 0 else 1) / (sc * 1e-3) / 1e9,
+                    "scan_unique_code_gbs": unique_bytes / (sc * 1e-3) / 1e9, "unique_code_bytes": unique_bytes,
+                    "points_scanned": scanned, "dtype": "f32" if args.lut_mode == 0 else "u8",
+                    "stages_ms": {kname: statistics.median(v) for kname, v in stages.items()},
+                    "config": config_dict(w.scaled(nq=nq, num_leaves_to_search=L), args)}
+            print(json.dumps(line), flush=True)
+    index.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

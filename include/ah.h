@@ -193,15 +193,29 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
 
 /*
  * Search tuning knobs (they never change results, only speed).
- *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves in
- *                            rank order, to bound its R-th best approximate
- *                            score before the scan (default 1024; the bound
- *                            uses max(R, value) points, at most 4096)
+ *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves, to
+ *                            bound its R-th best approximate score before the
+ *                            scan (default 1024; the bound uses
+ *                            max(value, 8 R) points, at most 4096)
+ *   AH_OPT_THRESHOLD_LEAVES  how many of the best leaves that sample is spread
+ *                            over, evenly; the rest of the sample follows
+ *                            rank order (default 1: a prefix in rank order)
+ *   AH_OPT_PROGRESSIVE_LEAVES  scan each query's best L1 leaves first, raise its
+ *                            bound to the R-th best point they kept, then scan
+ *                            up to 8x as many leaves at a time the same way:
+ *                            0 = automatic (several phases when the sample's
+ *                            bound is expected to keep many points and
+ *                            nq >= 64), -1 = one pass, n = L1
  *   AH_OPT_SCAN_CHUNK_TILES  32-point code tiles per scan work item (0 =
  *                            automatic, the default)
  * Errors: AH_ERR_INVALID_ARG for an unknown option or a value out of range.
  */
-enum { AH_OPT_THRESHOLD_SAMPLE = 1, AH_OPT_SCAN_CHUNK_TILES = 2 };
+enum {
+    AH_OPT_THRESHOLD_SAMPLE = 1,
+    AH_OPT_SCAN_CHUNK_TILES = 2,
+    AH_OPT_THRESHOLD_LEAVES = 3,
+    AH_OPT_PROGRESSIVE_LEAVES = 4
+};
 AH_API ah_status ah_set_option(ah_index *ix, int32_t option, int64_t value);
 
 /*

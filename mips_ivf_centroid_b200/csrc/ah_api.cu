@@ -31,9 +31,9 @@ ah_status cuda_fail(cudaError_t e, const char* what) {
     return e == cudaErrorMemoryAllocation ? AH_ERR_OOM : AH_ERR_CUDA;
 }
 
-constexpr int kStages = 8;
-const char* kStageNames[kStages] = {"centroid_scores", "top_leaves", "invert", "lut",
-                                    "threshold", "scan", "finish", "rescan"};
+constexpr int kStages = 10;
+const char* kStageNames[kStages] = {"centroid_scores", "top_leaves", "invert", "lut", "threshold",
+                                    "scan", "refine", "scan_rest", "finish", "rescan"};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -66,12 +66,17 @@ struct ah_index {
     size_t owned_bytes = 0;
     Workspace ws;
     bool profiling = false;
-    cudaEvent_t ev[kStages + 1]{};
+    static constexpr int kMaxMarks = 64;
+    cudaEvent_t ev[kMaxMarks]{};
+    int mark_stage[kMaxMarks]{};      // stage ending at mark i (-1: none)
+    int n_marks = 0;
     bool ev_ready = false;
     bool ev_recorded = false;
     int last_launches = 0;
     int last_nq = 0;
     int opt_threshold_sample = 1024;
+    int opt_threshold_leaves = 1;
+    int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
 };
 
@@ -204,6 +209,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     a.lut_mode = lut_mode;
     a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : (nq >= 64 ? 32 : 8);   // code tiles per scan item
     a.threshold_sample = ix->opt_threshold_sample;
+    a.threshold_leaves = ix->opt_threshold_leaves;
     a.out_ids = out_ids;
     a.out_scores = out_scores;
     if (tr) {
@@ -221,39 +227,74 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     const bool prof = ix->profiling && ix->ev_ready;
     int launches = 0;
     cudaError_t e;
-    auto mark = [&](int i) {
-        if (prof) cudaEventRecord(ix->ev[i], s);
+    // mark(stage): the interval since the previous mark belongs to `stage`
+    ix->n_marks = 0;
+    auto mark = [&](int stage) {
+        if (prof && ix->n_marks < ah_index::kMaxMarks) {
+            ix->mark_stage[ix->n_marks] = stage;
+            cudaEventRecord(ix->ev[ix->n_marks++], s);
+        }
     };
     e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)(2 * dix.nl + ix->ws.nq + 8), s);
     if (e != cudaSuccess) return cuda_fail(e, "memset");
-    mark(0);
+    mark(-1);
     if ((e = ah::launch_centroid_scores(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "centroid scores");
     launches += 1;
-    mark(1);
+    mark(0);
     if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
     launches += 1;
+    mark(1);
+    // Scan phases over leaf ranks [bounds[p], bounds[p+1]).  One phase when
+    // the bound from the sample is expected to keep few points; otherwise the
+    // first phase is small enough for that bound, each later phase covers up
+    // to 8x the leaves scanned so far, and between phases every query's bound
+    // is raised to the R-th best point kept (and its buffer compacted).
+    std::vector<int> bounds{0};
+    {
+        const int M = std::min(4096, std::max(std::max(a.R, ix->opt_threshold_sample), 8 * a.R));
+        const double avg_leaf = static_cast<double>(dix.n) / dix.nl;
+        const double expect_one_pass = 0.25 * a.R * L * avg_leaf / M;   // points kept by the sample's bound
+        int first = L;
+        if (ix->opt_progressive_leaves > 0) first = std::min(L, ix->opt_progressive_leaves);
+        else if (ix->opt_progressive_leaves == 0 && nq >= 64 && expect_one_pass > b.cap / 8)
+            first = std::max(1, std::min(L, static_cast<int>(4.0 * M / avg_leaf)));
+        for (int e2 = first; ; e2 = std::min(L, 8 * e2)) {
+            bounds.push_back(e2);
+            if (e2 >= L) break;
+        }
+    }
+    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], s)) != cudaSuccess) return cuda_fail(e, "invert");
+    launches += 3;
     mark(2);
-    if ((e = ah::launch_invert(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "invert");
-    launches += 2;
-    mark(3);
     if ((e = ah::launch_lut(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "lut");
     launches += 1;
-    mark(4);
+    mark(3);
     if ((e = ah::launch_threshold(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "threshold");
     launches += 1;
-    mark(5);
-    if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
-    launches += 1;
-    mark(6);
+    mark(4);
+    for (size_t p = 0; p + 1 < bounds.size(); ++p) {
+        if (p > 0) {
+            if ((e = ah::launch_tau_update(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "bound refinement");
+            if ((e = ah::launch_invert(dix, a, b, bounds[p], bounds[p + 1], s)) != cudaSuccess)
+                return cuda_fail(e, "invert");
+            launches += 4;
+            mark(6);
+        }
+        a.scan_counter = 0;
+        if ((e = cudaMemsetAsync(b.counters, 0, sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "memset");
+        if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
+        launches += 1;
+        mark(p == 0 ? 5 : 7);
+    }
     if ((e = ah::launch_finish(dix, a, b, 0, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "finish");
     launches += 1;
-    mark(7);
+    mark(8);
     for (int round = 1; round <= 2; ++round) {
         if ((e = ah::launch_redo_scan(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "rescan");
         if ((e = ah::launch_finish(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "finish after rescan");
         launches += 2;
     }
-    mark(8);
+    mark(9);
     if (prof) ix->ev_recorded = true;
     if (tr) {
         const size_t nL = (size_t)nq * L;
@@ -450,6 +491,14 @@ ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
             if (value < 1 || value > 4096) return fail(AH_ERR_INVALID_ARG, "threshold sample outside [1, 4096]");
             ix->opt_threshold_sample = static_cast<int>(value);
             return AH_OK;
+        case AH_OPT_THRESHOLD_LEAVES:
+            if (value < 1 || value > 4096) return fail(AH_ERR_INVALID_ARG, "threshold leaves outside [1, 4096]");
+            ix->opt_threshold_leaves = static_cast<int>(value);
+            return AH_OK;
+        case AH_OPT_PROGRESSIVE_LEAVES:
+            if (value < -1 || value > AH_MAX_LEAVES_SEARCHED) return fail(AH_ERR_INVALID_ARG, "progressive leaves outside [-1, 4096]");
+            ix->opt_progressive_leaves = static_cast<int>(value);
+            return AH_OK;
         case AH_OPT_SCAN_CHUNK_TILES:
             if (value < 0 || value > 1024) return fail(AH_ERR_INVALID_ARG, "scan chunk outside [0, 1024] tiles");
             ix->opt_chunk_tiles = static_cast<int>(value);
@@ -462,7 +511,7 @@ ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
 ah_status ah_set_profiling(ah_index* ix, int32_t on) {
     if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
     if (on && !ix->ev_ready) {
-        for (int i = 0; i <= kStages; ++i) {
+        for (int i = 0; i < ah_index::kMaxMarks; ++i) {
             cudaError_t e = cudaEventCreate(&ix->ev[i]);
             if (e != cudaSuccess) return cuda_fail(e, "event create");
         }
@@ -475,13 +524,18 @@ ah_status ah_set_profiling(ah_index* ix, int32_t on) {
 
 ah_status ah_stage_times(ah_index* ix, float* ms, int32_t max_stages, int32_t* n_stages) {
     if (!ix || !ms || !n_stages) return fail(AH_ERR_INVALID_ARG, "NULL argument");
-    if (!ix->ev_recorded) return fail(AH_ERR_INVALID_ARG, "no profiled search recorded");
-    cudaError_t e = cudaEventSynchronize(ix->ev[kStages]);
+    if (!ix->ev_recorded || ix->n_marks < 2) return fail(AH_ERR_INVALID_ARG, "no profiled search recorded");
+    cudaError_t e = cudaEventSynchronize(ix->ev[ix->n_marks - 1]);
     if (e != cudaSuccess) return cuda_fail(e, "event synchronize");
     int n = std::min<int>(kStages, max_stages);
-    for (int i = 0; i < n; ++i) {
-        e = cudaEventElapsedTime(&ms[i], ix->ev[i], ix->ev[i + 1]);
+    for (int i = 0; i < n; ++i) ms[i] = 0.0f;
+    for (int m = 1; m < ix->n_marks; ++m) {
+        const int st = ix->mark_stage[m];
+        if (st < 0 || st >= n) continue;
+        float t = 0.0f;
+        e = cudaEventElapsedTime(&t, ix->ev[m - 1], ix->ev[m]);
         if (e != cudaSuccess) return cuda_fail(e, "event elapsed");
+        ms[st] += t;
     }
     *n_stages = n;
     return AH_OK;
@@ -524,7 +578,7 @@ void ah_destroy(ah_index* ix) {
     if (ix->ptile) cudaFree(ix->ptile);
     if (ix->err) cudaFree(ix->err);
     if (ix->ev_ready)
-        for (int i = 0; i <= kStages; ++i) cudaEventDestroy(ix->ev[i]);
+        for (int i = 0; i < ah_index::kMaxMarks; ++i) cudaEventDestroy(ix->ev[i]);
     delete ix;
 }
 

@@ -157,8 +157,8 @@ cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, c
 
 constexpr int kSelThreads = 256;
 
-// One CTA per query: best L leaves by (score desc, leaf id asc); counts the
-// queries per leaf and the points the query will scan.
+// One CTA per query: best L leaves by (score desc, leaf id asc), and the
+// points the query will scan.
 __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
@@ -185,7 +185,6 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix,
         int leaf = key_id(key);
         b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
         b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
-        atomicAdd(&b.qcount[leaf], 1);
         local += ix.offs[leaf + 1] - ix.offs[leaf];
     }
     atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
@@ -273,20 +272,35 @@ __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex 
     }
 }
 
-__global__ void invert_scatter_kernel(SearchArgs a, SearchBuffers b) {
+// Queries per leaf over leaf ranks [r0, r1) of every query.
+__global__ void invert_count_kernel(SearchArgs a, SearchBuffers b, int r0, int r1) {
+    const int span = r1 - r0;
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    int64_t total = static_cast<int64_t>(a.nq) * a.L;
-    if (e >= total) return;
-    int q = static_cast<int>(e / a.L);
-    int leaf = b.leaves[e];
-    int pos = atomicAdd(&b.qcursor[leaf], 1);
+    if (e >= static_cast<int64_t>(a.nq) * span) return;
+    const int q = static_cast<int>(e / span), r = r0 + static_cast<int>(e - static_cast<int64_t>(q) * span);
+    atomicAdd(&b.qcount[b.leaves[static_cast<int64_t>(q) * a.L + r]], 1);
+}
+
+__global__ void invert_scatter_kernel(SearchArgs a, SearchBuffers b, int r0, int r1) {
+    const int span = r1 - r0;
+    int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (e >= static_cast<int64_t>(a.nq) * span) return;
+    const int q = static_cast<int>(e / span), r = r0 + static_cast<int>(e - static_cast<int64_t>(q) * span);
+    const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + r];
+    const int pos = atomicAdd(&b.qcursor[leaf], 1);
     b.qlist[b.qoff[leaf] + pos] = q;
 }
 
-cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+// leaf -> query lists (and scan work items) for the leaves of ranks [r0, r1)
+cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
+                          cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * 2 * static_cast<size_t>(ix.nl), s);   // qcount, qcursor
+    if (e != cudaSuccess) return e;
+    const int64_t total = static_cast<int64_t>(a.nq) * (r1 - r0);
+    const unsigned grid = static_cast<unsigned>((total + 255) / 256);
+    invert_count_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
     invert_offsets_kernel<<<1, kScanBlock, 0, s>>>(ix, b, scan_group(a.lut_mode), a.chunk);
-    int64_t total = static_cast<int64_t>(a.nq) * a.L;
-    invert_scatter_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(a, b);
+    invert_scatter_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
     return cudaGetLastError();
 }
 
@@ -468,14 +482,15 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 // threshold: R-th best approximate score over a prefix of the best leaves
 // ---------------------------------------------------------------------------
 
-// Slots sampled per query for the bound: the requested sample, at least R,
-// at most kMaxThresholdSample.
+// Slots sampled per query for the bound: the requested sample, at least 8R
+// (so about R/8 of the sample's points pass), at most kMaxThresholdSample.
 __host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
-    return min(kMaxThresholdSample, max(R, requested));
+    return min(kMaxThresholdSample, max(max(R, requested), 8 * R));
 }
 
-// One CTA per query.  Scores the first M = min(points, threshold_sample) slots of
-// the query's leaves in rank order; the R-th largest (score, id) key among them
+// One CTA per query.  Scores a sample of M = min(points, threshold_sample)
+// slots of the query's best leaves (an even share of the S best, topped up in
+// rank order); the R-th largest (score, id) key among them
 // is a lower bound on the R-th largest over all its leaves (a subset's R-th
 // best can only be lower), so every point of the final top R has a key >= it.
 // With fewer than R points in total the bound is 0 (keep everything).
@@ -491,12 +506,12 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
     load_query_table<MODE>(ix, b, q, lut);
     __syncthreads();
     const int M = threshold_sample(R, a.threshold_sample);
+    // score slots [start, start + m) of the query's leaf of rank i into vals
     int taken = 0;
-    for (int i = 0; i < a.L && taken < M; ++i) {
-        int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
-        int s0 = ix.offs[leaf], sz = ix.offs[leaf + 1] - s0;
-        int p0 = ix.ptile[leaf] * 32;
-        int m = min(sz, M - taken);
+    auto score_range = [&](int i, int start, int m) {
+        const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
+        const int s0 = ix.offs[leaf] + start;
+        const int p0 = ix.ptile[leaf] * 32 + start;
         for (int t0 = 0; t0 < m; t0 += 4 * kSelThreads) {
             int32_t ps[4];
             bool ok[4];
@@ -515,6 +530,19 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
             }
         }
         taken += m;
+    };
+    auto leaf_size = [&](int i) {
+        const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
+        return ix.offs[leaf + 1] - ix.offs[leaf];
+    };
+    // the first M/S slots of each of the S best leaves, then (if short) the
+    // remaining slots of the leaves in rank order
+    const int S = max(1, min(a.L, a.threshold_leaves));
+    const int per = M / S;
+    for (int i = 0; i < S; ++i) score_range(i, 0, min(leaf_size(i), per));
+    for (int i = 0; i < a.L && taken < M; ++i) {
+        const int start = (i < S) ? min(leaf_size(i), per) : 0;
+        score_range(i, start, min(leaf_size(i) - start, M - taken));
     }
     __syncthreads();
     uint64_t tau = 0ull;
@@ -641,7 +669,7 @@ struct TileJob {
 // The warps of a CTA split the item's tiles; a lane owns one slot.  Blocks are
 // summed in order 0..B-1 with IEEE fp32 adds (two queries per packed add), the
 // order every kernel that scores a slot uses.
-template <int G>
+template <int G, int NT>
 __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                                const TileJob& job, const int* s_q, const uint32_t* s_th,
                                                const uint32_t* s_tl) {
@@ -649,7 +677,7 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
     const float2* lut2 = reinterpret_cast<const float2*>(smem);
-    for (int t = job.t0 + warp; t < job.t1; t += kScanThreads / 32) {
+    for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
         const int slot = job.slot_base + 32 * t + lane;
         const bool valid = slot < job.send;
         const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
@@ -678,7 +706,7 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
     }
 }
 
-template <int G>
+template <int G, int NT>
 __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                               const TileJob& job, const int* s_q, const uint32_t* s_th,
                                               const uint32_t* s_tl) {
@@ -686,7 +714,7 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
     const uint32_t* lutw = reinterpret_cast<const uint32_t*>(smem);
-    for (int t = job.t0 + warp; t < job.t1; t += kScanThreads / 32) {
+    for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
         const int slot = job.slot_base + 32 * t + lane;
         const bool valid = slot < job.send;
         const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
@@ -734,9 +762,9 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
 
-template <int MODE>
-__global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(DeviceIndex ix, SearchArgs a,
-                                                                                 SearchBuffers b) {
+template <int MODE, int NT>
+__global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : 1)) scan_kernel(DeviceIndex ix, SearchArgs a,
+                                                                                         SearchBuffers b) {
     constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
     constexpr int GSTEP = (MODE == 0) ? 2 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -749,13 +777,13 @@ __global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(
     int* s_item_off = reinterpret_cast<int*>(smem + lut_bytes);
     const bool off_in_smem = a.scan_item_off_smem != 0;
     if (off_in_smem)
-        for (int i = threadIdx.x; i <= ix.nl; i += kScanThreads) s_item_off[i] = b.item_off[i];
+        for (int i = threadIdx.x; i <= ix.nl; i += NT) s_item_off[i] = b.item_off[i];
     const int* item_off = off_in_smem ? s_item_off : b.item_off;
 
     for (;;) {
         __syncthreads();   // previous item's tables are no longer read
         if (threadIdx.x == 0) {
-            int item = atomicAdd(&b.counters[0], 1);
+            int item = atomicAdd(&b.counters[a.scan_counter], 1);
             s_item = item;
             if (item < total_items) {
                 int lo = 0, hi = ix.nl;
@@ -800,7 +828,7 @@ __global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(
                 const int qa = s_q[2 * pr], qb = s_q[2 * pr + 1];
                 const float* la = b.lut_f32 + static_cast<int64_t>(qa < 0 ? 0 : qa) * per_q;
                 const float* lb = b.lut_f32 + static_cast<int64_t>(qb < 0 ? 0 : qb) * per_q;
-                for (int r = threadIdx.x; r < per_q; r += kScanThreads) {
+                for (int r = threadIdx.x; r < per_q; r += NT) {
                     const float va = (qa >= 0) ? la[r] : 0.0f;
                     const float vb = (qb >= 0) ? lb[r] : 0.0f;
                     lf[((r >> 4) * half + pr) * kCenters + (r & 15)] = make_float2(va, vb);
@@ -819,7 +847,7 @@ __global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(
                     ok[u] = qq >= 0;
                     src[u] = b.lut_u8 + static_cast<int64_t>(ok[u] ? qq : 0) * per_q;
                 }
-                for (int r = threadIdx.x; r < per_q; r += kScanThreads) {
+                for (int r = threadIdx.x; r < per_q; r += NT) {
                     uint32_t v = 0u;
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
@@ -831,17 +859,17 @@ __global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(
         __syncthreads();
         if (MODE == 0) {
             switch (G) {
-                case 8: scan_tiles_f32<8>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 6: scan_tiles_f32<6>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 4: scan_tiles_f32<4>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                default: scan_tiles_f32<2>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 8: scan_tiles_f32<8, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 6: scan_tiles_f32<6, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 4: scan_tiles_f32<4, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                default: scan_tiles_f32<2, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
             }
         } else {
             switch (G) {
-                case 16: scan_tiles_u8<16>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 12: scan_tiles_u8<12>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 8: scan_tiles_u8<8>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                default: scan_tiles_u8<4>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 16: scan_tiles_u8<16, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 12: scan_tiles_u8<12, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 8: scan_tiles_u8<8, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                default: scan_tiles_u8<4, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
             }
         }
     }
@@ -849,7 +877,7 @@ __global__ void __launch_bounds__(kScanThreads, AH_SCAN_MIN_BLOCKS) scan_kernel(
 
 int scan_group(int lut_mode) { return lut_mode == 0 ? kGroupF32 : kGroupU8; }
 
-template <int MODE>
+template <int MODE, int NT>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
     constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
@@ -857,19 +885,83 @@ static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const Sear
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
     a.scan_item_off_smem = (smem + off_bytes <= 200 * 1024 && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE>), smem, true);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT>), smem, true);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE>, kScanThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT>, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    scan_kernel<MODE><<<num_sms * per_sm, kScanThreads, smem, s>>>(ix, a, b);
+    scan_kernel<MODE, NT><<<num_sms * per_sm, NT, smem, s>>>(ix, a, b);
     return cudaGetLastError();
 }
 
+// Wide tables leave room for one CTA per SM: use 1024 threads then.
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s) {
-    if (a.lut_mode == 0) return launch_scan_t<0>(ix, a, b, num_sms, s);
-    return launch_scan_t<1>(ix, a, b, num_sms, s);
+    const size_t table = static_cast<size_t>(ix.B) * (a.lut_mode == 0 ? kGroupF32 * kCenters * 4 : kGroupU8 * kCenters);
+    const bool wide = table > 64 * 1024;
+    if (a.lut_mode == 0) return wide ? launch_scan_t<0, 1024>(ix, a, b, num_sms, s) : launch_scan_t<0, 256>(ix, a, b, num_sms, s);
+    return wide ? launch_scan_t<1, 1024>(ix, a, b, num_sms, s) : launch_scan_t<1, 256>(ix, a, b, num_sms, s);
+}
+
+// ---------------------------------------------------------------------------
+// bound refinement between the two scan phases
+// ---------------------------------------------------------------------------
+
+// One CTA per query, between scan phases: every point of the leaves scanned so
+// far whose key reaches the current bound is in the buffer, so when at least R
+// are there, the R-th best of them is a tighter lower bound on the query's
+// R-th best over all its leaves.  The buffer is then compacted in place to the
+// keys that reach the new bound (order kept; writes only move entries left,
+// and each chunk is read completely before any of it is written).
+__global__ void __launch_bounds__(kSelThreads) tau_update_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    __shared__ SelectScratch scr;
+    __shared__ int s_kept;
+    __shared__ int s_warp[kSelThreads / 32];
+    const int q = blockIdx.x;
+    const int cnt = b.count[q];
+    if (cnt < a.R || cnt > b.cap) return;       // too few to bound, or overflowed (handled after the scan)
+    uint64_t* ck = b.ckey + static_cast<int64_t>(q) * b.cap;
+    int32_t* cs = b.cslot + static_cast<int64_t>(q) * b.cap;
+    auto get = [&](int i) { return ck[i]; };
+    uint64_t t = block_kth_largest<kSelThreads>(get, cnt, a.R, scr);
+    const uint64_t old = b.tau[q];
+    if (t < old) t = old;
+    if (threadIdx.x == 0) {
+        b.tau[q] = t;
+        s_kept = 0;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = 0; base < cnt; base += kSelThreads) {
+        const int i = base + threadIdx.x;
+        const bool in = i < cnt;
+        const uint64_t k = in ? ck[i] : 0ull;
+        const int32_t sl = in ? cs[i] : 0;
+        const bool keep = in && k >= t;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, keep);
+        if (lane == 0) s_warp[warp] = __popc(m);
+        __syncthreads();
+        int before = s_kept;
+        for (int w = 0; w < warp; ++w) before += s_warp[w];
+        if (keep) {
+            const int pos = before + __popc(m & ((1u << lane) - 1u));
+            ck[pos] = k;
+            cs[pos] = sl;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tot = 0;
+            for (int w = 0; w < kSelThreads / 32; ++w) tot += s_warp[w];
+            s_kept += tot;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) b.count[q] = s_kept;
+}
+
+cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    tau_update_kernel<<<a.nq, kSelThreads, 0, s>>>(ix, a, b);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------

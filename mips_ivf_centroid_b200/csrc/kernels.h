@@ -42,8 +42,9 @@ struct SearchBuffers {
     int32_t* cslot;         // [nq][cap] and their slots
     int32_t* count;         // [nq]          (zeroed per search)
     int32_t* redo;          // [2][nq]       queries to rescan after rounds 0 and 1
-    int32_t* counters;      // [8]           (zeroed per search): 0 scan work, 1..2 redo list sizes,
-                            //               3..4 rescan work of rounds 1..2
+    int32_t* counters;      // [8]           (zeroed per search): 0 scan work (first phase), 1..2 redo
+                            //               list sizes, 3..4 rescan work of rounds 1..2, 5 scan work
+                            //               (second phase)
     // per leaf
     int32_t* qcount;        // [NL]          (zeroed per search)
     int32_t* qcursor;       // [NL]          (zeroed per search)
@@ -75,6 +76,8 @@ struct SearchArgs {
     int reorder_vec4;           // set by the finish launcher: 16-byte vector loads allowed
     int reorder_lanes;          // set by the finish launcher: lanes per rescored candidate
     int threshold_sample;       // slots sampled per query for the filter bound (requested)
+    int threshold_leaves;       // best leaves the sample is spread over
+    int scan_counter;           // index into counters[] of the scan's work counter
 };
 
 // Build-time: the leaf-padded tiled code copy.
@@ -83,7 +86,9 @@ cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, in
 
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s);
-cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
+cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
+                          cudaStream_t s);
+cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s);

@@ -210,6 +210,8 @@ class Index:
 
     OPT_THRESHOLD_SAMPLE = 1
     OPT_SCAN_CHUNK_TILES = 2
+    OPT_THRESHOLD_LEAVES = 3
+    OPT_PROGRESSIVE_LEAVES = 4
 
     def set_option(self, option: int, value: int):
         """Tuning knob (ah_set_option): results are unchanged, only speed."""

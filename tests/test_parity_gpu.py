@@ -253,3 +253,21 @@ def test_worked_example_scan_counter(Index):
     assert (tr["scanned"].cpu().numpy() == 100_000).all()
     assert info["points_scanned"] == 4 * 100_000
     assert info["points_scanned"] // 4 * 64 == 6_400_000
+
+
+@pytest.mark.parametrize("lut_mode", [0, 1])
+def test_speed_knobs_do_not_change_results(Index, lut_mode):
+    # progressive bound on/off, sample size and spread, scan chunk: same ids and scores
+    w, X, Q, ix, arr = _workload("sweep-mini")
+    index = Index(ix)
+    qg = torch.from_numpy(Q).cuda()
+    ref = index.search(qg, 10, 64, 100, lut_mode)
+    for opt, val in [(Index.OPT_PROGRESSIVE_LEAVES, -1), (Index.OPT_PROGRESSIVE_LEAVES, 3),
+                     (Index.OPT_THRESHOLD_SAMPLE, 64), (Index.OPT_THRESHOLD_LEAVES, 8),
+                     (Index.OPT_SCAN_CHUNK_TILES, 3)]:
+        index.set_option(opt, val)
+        got = index.search(qg, 10, 64, 100, lut_mode)
+        torch.testing.assert_close(got[0], ref[0], rtol=0, atol=0)
+        torch.testing.assert_close(got[1], ref[1], rtol=0, atol=0)
+    index.sync_status()
+    index.close()
