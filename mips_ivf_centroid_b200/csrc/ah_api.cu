@@ -240,10 +240,6 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     mark(-1);
     if ((e = ah::launch_centroid_scores(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "centroid scores");
     launches += 1;
-    mark(0);
-    if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
-    launches += 1;
-    mark(1);
     // Scan phases over leaf ranks [bounds[p], bounds[p+1]).  One phase when
     // the bound from the sample is expected to keep few points; otherwise the
     // first phase is small enough for that bound, each later phase covers up
@@ -263,8 +259,13 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
             if (e2 >= L) break;
         }
     }
-    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], s)) != cudaSuccess) return cuda_fail(e, "invert");
-    launches += 3;
+    mark(0);
+    a.count_ranks = bounds[1];
+    if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
+    launches += 1;
+    mark(1);
+    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], true, s)) != cudaSuccess) return cuda_fail(e, "invert");
+    launches += 2;
     mark(2);
     if ((e = ah::launch_lut(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "lut");
     launches += 1;
@@ -275,7 +276,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     for (size_t p = 0; p + 1 < bounds.size(); ++p) {
         if (p > 0) {
             if ((e = ah::launch_tau_update(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "bound refinement");
-            if ((e = ah::launch_invert(dix, a, b, bounds[p], bounds[p + 1], s)) != cudaSuccess)
+            if ((e = ah::launch_invert(dix, a, b, bounds[p], bounds[p + 1], false, s)) != cudaSuccess)
                 return cuda_fail(e, "invert");
             launches += 4;
             mark(6);

@@ -98,23 +98,27 @@ cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, in
 // partitioning: centroid scores and top-L leaves
 // ---------------------------------------------------------------------------
 
-constexpr int kGemmBM = 64, kGemmBN = 64, kGemmBK = 16;
+constexpr int kGemmBK = 16;
 
-// S[q][c] = sum_t Q[q][t] * C[c][t]  (fp32, SIMT; 64x64 tile, 4x4 per thread)
+// S[q][c] = sum_t Q[q][t] * C[c][t]  (fp32, SIMT; TM x TM tile, 16x16 threads,
+// (TM/16)^2 outputs per thread)
+template <int TM>
 __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __restrict__ Q, const float* __restrict__ C,
                                                               float* __restrict__ S, int nq, int nl, int d) {
-    __shared__ float As[kGemmBK][kGemmBM + 4];
-    __shared__ float Bs[kGemmBK][kGemmBN + 4];
+    constexpr int PT = TM / 16;              // outputs per thread per dimension
+    constexpr int LOADS = TM * kGemmBK / 256;
+    __shared__ float As[kGemmBK][TM + 4];
+    __shared__ float Bs[kGemmBK][TM + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * kGemmBN;
-    float acc[4][4];
+    const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TM;
+    float acc[PT][PT];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < PT; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+        for (int j = 0; j < PT; ++j) acc[i][j] = 0.0f;
     for (int k0 = 0; k0 < d; k0 += kGemmBK) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < LOADS; ++r) {
             int e = threadIdx.x + 256 * r;
             int row = e >> 4, col = e & 15;
             int gk = k0 + col;
@@ -125,40 +129,48 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __res
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < kGemmBK; ++kk) {
-            float a[4], b[4];
+            float av[PT], bv[PT];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+            for (int i = 0; i < PT; ++i) av[i] = As[kk][ty + 16 * i];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+            for (int j = 0; j < PT; ++j) bv[j] = Bs[kk][tx + 16 * j];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < PT; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < PT; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < PT; ++i) {
         int gm = m0 + ty + 16 * i;
         if (gm >= nq) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < PT; ++j) {
             int gn = n0 + tx + 16 * j;
             if (gn < nl) S[static_cast<int64_t>(gm) * nl + gn] = acc[i][j];
         }
     }
 }
 
+// 64x64 tiles, 32x32 for very small problems (more CTAs in flight).
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
-    dim3 grid((ix.nl + kGemmBN - 1) / kGemmBN, (a.nq + kGemmBM - 1) / kGemmBM);
-    centroid_scores_kernel<<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+    const int64_t big = static_cast<int64_t>((ix.nl + 63) / 64) * ((a.nq + 63) / 64);
+    if (big >= 64) {
+        dim3 grid((ix.nl + 63) / 64, (a.nq + 63) / 64);
+        centroid_scores_kernel<64><<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+    } else {
+        dim3 grid((ix.nl + 31) / 32, (a.nq + 31) / 32);
+        centroid_scores_kernel<32><<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+    }
     return cudaGetLastError();
 }
 
 constexpr int kSelThreads = 256;
 
-// One CTA per query: best L leaves by (score desc, leaf id asc), and the
-// points the query will scan.
+// One CTA per query: best L leaves by (score desc, leaf id asc), the points
+// the query will scan, and (for leaf ranks below count_ranks) the queries per
+// leaf of the first scan phase.
 __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
@@ -185,6 +197,7 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix,
         int leaf = key_id(key);
         b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
         b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
+        if (i < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);     // queries per leaf, first scan phase
         local += ix.offs[leaf + 1] - ix.offs[leaf];
     }
     atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
@@ -205,7 +218,82 @@ static cudaError_t launch_top_leaves_block(const DeviceIndex& ix, SearchArgs a, 
 
 constexpr int kWarpMaxK = 256;          // warp-cooperative selection up to this K
 
+// The K = min(K, n) largest of n <= 4*NT staged keys (and payloads) through
+// registers: block_kth_reg finds the K-th key, the keys at or above it are
+// gathered (atomic positions; sorted descending when `sort`, padding key 0 up
+// to next_pow2(K)).  Returns K on every thread.
+template <int NT>
+__device__ int block_topk_reg(const uint64_t* keys, const int32_t* vals, int n, int K, RegSelectScratch<NT>& rs,
+                              int* counter, uint64_t* out_k, int32_t* out_v, bool sort) {
+    constexpr int KPL = 4;
+    uint64_t kk[KPL];
+    int32_t vv[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const int i = threadIdx.x + NT * j;
+        kk[j] = (i < n) ? keys[i] : 0ull;
+        vv[j] = (i < n && vals) ? vals[i] : -1;
+    }
+    if (K > n) K = n;
+    if (K <= 0) return 0;
+    if (threadIdx.x == 0) *counter = 0;
+    const uint64_t thr = (K < n) ? block_kth_reg<KPL, NT>(kk, n, K, rs) : 1ull;
+    if (K >= n) __syncthreads();
+    const int P2 = next_pow2(K);
+    for (int i = K + threadIdx.x; i < P2; i += NT) {
+        out_k[i] = 0ull;
+        if (out_v) out_v[i] = -1;
+    }
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        if (kk[j] != 0ull && kk[j] >= thr) {
+            const int pos = atomicAdd(counter, 1);
+            out_k[pos] = kk[j];
+            if (out_v) out_v[pos] = vv[j];
+        }
+    }
+    __syncthreads();
+    if (sort) block_sort_desc<NT>(out_k, out_v, P2);
+    return K;
+}
+
+constexpr int kTopWarps = 8;
+
+// One warp per query when the centroids fit 32 per lane: the scores stay in
+// registers and the selection needs no shared-memory passes.
+__global__ void __launch_bounds__(kTopWarps * 32) top_leaves_warp_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = blockIdx.x * kTopWarps + warp;
+    if (q >= a.nq) return;
+    const int L = a.L, nl = ix.nl, P2 = next_pow2(L);
+    uint64_t* keys = reinterpret_cast<uint64_t*>(smem) + static_cast<size_t>(warp) * P2;
+    const float* row = b.cscore + static_cast<int64_t>(q) * nl;
+    auto get = [&](int i) { return make_key(float_key(row[i]), i); };
+    auto pay = [&](int i) { return i; };
+    warp_topk_reg<32>(get, pay, nl, L, keys, nullptr, true);
+    long long local = 0;
+    for (int i = lane; i < L; i += 32) {
+        const uint64_t key = keys[i];
+        const int leaf = key_id(key);
+        b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
+        b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
+        if (i < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);
+        local += ix.offs[leaf + 1] - ix.offs[leaf];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, off);
+    if (lane == 0) b.scanned[q] = local;
+}
+
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+    if (ix.nl <= 32 * 32 && a.L <= kWarpMaxK) {
+        const size_t smem = static_cast<size_t>(kTopWarps) * next_pow2(a.L) * sizeof(uint64_t);
+        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_warp_kernel), smem, false);
+        if (e != cudaSuccess) return e;
+        top_leaves_warp_kernel<<<(a.nq + kTopWarps - 1) / kTopWarps, kTopWarps * 32, smem, s>>>(ix, a, b);
+        return cudaGetLastError();
+    }
     return launch_top_leaves_block(ix, a, b, s);
 }
 
@@ -292,13 +380,16 @@ __global__ void invert_scatter_kernel(SearchArgs a, SearchBuffers b, int r0, int
 }
 
 // leaf -> query lists (and scan work items) for the leaves of ranks [r0, r1)
+// (counted: the queries per leaf are already in qcount and qcursor is zero)
 cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
-                          cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * 2 * static_cast<size_t>(ix.nl), s);   // qcount, qcursor
-    if (e != cudaSuccess) return e;
+                          bool counted, cudaStream_t s) {
     const int64_t total = static_cast<int64_t>(a.nq) * (r1 - r0);
     const unsigned grid = static_cast<unsigned>((total + 255) / 256);
-    invert_count_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
+    if (!counted) {
+        cudaError_t e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * 2 * static_cast<size_t>(ix.nl), s);   // qcount, qcursor
+        if (e != cudaSuccess) return e;
+        invert_count_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
+    }
     invert_offsets_kernel<<<1, kScanBlock, 0, s>>>(ix, b, scan_group(a.lut_mode), a.chunk);
     invert_scatter_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
     return cudaGetLastError();
@@ -498,6 +589,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
+    __shared__ RegSelectScratch<kSelThreads> rs;
     const int q = blockIdx.x;
     const int R = a.R;
     unsigned char* lut = smem;
@@ -545,12 +637,24 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
         score_range(i, start, min(leaf_size(i) - start, M - taken));
     }
     __syncthreads();
-    uint64_t tau = 0ull;
-    if (taken >= R) {
+    if (taken <= 4 * kSelThreads) {
+        uint64_t tau = 0ull;
+        if (taken >= R) {
+            uint64_t kk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = threadIdx.x + kSelThreads * j;
+                kk[j] = (i < taken) ? vals[i] : 0ull;
+            }
+            tau = block_kth_reg<4, kSelThreads>(kk, taken, R, rs);
+        }
+        if (threadIdx.x == 0) b.tau[q] = tau;
+    } else {
         auto get = [&](int i) { return vals[i]; };
-        tau = block_kth_largest<kSelThreads>(get, taken, R, scr);
+        uint64_t tau = 0ull;
+        if (taken >= R) tau = block_kth_largest<kSelThreads>(get, taken, R, scr);
+        if (threadIdx.x == 0) b.tau[q] = tau;
     }
-    if (threadIdx.x == 0) b.tau[q] = tau;
     (void)top;
 }
 
@@ -915,6 +1019,7 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
 // and each chunk is read completely before any of it is written).
 __global__ void __launch_bounds__(kSelThreads) tau_update_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     __shared__ SelectScratch scr;
+    __shared__ RegSelectScratch<kSelThreads> rs;
     __shared__ int s_kept;
     __shared__ int s_warp[kSelThreads / 32];
     const int q = blockIdx.x;
@@ -923,7 +1028,18 @@ __global__ void __launch_bounds__(kSelThreads) tau_update_kernel(DeviceIndex ix,
     uint64_t* ck = b.ckey + static_cast<int64_t>(q) * b.cap;
     int32_t* cs = b.cslot + static_cast<int64_t>(q) * b.cap;
     auto get = [&](int i) { return ck[i]; };
-    uint64_t t = block_kth_largest<kSelThreads>(get, cnt, a.R, scr);
+    uint64_t t;
+    if (cnt <= 4 * kSelThreads) {
+        uint64_t kk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = threadIdx.x + kSelThreads * j;
+            kk[j] = (i < cnt) ? ck[i] : 0ull;
+        }
+        t = block_kth_reg<4, kSelThreads>(kk, cnt, a.R, rs);
+    } else {
+        t = block_kth_largest<kSelThreads>(get, cnt, a.R, scr);
+    }
     const uint64_t old = b.tau[q];
     if (t < old) t = old;
     if (threadIdx.x == 0) {
@@ -1049,7 +1165,8 @@ size_t finish_smem_bytes(int R, int d) {
 //     keeps the best k by (exact score, id).
 template <int MODE>
 __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, int q,
-                             unsigned char* smem, SelectScratch& scr) {
+                             unsigned char* smem, SelectScratch& scr,
+                             RegSelectScratch<kFinishThreads>& rs) {
     const int cap = b.cap, R = a.R, k = a.k, d = ix.d;
     const int P2 = next_pow2(R);
     uint64_t* skeys = reinterpret_cast<uint64_t*>(smem);            // [kStageCap]
@@ -1096,8 +1213,10 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         // only the keys that reach it.
         for (int i = threadIdx.x; i < kStageCap; i += kFinishThreads) skeys[i] = ck[i];
         __syncthreads();
-        auto sget = [&](int i) { return skeys[i]; };
-        const uint64_t bound = block_kth_largest<kFinishThreads>(sget, kStageCap, R, scr);
+        uint64_t sk[kStageCap / kFinishThreads];
+#pragma unroll
+        for (int j = 0; j < kStageCap / kFinishThreads; ++j) sk[j] = skeys[threadIdx.x + kFinishThreads * j];
+        const uint64_t bound = block_kth_reg<kStageCap / kFinishThreads, kFinishThreads>(sk, kStageCap, R, rs);
         if (threadIdx.x == 0) scr.count = 0;
         __syncthreads();
         constexpr int U = 4;
@@ -1124,7 +1243,9 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         if (scr.count <= kStageCap) staged = scr.count;
         __syncthreads();
     }
-    if (staged >= 0) {
+    if (staged >= 0 && staged <= 4 * kFinishThreads) {
+        K = block_topk_reg<kFinishThreads>(skeys, sslots, staged, R, rs, &scr.count, okeys, oslots, sorted);
+    } else if (staged >= 0) {
         auto get = [&](int i) { return skeys[i]; };
         auto pay = [&](int i) { return sslots[i]; };
         K = block_topk<kFinishThreads>(get, pay, staged, R, scr, okeys, oslots, b.err, sorted);
@@ -1207,7 +1328,8 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
     auto epay = [&](int i) { return i; };
     if (k <= kWarpMaxK) {
         if (threadIdx.x < 32) {
-            const int Kk = warp_topk(eget, epay, K, k, whist, okeys, nullptr);
+            const int Kk = (K <= 32 * 4) ? warp_topk_reg<4>(eget, epay, K, k, okeys, nullptr, true)
+                                         : warp_topk(eget, epay, K, k, whist, okeys, nullptr);
             for (int i = threadIdx.x; i < k; i += 32) {
                 const bool have = i < Kk;
                 a.out_ids[oo + i] = have ? key_id(okeys[i]) : -1;
@@ -1228,14 +1350,15 @@ template <int MODE>
 __global__ void __launch_bounds__(kFinishThreads, 6) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
+    __shared__ RegSelectScratch<kFinishThreads> rs;
     if (round == 0) {
-        finish_query<MODE>(ix, a, b, 0, blockIdx.x, smem, scr);
+        finish_query<MODE>(ix, a, b, 0, blockIdx.x, smem, scr, rs);
         return;
     }
     // rescan rounds: a small grid walks the previous round's redo list
     const int n = b.counters[round];
     for (int e = blockIdx.x; e < n; e += gridDim.x) {
-        finish_query<MODE>(ix, a, b, round, b.redo[static_cast<int64_t>(round - 1) * a.nq + e], smem, scr);
+        finish_query<MODE>(ix, a, b, round, b.redo[static_cast<int64_t>(round - 1) * a.nq + e], smem, scr, rs);
         __syncthreads();
     }
 }

@@ -78,6 +78,7 @@ struct SearchArgs {
     int threshold_sample;       // slots sampled per query for the filter bound (requested)
     int threshold_leaves;       // best leaves the sample is spread over
     int scan_counter;           // index into counters[] of the scan's work counter
+    int count_ranks;            // top-L kernel counts queries per leaf for ranks below this
 };
 
 // Build-time: the leaf-padded tiled code copy.
@@ -87,7 +88,7 @@ cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, in
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
-                          cudaStream_t s);
+                          bool counted, cudaStream_t s);
 cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);

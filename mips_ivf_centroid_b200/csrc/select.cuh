@@ -412,3 +412,213 @@ __device__ uint64_t warp_kth_largest(GetKey get, int n, int K, int* hist) {
 }
 
 }  // namespace ah
+
+// ---------------------------------------------------------------------------
+// Register-resident warp selection: each lane holds up to KPL keys in
+// registers (unused entries hold 0, which no real key equals or undercuts:
+// real keys have a nonzero score part).  Radix selection one bit at a time:
+// per bit every lane counts its keys in the candidate bucket and the warp sums
+// the counts, so there are no shared-memory passes and no block barriers.
+// ---------------------------------------------------------------------------
+namespace ah {
+
+// The K-th largest of the warp's keys (1 <= K <= number of real keys); all
+// lanes return it.
+template <int KPL>
+__device__ uint64_t warp_kth_reg(const uint64_t (&k)[KPL], int K) {
+    // bits every real key shares are skipped
+    uint64_t kand = ~0ull, kor = 0ull;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        if (k[j] != 0ull) kand &= k[j];
+        kor |= k[j];
+    }
+    kand = warp_and64(kand);
+    kor = warp_or64(kor);
+    const uint64_t diff = kand ^ kor;
+    if (diff == 0ull) return kor;                       // one distinct real key
+    const int top = 63 - __clzll(static_cast<long long>(diff));
+    uint64_t prefix = (top >= 63) ? 0ull : (kand & (~0ull << (top + 1)));
+    int need = K;
+    for (int bit = top; bit >= 0; --bit) {
+        const uint64_t hm = ~0ull << bit;               // bits >= bit
+        const uint64_t cand = prefix | (1ull << bit);
+        int c = 0, in_low = 0;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+            const uint64_t m = k[j] & hm;
+            c += (m == cand);
+            in_low += (m == prefix);
+        }
+        c = __reduce_add_sync(0xFFFFFFFFu, c);
+        in_low = __reduce_add_sync(0xFFFFFFFFu, in_low);
+        if (c >= need) {
+            prefix = cand;
+            if (c == need) break;                       // the bucket is exactly the rest
+        } else {
+            need -= c;
+            if (in_low == need) break;                  // keys with this bit clear are exactly the rest
+        }
+    }
+    // the K-th largest is the smallest key in the final bucket
+    uint64_t mn = ~0ull;
+    const int bits_left = 0;
+    (void)bits_left;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j)
+        if (k[j] >= prefix && k[j] != 0ull && k[j] < mn) mn = k[j];
+    const unsigned hi = __reduce_min_sync(0xFFFFFFFFu, static_cast<unsigned>(mn >> 32));
+    const unsigned lo = __reduce_min_sync(0xFFFFFFFFu, (static_cast<unsigned>(mn >> 32) == hi)
+                                                           ? static_cast<unsigned>(mn) : 0xFFFFFFFFu);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+}  // namespace ah
+
+namespace ah {
+
+// Compact the warp's keys >= thr (and payloads) to out_k/out_v; returns the
+// count.  Order: register slot j, then lane.
+template <int KPL>
+__device__ __forceinline__ int warp_gather_ge(const uint64_t (&k)[KPL], const int32_t (&v)[KPL], uint64_t thr,
+                                              uint64_t* out_k, int32_t* out_v) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const bool sel = k[j] != 0ull && k[j] >= thr;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            out_k[pos] = k[j];
+            if (out_v) out_v[pos] = v[j];
+        }
+        base += __popc(m);
+    }
+    __syncwarp();
+    return base;
+}
+
+// The K = min(K, n) largest of n <= 32*KPL keys read by get(i) (payload pay(i)),
+// by one warp through registers; written to out_k/out_v (capacity
+// next_pow2(K)), sorted descending if `sort` (padding key 0).  Returns K.
+template <int KPL, class GetKey, class GetVal>
+__device__ int warp_topk_reg(GetKey get, GetVal pay, int n, int K, uint64_t* out_k, int32_t* out_v, bool sort) {
+    const int lane = threadIdx.x & 31;
+    uint64_t k[KPL];
+    int32_t v[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const int i = lane + 32 * j;
+        k[j] = (i < n) ? get(i) : 0ull;
+        v[j] = (i < n && out_v) ? pay(i) : -1;
+    }
+    if (K > n) K = n;
+    if (K <= 0) return 0;
+    const uint64_t thr = (K < n) ? warp_kth_reg<KPL>(k, K) : 1ull;
+    const int P2 = next_pow2(K);
+    for (int i = K + lane; i < P2; i += 32) {
+        out_k[i] = 0ull;
+        if (out_v) out_v[i] = -1;
+    }
+    warp_gather_ge<KPL>(k, v, thr, out_k, out_v);
+    if (sort) warp_sort_desc(out_k, out_v, P2);
+    return K;
+}
+
+}  // namespace ah
+
+namespace ah {
+
+// Scratch for block_kth_reg: per-warp partial counts, double-buffered by bit
+// parity so one barrier per bit suffices, plus the and/or/min exchange.
+template <int NT>
+struct RegSelectScratch {
+    int part[2][NT / 32];
+    unsigned long long w64[NT / 32];
+    unsigned long long w64b[NT / 32];
+};
+
+template <int NT>
+__device__ __forceinline__ int block_sum_parity(int v, RegSelectScratch<NT>& s, int parity) {
+    v = __reduce_add_sync(0xFFFFFFFFu, v);
+    if ((threadIdx.x & 31) == 0) s.part[parity][threadIdx.x >> 5] = v;
+    __syncthreads();
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) t += s.part[parity][w];
+    return t;
+}
+
+// K-th largest of the block's register-held keys (KPL per thread, key 0 =
+// empty, n > 0 real keys in total, 1 <= K <= n).  Bitwise radix from the
+// highest bit where the keys differ; a bit's step counts the keys of the
+// current bucket that have the bit set (one warp reduction and one barrier).
+// The running bucket size makes the count of the other half free, and the
+// walk stops as soon as the bucket holding the K-th key is exactly the
+// remainder, whose minimum is then the answer.  Every thread returns it.
+template <int KPL, int NT>
+__device__ uint64_t block_kth_reg(const uint64_t (&k)[KPL], int n, int K, RegSelectScratch<NT>& s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t kand = ~0ull, kor = 0ull;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        if (k[j] != 0ull) kand &= k[j];
+        kor |= k[j];
+    }
+    kand = warp_and64(kand);
+    kor = warp_or64(kor);
+    if (lane == 0) {
+        s.w64[warp] = kand;
+        s.w64b[warp] = kor;
+    }
+    __syncthreads();
+    kand = ~0ull;
+    kor = 0ull;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        kand &= s.w64[w];
+        kor |= s.w64b[w];
+    }
+    __syncthreads();  // s.w64 is reused for the minimum below
+    const uint64_t diff = kand ^ kor;
+    if (diff == 0ull) return kor;  // all keys equal
+    const int top = 63 - __clzll(diff);
+    uint64_t prefix = (top >= 63) ? 0ull : (kand & (~0ull << (top + 1)));
+    int need = K, in_bucket = n, parity = 0;
+    for (int bit = top; bit >= 0; --bit) {
+        const uint64_t hm = ~0ull << bit;
+        const uint64_t cand = prefix | (1ull << bit);
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) c += ((k[j] & hm) == cand) ? 1 : 0;
+        c = block_sum_parity<NT>(c, s, parity);
+        parity ^= 1;
+        if (c >= need) {
+            prefix = cand;
+            in_bucket = c;
+        } else {
+            need -= c;
+            in_bucket -= c;
+        }
+        if (in_bucket == need) break;
+    }
+    uint64_t mn = ~0ull;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j)
+        if (k[j] != 0ull && k[j] >= prefix && k[j] < mn) mn = k[j];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, mn, off);
+        mn = o < mn ? o : mn;
+    }
+    if (lane == 0) s.w64[warp] = mn;
+    __syncthreads();
+    mn = ~0ull;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) mn = s.w64[w] < mn ? s.w64[w] : mn;
+    __syncthreads();
+    return mn;
+}
+
+}  // namespace ah
