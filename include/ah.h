@@ -228,7 +228,10 @@ AH_API ah_status ah_sync_status(ah_index *ix, void *cuda_stream);
  * Stage timing.  With profiling on, each search records CUDA events around its
  * stages on the search stream; ah_stage_times() synchronises on the last
  * event and writes up to max_stages durations in milliseconds (stage order as
- * ah_stage_name(i)), setting *n_stages.  Synchronous.
+ * ah_stage_name(i)), setting *n_stages.  Synchronous.  on: 0 off, 1 every
+ * stage, 2 the scan phases only (the other stages read 0; the kernels before
+ * and after the scan then keep their overlapped launches).  Other values:
+ * AH_ERR_INVALID_ARG.
  */
 AH_API ah_status ah_set_profiling(ah_index *ix, int32_t on);
 AH_API ah_status ah_stage_times(ah_index *ix, float *ms, int32_t max_stages, int32_t *n_stages);

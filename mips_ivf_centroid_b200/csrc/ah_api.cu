@@ -65,7 +65,7 @@ struct ah_index {
     int* err = nullptr;
     size_t owned_bytes = 0;
     Workspace ws;
-    bool profiling = false;
+    int profiling = 0;               // 0 off, 1 every stage, 2 scan phases only
     static constexpr int kMaxMarks = 64;
     cudaEvent_t ev[kMaxMarks]{};
     int mark_stage[kMaxMarks]{};      // stage ending at mark i (-1: none)
@@ -229,8 +229,10 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     cudaError_t e;
     // mark(stage): the interval since the previous mark belongs to `stage`
     ix->n_marks = 0;
+    // level 2 marks only the scan phases (stages 4..7: the first such mark
+    // opens the interval), so the rest of the kernel chain runs unbroken
     auto mark = [&](int stage) {
-        if (prof && ix->n_marks < ah_index::kMaxMarks) {
+        if (prof && ix->n_marks < ah_index::kMaxMarks && (ix->profiling == 1 || (stage >= 4 && stage <= 7))) {
             ix->mark_stage[ix->n_marks] = stage;
             cudaEventRecord(ix->ev[ix->n_marks++], s);
         }
@@ -518,7 +520,8 @@ ah_status ah_set_profiling(ah_index* ix, int32_t on) {
         }
         ix->ev_ready = true;
     }
-    ix->profiling = on != 0;
+    if (on < 0 || on > 2) return fail(AH_ERR_INVALID_ARG, "profiling level must be 0, 1 or 2");
+    ix->profiling = on;
     ix->ev_recorded = false;
     return AH_OK;
 }

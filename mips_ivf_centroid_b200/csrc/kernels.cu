@@ -21,6 +21,7 @@
 #include <cstdint>
 #include <mutex>
 #include <unordered_map>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -48,6 +49,36 @@ static cudaError_t ensure_smem(const void* kernel, size_t bytes, bool max_carveo
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) g_attr_smem[key] = static_cast<int>(bytes);
     return e;
+}
+
+
+// Programmatic dependent launch.  The search kernels form one chain on a
+// stream; each is launched with the programmatic-serialization attribute, so
+// its CTAs may be scheduled while the previous kernel drains, and its first
+// action is to wait until that kernel has finished and its writes are
+// visible (a no-op when the previous operation was not a kernel launched
+// this way).  Each kernel then lets the next one launch; that next kernel
+// waits the same way before reading anything, so every kernel still sees all
+// earlier results.
+__device__ __forceinline__ void chain_entry() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------
@@ -105,6 +136,7 @@ constexpr int kGemmBK = 16;
 template <int TM>
 __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __restrict__ Q, const float* __restrict__ C,
                                                               float* __restrict__ S, int nq, int nl, int d) {
+    chain_entry();
     constexpr int PT = TM / 16;              // outputs per thread per dimension
     constexpr int LOADS = TM * kGemmBK / 256;
     __shared__ float As[kGemmBK][TM + 4];
@@ -158,20 +190,27 @@ cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, c
     const int64_t big = static_cast<int64_t>((ix.nl + 63) / 64) * ((a.nq + 63) / 64);
     if (big >= 64) {
         dim3 grid((ix.nl + 63) / 64, (a.nq + 63) / 64);
-        centroid_scores_kernel<64><<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+        if (const cudaError_t le = launch_chained(centroid_scores_kernel<64>, dim3(grid), dim3(256), 0, s, a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d); le != cudaSuccess) return le;
     } else {
         dim3 grid((ix.nl + 31) / 32, (a.nq + 31) / 32);
-        centroid_scores_kernel<32><<<grid, 256, 0, s>>>(a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+        if (const cudaError_t le = launch_chained(centroid_scores_kernel<32>, dim3(grid), dim3(256), 0, s, a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
 
+#ifndef AH_REORDER_BATCH
+#define AH_REORDER_BATCH 4
+#endif
+#ifndef AH_FINISH_MIN_BLOCKS
+#define AH_FINISH_MIN_BLOCKS 6
+#endif
 constexpr int kSelThreads = 256;
 
 // One CTA per query: best L leaves by (score desc, leaf id asc), the points
 // the query will scan, and (for leaf ranks below count_ranks) the queries per
 // leaf of the first scan phase.
 __global__ void __launch_bounds__(kSelThreads) top_leaves_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     __shared__ long long s_scanned;
@@ -212,27 +251,26 @@ static cudaError_t launch_top_leaves_block(const DeviceIndex& ix, SearchArgs a, 
     if (a.topl_row_smem) smem += row;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_kernel), smem, true);
     if (e != cudaSuccess) return e;
-    top_leaves_kernel<<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+    if (const cudaError_t le = launch_chained(top_leaves_kernel, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
 constexpr int kWarpMaxK = 256;          // warp-cooperative selection up to this K
 
-// The K = min(K, n) largest of n <= 4*NT staged keys (and payloads) through
-// registers: block_kth_reg finds the K-th key, the keys at or above it are
-// gathered (atomic positions; sorted descending when `sort`, padding key 0 up
-// to next_pow2(K)).  Returns K on every thread.
-template <int NT>
-__device__ int block_topk_reg(const uint64_t* keys, const int32_t* vals, int n, int K, RegSelectScratch<NT>& rs,
-                              int* counter, uint64_t* out_k, int32_t* out_v, bool sort) {
-    constexpr int KPL = 4;
+// The K = min(K, n) largest of n <= KPL*NT keys read by get(i) (payload
+// pay(i)) through registers: block_kth_reg finds the K-th key, the keys at or
+// above it are gathered (atomic positions; sorted descending when `sort`,
+// padding key 0 up to next_pow2(K)).  Returns K on every thread.
+template <int KPL, int NT, class GetKey, class GetVal>
+__device__ int block_topk_reg(GetKey get, GetVal pay, int n, int K, RegSelectScratch<NT>& rs, int* counter,
+                              uint64_t* out_k, int32_t* out_v, bool sort) {
     uint64_t kk[KPL];
     int32_t vv[KPL];
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
         const int i = threadIdx.x + NT * j;
-        kk[j] = (i < n) ? keys[i] : 0ull;
-        vv[j] = (i < n && vals) ? vals[i] : -1;
+        kk[j] = (i < n) ? get(i) : 0ull;
+        vv[j] = (i < n && out_v) ? pay(i) : -1;
     }
     if (K > n) K = n;
     if (K <= 0) return 0;
@@ -257,11 +295,44 @@ __device__ int block_topk_reg(const uint64_t* keys, const int32_t* vals, int n, 
     return K;
 }
 
+// One CTA per query with the score row in registers (KPL per thread): for
+// 1024 < centroids <= KPL * 256.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads) top_leaves_reg_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ RegSelectScratch<kSelThreads> rs;
+    __shared__ int s_count;
+    __shared__ long long s_scanned;
+    const int q = blockIdx.x;
+    const int L = a.L, nl = ix.nl;
+    uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
+    const float* row = b.cscore + static_cast<int64_t>(q) * nl;
+    auto get = [&](int i) { return make_key(float_key(row[i]), i); };
+    auto pay = [&](int i) { return i; };
+    if (threadIdx.x == 0) s_scanned = 0;
+    block_topk_reg<KPL, kSelThreads>(get, pay, nl, L, rs, &s_count, keys, static_cast<int32_t*>(nullptr), true);
+    long long local = 0;
+    for (int i = threadIdx.x; i < L; i += kSelThreads) {
+        const uint64_t key = keys[i];
+        const int leaf = key_id(key);
+        b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
+        b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
+        if (i < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);
+        local += ix.offs[leaf + 1] - ix.offs[leaf];
+    }
+    atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
+    __syncthreads();
+    if (threadIdx.x == 0) b.scanned[q] = s_scanned;
+}
+
+constexpr int kReorderBatch = AH_REORDER_BATCH;
 constexpr int kTopWarps = 8;
 
 // One warp per query when the centroids fit 32 per lane: the scores stay in
 // registers and the selection needs no shared-memory passes.
 __global__ void __launch_bounds__(kTopWarps * 32) top_leaves_warp_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = blockIdx.x * kTopWarps + warp;
@@ -291,7 +362,19 @@ cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchB
         const size_t smem = static_cast<size_t>(kTopWarps) * next_pow2(a.L) * sizeof(uint64_t);
         cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_warp_kernel), smem, false);
         if (e != cudaSuccess) return e;
-        top_leaves_warp_kernel<<<(a.nq + kTopWarps - 1) / kTopWarps, kTopWarps * 32, smem, s>>>(ix, a, b);
+        if (const cudaError_t le = launch_chained(top_leaves_warp_kernel, dim3((a.nq + kTopWarps - 1) / kTopWarps), dim3(kTopWarps * 32), smem, s, ix, a, b); le != cudaSuccess) return le;
+        return cudaGetLastError();
+    }
+    if (ix.nl <= 16 * kSelThreads) {
+        const size_t smem = static_cast<size_t>(next_pow2(a.L)) * sizeof(uint64_t);
+        const void* fn = (ix.nl <= 8 * kSelThreads) ? reinterpret_cast<const void*>(top_leaves_reg_kernel<8>)
+                                                    : reinterpret_cast<const void*>(top_leaves_reg_kernel<16>);
+        cudaError_t e = ensure_smem(fn, smem, false);
+        if (e != cudaSuccess) return e;
+        const cudaError_t le = (ix.nl <= 8 * kSelThreads)
+            ? launch_chained(top_leaves_reg_kernel<8>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b)
+            : launch_chained(top_leaves_reg_kernel<16>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b);
+        if (le != cudaSuccess) return le;
         return cudaGetLastError();
     }
     return launch_top_leaves_block(ix, a, b, s);
@@ -333,6 +416,7 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, 
 // Single CTA: qoff = exclusive scan of queries per leaf; item_off = exclusive
 // scan of work items per leaf (query groups x chunks of `chunk` code tiles).
 __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex ix, SearchBuffers b, int group, int chunk) {
+    chain_entry();
     __shared__ int warp_sums[32];
     __shared__ int total_q, total_i;
     int carry_q = 0, carry_i = 0;
@@ -362,6 +446,7 @@ __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex 
 
 // Queries per leaf over leaf ranks [r0, r1) of every query.
 __global__ void invert_count_kernel(SearchArgs a, SearchBuffers b, int r0, int r1) {
+    chain_entry();
     const int span = r1 - r0;
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e >= static_cast<int64_t>(a.nq) * span) return;
@@ -370,6 +455,7 @@ __global__ void invert_count_kernel(SearchArgs a, SearchBuffers b, int r0, int r
 }
 
 __global__ void invert_scatter_kernel(SearchArgs a, SearchBuffers b, int r0, int r1) {
+    chain_entry();
     const int span = r1 - r0;
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e >= static_cast<int64_t>(a.nq) * span) return;
@@ -388,10 +474,10 @@ cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const Sear
     if (!counted) {
         cudaError_t e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * 2 * static_cast<size_t>(ix.nl), s);   // qcount, qcursor
         if (e != cudaSuccess) return e;
-        invert_count_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
+        if (const cudaError_t le = launch_chained(invert_count_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     }
-    invert_offsets_kernel<<<1, kScanBlock, 0, s>>>(ix, b, scan_group(a.lut_mode), a.chunk);
-    invert_scatter_kernel<<<grid, 256, 0, s>>>(a, b, r0, r1);
+    if (const cudaError_t le = launch_chained(invert_offsets_kernel, dim3(1), dim3(kScanBlock), 0, s, ix, b, scan_group(a.lut_mode), a.chunk); le != cudaSuccess) return le;
+    if (const cudaError_t le = launch_chained(invert_scatter_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -407,6 +493,7 @@ __device__ __forceinline__ float lut_entry(const float* __restrict__ q, const fl
 }
 
 __global__ void lut_f32_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int per_q = ix.B * kCenters;
     if (e >= static_cast<int64_t>(a.nq) * per_q) return;
@@ -420,6 +507,7 @@ __global__ void lut_f32_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
 // One CTA per query: the uint8 table, delta and bias, all in fp32 with
 // round-to-nearest operations in a fixed order.
 __global__ void __launch_bounds__(256) lut_u8_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     float* lut = reinterpret_cast<float*>(smem);          // [B*16]
     float* mins = lut + ix.B * kCenters;                  // [B]
@@ -460,12 +548,12 @@ __global__ void __launch_bounds__(256) lut_u8_kernel(DeviceIndex ix, SearchArgs 
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
     if (a.lut_mode == 0) {
         int64_t total = static_cast<int64_t>(a.nq) * ix.B * kCenters;
-        lut_f32_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(ix, a, b);
+        if (const cudaError_t le = launch_chained(lut_f32_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, s, ix, a, b); le != cudaSuccess) return le;
     } else {
         size_t smem = (static_cast<size_t>(ix.B) * kCenters + ix.B) * sizeof(float);
         cudaError_t e = ensure_smem(reinterpret_cast<const void*>(lut_u8_kernel), smem, true);
         if (e != cudaSuccess) return e;
-        lut_u8_kernel<<<a.nq, 256, smem, s>>>(ix, a, b);
+        if (const cudaError_t le = launch_chained(lut_u8_kernel, dim3(a.nq), dim3(256), smem, s, ix, a, b); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -513,13 +601,20 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
         const int32_t sl = valid[u] ? pos[u] : 0;
         cw[u] = codes_il + (static_cast<int64_t>(sl >> 5) * W) * 32 + (sl & 31);
     }
+    // the next word of each slot is loaded while the current one is looked up
+    uint32_t nxt[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) nxt[u] = cw[u][0];
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int w = 0; w < W; ++w) {
             uint32_t c[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) c[u] = cw[u][w * 32];
+            for (int u = 0; u < 4; ++u) {
+                c[u] = nxt[u];
+                if (w + 1 < W) nxt[u] = cw[u][(w + 1) * 32];
+            }
             const int nb = min(8, B - 8 * w);
             const float* base = lf + 8 * w * kCenters;
             if (nb == 8) {
@@ -540,7 +635,10 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
         for (int w = 0; w < W; ++w) {
             uint32_t c[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) c[u] = cw[u][w * 32];
+            for (int u = 0; u < 4; ++u) {
+                c[u] = nxt[u];
+                if (w + 1 < W) nxt[u] = cw[u][(w + 1) * 32];
+            }
             const int nb = min(8, B - 8 * w);
             const unsigned char* base = lut + 8 * w * kCenters;
             for (int i = 0; i < nb; ++i)
@@ -587,6 +685,7 @@ __host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
 // With fewer than R points in total the bound is 0 (keep everything).
 template <int MODE>
 __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kSelThreads> rs;
@@ -614,11 +713,14 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
                 ok[u] = t < m;
                 ps[u] = p0 + t;
             }
+            int32_t sid[4];              // loaded ahead, to overlap the code loads
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sid[u] = ok[u] ? ix.slot_ids[s0 + t0 + u * kSelThreads + threadIdx.x] : 0;
             slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, v);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int t = t0 + u * kSelThreads + threadIdx.x;
-                if (ok[u]) vals[taken + t] = make_key(v[u], ix.slot_ids[s0 + t]);
+                if (ok[u]) vals[taken + t] = make_key(v[u], sid[u]);
             }
         }
         taken += m;
@@ -664,11 +766,11 @@ cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const S
     if (a.lut_mode == 0) {
         e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
-        threshold_kernel<0><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+        if (const cudaError_t le = launch_chained(threshold_kernel<0>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
     } else {
         e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<1>), smem, true);
         if (e != cudaSuccess) return e;
-        threshold_kernel<1><<<a.nq, kSelThreads, smem, s>>>(ix, a, b);
+        if (const cudaError_t le = launch_chained(threshold_kernel<1>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -869,6 +971,7 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 template <int MODE, int NT>
 __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : 1)) scan_kernel(DeviceIndex ix, SearchArgs a,
                                                                                          SearchBuffers b) {
+    chain_entry();
     constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
     constexpr int GSTEP = (MODE == 0) ? 2 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -995,7 +1098,7 @@ static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const Sear
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT>, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    scan_kernel<MODE, NT><<<num_sms * per_sm, NT, smem, s>>>(ix, a, b);
+    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -1018,6 +1121,7 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
 // keys that reach the new bound (order kept; writes only move entries left,
 // and each chunk is read completely before any of it is written).
 __global__ void __launch_bounds__(kSelThreads) tau_update_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kSelThreads> rs;
     __shared__ int s_kept;
@@ -1076,7 +1180,7 @@ __global__ void __launch_bounds__(kSelThreads) tau_update_kernel(DeviceIndex ix,
 }
 
 cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
-    tau_update_kernel<<<a.nq, kSelThreads, 0, s>>>(ix, a, b);
+    if (const cudaError_t le = launch_chained(tau_update_kernel, dim3(a.nq), dim3(kSelThreads), 0, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -1089,6 +1193,7 @@ cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const 
 // to redo every CTA exits after one atomic.
 template <int MODE>
 __global__ void __launch_bounds__(kSelThreads) redo_scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_item;
     const int* list = b.redo + static_cast<int64_t>(round - 1) * a.nq;
@@ -1129,11 +1234,11 @@ cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const S
     if (a.lut_mode == 0) {
         e = ensure_smem(reinterpret_cast<const void*>(redo_scan_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
-        redo_scan_kernel<0><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
+        if (const cudaError_t le = launch_chained(redo_scan_kernel<0>, dim3(grid), dim3(kSelThreads), smem, s, ix, a, b, round); le != cudaSuccess) return le;
     } else {
         e = ensure_smem(reinterpret_cast<const void*>(redo_scan_kernel<1>), smem, true);
         if (e != cudaSuccess) return e;
-        redo_scan_kernel<1><<<grid, kSelThreads, smem, s>>>(ix, a, b, round);
+        if (const cudaError_t le = launch_chained(redo_scan_kernel<1>, dim3(grid), dim3(kSelThreads), smem, s, ix, a, b, round); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -1200,7 +1305,21 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
     const bool sorted = a.reorder_num == 0 || a.tr_cand_ids || a.tr_cand_scores || a.tr_cand_sums;
     int K;
     int staged = -1;                  // keys staged in shared memory, or -1: read from global
-    if (cnt <= kStageCap) {
+    if (cnt <= 8 * 32 && R <= kWarpMaxK) {
+        // few kept candidates: one warp selects straight from global memory
+        if (threadIdx.x < 32) {
+            int kk;
+            if (cnt <= 2 * 32)
+                kk = warp_topk_src<2>(ck, cs, cnt, R, okeys, oslots, sorted);
+            else if (cnt <= 4 * 32)
+                kk = warp_topk_src<4>(ck, cs, cnt, R, okeys, oslots, sorted);
+            else
+                kk = warp_topk_src<8>(ck, cs, cnt, R, okeys, oslots, sorted);
+            if (threadIdx.x == 0) scr.count = kk;
+        }
+        __syncthreads();
+        staged = -2;
+    } else if (cnt <= kStageCap) {
         for (int i = threadIdx.x; i < cnt; i += kFinishThreads) {
             skeys[i] = ck[i];
             sslots[i] = cs[i];
@@ -1208,15 +1327,25 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         staged = cnt;
         __syncthreads();
     } else if (R < kStageCap) {
-        // Many kept candidates: the R-th best of the first kStageCap is a lower
-        // bound on the R-th best of all (a subset's), so one batched pass keeps
-        // only the keys that reach it.
-        for (int i = threadIdx.x; i < kStageCap; i += kFinishThreads) skeys[i] = ck[i];
-        __syncthreads();
-        uint64_t sk[kStageCap / kFinishThreads];
+        // Many kept candidates: the R-th best of any subset is a lower bound on
+        // the R-th best of all, so the largest such bound over kStageCap-key
+        // chunks (keys below the running bound dropped first) lets one
+        // batched pass keep only the keys that reach it.
+        constexpr int CPT = kStageCap / kFinishThreads;
+        uint64_t bound = 0ull;
+        for (int c0 = 0; c0 < cnt; c0 += kStageCap) {
+            uint64_t sk[CPT];
+            int live = 0;
 #pragma unroll
-        for (int j = 0; j < kStageCap / kFinishThreads; ++j) sk[j] = skeys[threadIdx.x + kFinishThreads * j];
-        const uint64_t bound = block_kth_reg<kStageCap / kFinishThreads, kFinishThreads>(sk, kStageCap, R, rs);
+            for (int j = 0; j < CPT; ++j) {
+                const int i = c0 + threadIdx.x + kFinishThreads * j;
+                const uint64_t key = (i < cnt) ? ck[i] : 0ull;
+                sk[j] = (key >= bound) ? key : 0ull;
+                live += (sk[j] != 0ull) ? 1 : 0;
+            }
+            live = block_sum_parity<kFinishThreads>(live, rs, (c0 / kStageCap) & 1);
+            if (live > R) bound = block_kth_reg<CPT, kFinishThreads>(sk, live, R, rs);
+        }
         if (threadIdx.x == 0) scr.count = 0;
         __syncthreads();
         constexpr int U = 4;
@@ -1243,8 +1372,12 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         if (scr.count <= kStageCap) staged = scr.count;
         __syncthreads();
     }
-    if (staged >= 0 && staged <= 4 * kFinishThreads) {
-        K = block_topk_reg<kFinishThreads>(skeys, sslots, staged, R, rs, &scr.count, okeys, oslots, sorted);
+    if (staged == -2) {
+        K = scr.count;
+    } else if (staged >= 0 && staged <= 4 * kFinishThreads) {
+        auto get = [&](int i) { return skeys[i]; };
+        auto pay = [&](int i) { return sslots[i]; };
+        K = block_topk_reg<4, kFinishThreads>(get, pay, staged, R, rs, &scr.count, okeys, oslots, sorted);
     } else if (staged >= 0) {
         auto get = [&](int i) { return skeys[i]; };
         auto pay = [&](int i) { return sslots[i]; };
@@ -1291,25 +1424,51 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
             const int64_t slot = oslots[i];
             if (a.reorder_vec4) {        // d % 4 == 0 and 16-byte aligned rows (checked on the host)
                 const float4* q4 = reinterpret_cast<const float4*>(qv);
+                // The row loads are issued kReorderBatch at a time ahead of
+                // the multiply-adds (same accumulation order), so a lane waits
+                // for memory once per batch rather than once per load.
+                const int n4 = d / 4;
                 if (ix.reorder_bf16) {
                     const uint2* v = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d);
-                    for (int t = gl; t < d / 4; t += lpc) {
-                        const uint2 h = v[t];
-                        const float4 x = q4[t];
-                        acc = fmaf(x.x, __uint_as_float(h.x << 16), acc);
-                        acc = fmaf(x.y, __uint_as_float(h.x & 0xFFFF0000u), acc);
-                        acc = fmaf(x.z, __uint_as_float(h.y << 16), acc);
-                        acc = fmaf(x.w, __uint_as_float(h.y & 0xFFFF0000u), acc);
+                    for (int t0 = gl; t0 < n4; t0 += kReorderBatch * lpc) {
+                        uint2 h[kReorderBatch];
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            h[u] = (t < n4) ? v[t] : make_uint2(0u, 0u);
+                        }
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            if (t < n4) {
+                                const float4 x = q4[t];
+                                acc = fmaf(x.x, __uint_as_float(h[u].x << 16), acc);
+                                acc = fmaf(x.y, __uint_as_float(h[u].x & 0xFFFF0000u), acc);
+                                acc = fmaf(x.z, __uint_as_float(h[u].y << 16), acc);
+                                acc = fmaf(x.w, __uint_as_float(h[u].y & 0xFFFF0000u), acc);
+                            }
+                        }
                     }
                 } else {
                     const float4* v = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(ix.reorder_vecs) + slot * d);
-                    for (int t = gl; t < d / 4; t += lpc) {
-                        const float4 h = v[t];
-                        const float4 x = q4[t];
-                        acc = fmaf(x.x, h.x, acc);
-                        acc = fmaf(x.y, h.y, acc);
-                        acc = fmaf(x.z, h.z, acc);
-                        acc = fmaf(x.w, h.w, acc);
+                    for (int t0 = gl; t0 < n4; t0 += kReorderBatch * lpc) {
+                        float4 h[kReorderBatch];
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            h[u] = (t < n4) ? v[t] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            if (t < n4) {
+                                const float4 x = q4[t];
+                                acc = fmaf(x.x, h[u].x, acc);
+                                acc = fmaf(x.y, h[u].y, acc);
+                                acc = fmaf(x.z, h[u].z, acc);
+                                acc = fmaf(x.w, h[u].w, acc);
+                            }
+                        }
                     }
                 }
             } else if (ix.reorder_bf16) {
@@ -1347,7 +1506,8 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kFinishThreads, 6) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+__global__ void __launch_bounds__(kFinishThreads, AH_FINISH_MIN_BLOCKS) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
+    chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kFinishThreads> rs;
@@ -1385,10 +1545,10 @@ cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffe
     cudaError_t e;
     if (a.lut_mode == 0) {
         if ((e = prefer_shared(finish_kernel<0>, smem)) != cudaSuccess) return e;
-        finish_kernel<0><<<grid, kFinishThreads, smem, s>>>(ix, a, b, round);
+        if (const cudaError_t le = launch_chained(finish_kernel<0>, dim3(grid), dim3(kFinishThreads), smem, s, ix, a, b, round); le != cudaSuccess) return le;
     } else {
         if ((e = prefer_shared(finish_kernel<1>, smem)) != cudaSuccess) return e;
-        finish_kernel<1><<<grid, kFinishThreads, smem, s>>>(ix, a, b, round);
+        if (const cudaError_t le = launch_chained(finish_kernel<1>, dim3(grid), dim3(kFinishThreads), smem, s, ix, a, b, round); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }

@@ -422,11 +422,15 @@ __device__ uint64_t warp_kth_largest(GetKey get, int n, int K, int* hist) {
 // ---------------------------------------------------------------------------
 namespace ah {
 
-// The K-th largest of the warp's keys (1 <= K <= number of real keys); all
-// lanes return it.
+// The K-th largest of the warp's keys (n > 0 real keys in total, key 0 =
+// empty, 1 <= K <= n); all lanes return it.  Bitwise radix from the highest
+// bit where the keys differ: each step counts the current bucket's keys with
+// the bit set (one warp reduction; the running bucket size gives the other
+// half), and the walk stops once the bucket holding the K-th key is exactly
+// the remainder.  While the bit is in the upper word only those words are
+// compared.
 template <int KPL>
-__device__ uint64_t warp_kth_reg(const uint64_t (&k)[KPL], int K) {
-    // bits every real key shares are skipped
+__device__ uint64_t warp_kth_reg(const uint64_t (&k)[KPL], int n, int K) {
     uint64_t kand = ~0ull, kor = 0ull;
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
@@ -437,33 +441,54 @@ __device__ uint64_t warp_kth_reg(const uint64_t (&k)[KPL], int K) {
     kor = warp_or64(kor);
     const uint64_t diff = kand ^ kor;
     if (diff == 0ull) return kor;                       // one distinct real key
-    const int top = 63 - __clzll(static_cast<long long>(diff));
-    uint64_t prefix = (top >= 63) ? 0ull : (kand & (~0ull << (top + 1)));
-    int need = K;
-    for (int bit = top; bit >= 0; --bit) {
-        const uint64_t hm = ~0ull << bit;               // bits >= bit
-        const uint64_t cand = prefix | (1ull << bit);
-        int c = 0, in_low = 0;
+    int bit = 63 - __clzll(static_cast<long long>(diff));
+    uint64_t prefix = (bit >= 63) ? 0ull : (kand & (~0ull << (bit + 1)));
+    int need = K, in_bucket = n;
+    bool done = false;
+    if (bit >= 32) {                                    // prefix has no low bits yet
+        unsigned phi = static_cast<unsigned>(prefix >> 32);
+        for (; bit >= 32; --bit) {
+            const unsigned hm = ~0u << (bit - 32);
+            const unsigned cand = phi | (1u << (bit - 32));
+            int c = 0;
 #pragma unroll
-        for (int j = 0; j < KPL; ++j) {
-            const uint64_t m = k[j] & hm;
-            c += (m == cand);
-            in_low += (m == prefix);
+            for (int j = 0; j < KPL; ++j) c += ((static_cast<unsigned>(k[j] >> 32) & hm) == cand) ? 1 : 0;
+            c = __reduce_add_sync(0xFFFFFFFFu, c);
+            if (c >= need) {
+                phi = cand;
+                in_bucket = c;
+            } else {
+                need -= c;
+                in_bucket -= c;
+            }
+            if (in_bucket == need) {
+                done = true;
+                break;
+            }
         }
-        c = __reduce_add_sync(0xFFFFFFFFu, c);
-        in_low = __reduce_add_sync(0xFFFFFFFFu, in_low);
-        if (c >= need) {
-            prefix = cand;
-            if (c == need) break;                       // the bucket is exactly the rest
-        } else {
-            need -= c;
-            if (in_low == need) break;                  // keys with this bit clear are exactly the rest
+        prefix = static_cast<uint64_t>(phi) << 32;
+    }
+    if (!done) {
+        for (; bit >= 0; --bit) {
+            const uint64_t hm = ~0ull << bit;
+            const uint64_t cand = prefix | (1ull << bit);
+            int c = 0;
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) c += ((k[j] & hm) == cand) ? 1 : 0;
+            c = __reduce_add_sync(0xFFFFFFFFu, c);
+            if (c >= need) {
+                prefix = cand;
+                in_bucket = c;
+            } else {
+                need -= c;
+                in_bucket -= c;
+            }
+            if (in_bucket == need) break;
         }
     }
-    // the K-th largest is the smallest key in the final bucket
+    // the K-th largest is the smallest real key of the final bucket, which is
+    // the smallest real key >= prefix
     uint64_t mn = ~0ull;
-    const int bits_left = 0;
-    (void)bits_left;
 #pragma unroll
     for (int j = 0; j < KPL; ++j)
         if (k[j] >= prefix && k[j] != 0ull && k[j] < mn) mn = k[j];
@@ -515,13 +540,52 @@ __device__ int warp_topk_reg(GetKey get, GetVal pay, int n, int K, uint64_t* out
     }
     if (K > n) K = n;
     if (K <= 0) return 0;
-    const uint64_t thr = (K < n) ? warp_kth_reg<KPL>(k, K) : 1ull;
+    const uint64_t thr = (K < n) ? warp_kth_reg<KPL>(k, n, K) : 1ull;
     const int P2 = next_pow2(K);
     for (int i = K + lane; i < P2; i += 32) {
         out_k[i] = 0ull;
         if (out_v) out_v[i] = -1;
     }
     warp_gather_ge<KPL>(k, v, thr, out_k, out_v);
+    if (sort) warp_sort_desc(out_k, out_v, P2);
+    return K;
+}
+
+
+// The K = min(K, n) largest of keys[0..n) (n <= 32*KPL; any address space)
+// by one warp, with payload vals[i] (may be null) fetched only for the keys
+// kept.  Output as warp_topk_reg.  Returns K.
+template <int KPL>
+__device__ int warp_topk_src(const uint64_t* keys, const int32_t* vals, int n, int K, uint64_t* out_k,
+                             int32_t* out_v, bool sort) {
+    const int lane = threadIdx.x & 31;
+    uint64_t k[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const int i = lane + 32 * j;
+        k[j] = (i < n) ? keys[i] : 0ull;
+    }
+    if (K > n) K = n;
+    if (K <= 0) return 0;
+    const uint64_t thr = (K < n) ? warp_kth_reg<KPL>(k, n, K) : 1ull;
+    const int P2 = next_pow2(K);
+    for (int i = K + lane; i < P2; i += 32) {
+        out_k[i] = 0ull;
+        if (out_v) out_v[i] = -1;
+    }
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const bool sel = k[j] != 0ull && k[j] >= thr;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            out_k[pos] = k[j];
+            if (out_v) out_v[pos] = vals[lane + 32 * j];
+        }
+        base += __popc(m);
+    }
+    __syncwarp();
     if (sort) warp_sort_desc(out_k, out_v, P2);
     return K;
 }

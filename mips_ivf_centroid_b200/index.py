@@ -218,8 +218,9 @@ class Index:
         _check(self._lib, self._lib.ah_set_option(self._h, option, value))
 
     # -- instrumentation ------------------------------------------------------
-    def set_profiling(self, on: bool = True):
-        _check(self._lib, self._lib.ah_set_profiling(self._h, 1 if on else 0))
+    def set_profiling(self, on=True):
+        """0/False off, 1/True every stage, 2 the scan phases only."""
+        _check(self._lib, self._lib.ah_set_profiling(self._h, int(on)))
 
     def stage_times(self) -> dict:
         ms = (ctypes.c_float * 16)()

@@ -40,6 +40,12 @@ def _workload(name):
                                           n_means=60, training_sample_size=20_000),
         "sweep-mini": W["sweep"].scaled(n=200_000, num_leaves=1000, num_leaves_to_search=64, nq=256,
                                         n_means=800, training_sample_size=200_000),
+        "leaves-1500": W["glove"].scaled(n=30_000, d=32, num_leaves=1500, num_leaves_to_search=40, nq=128,
+                                         n_means=100, training_sample_size=30_000),
+        "leaves-3000": W["glove"].scaled(n=30_000, d=32, num_leaves=3000, num_leaves_to_search=64, nq=128,
+                                         n_means=100, training_sample_size=30_000),
+        "leaves-5000": W["glove"].scaled(n=50_000, d=32, num_leaves=5000, num_leaves_to_search=16, nq=128,
+                                         n_means=100, training_sample_size=50_000),
         "small-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=600, num_leaves_to_search=2, nq=64,
                                           n_means=10, training_sample_size=3_000, code_loss="l2",
                                           threshold_T=None),
@@ -155,6 +161,14 @@ def test_openai_mini_u8(Index):
 
 def test_sweep_mini(Index):
     compare(Index, "sweep-mini", 10, 64, 100, 0)
+
+
+@pytest.mark.parametrize("name", ["leaves-1500", "leaves-3000", "leaves-5000"])
+def test_many_centroids(Index, name):
+    # more centroids than one warp holds in registers (two register widths)
+    # and more than the block's register form holds (shared-memory radix)
+    w = _workload(name)[0]
+    compare(Index, name, 10, w.num_leaves_to_search, 100, 0)
 
 
 def test_all_leaves(Index):
