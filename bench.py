@@ -64,6 +64,42 @@ def dist_env():
     return rank, world, local
 
 
+def init_ranks(world, dev):
+    """Process group for N > 1 ranks (NCCL on GPUs, gloo on CPU), with a short
+    timeout so ranks waiting for a missing peer end with an error."""
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world <= 1:
+        return False
+    if dev.type == "cuda":
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    else:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=120))
+    return True
+
+
+def max_over_ranks(x, dev, world):
+    """The largest of every rank's x (device time: the slowest rank sets the job's time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, nq_per_rank, total_ms, steps):
+    """Whole-job queries/s (every rank searches its own batch each step) and ms per step."""
+    ms_per_step = total_ms / steps
+    return world * nq_per_rank / (ms_per_step * 1e-3), ms_per_step
+
+
+def rank_workload(w, rank):
+    """Rank r searches its own query batch (query seed + 1000 r) over the same index."""
+    return w.scaled(query_seed=w.query_seed + 1000 * rank)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
@@ -204,14 +240,12 @@ def run_ours(args):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    init_ranks(world, dev)
 
     from mips_ivf_centroid_b200 import Index, build as ahbuild, datagen
     ahbuild.build()
     w = workload_spec(args)
-    wq = w.scaled(query_seed=w.query_seed + 1000 * rank)          # each rank: its own batch
+    wq = rank_workload(w, rank)                                    # each rank: its own batch
     X = datagen.make_data(w)
     Q = datagen.make_queries(wq)
     ix = datagen.build_index(w, X, dev)
@@ -270,13 +304,10 @@ def run_ours(args):
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     dev_ms = sum(step_ms)
     launches = index.last_search_info()["launches"]
+    dev_ms = max_over_ranks(dev_ms, dev, world)
     if world > 1:
-        t = torch.tensor([dev_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dev_ms = float(t.item())
         dist.barrier()
-    ms_per_step = dev_ms / args.steps
-    value = world * w.nq / (ms_per_step * 1e-3)
+    value, ms_per_step = job_throughput(world, w.nq, dev_ms, args.steps)
 
     # e2e through the host entry point: pinned host queries in, host results out
     hq = torch.from_numpy(Q).pin_memory()
@@ -293,11 +324,7 @@ def run_ours(args):
         t0 = time.perf_counter()
         index.search_host(hq, k, L, R, mode, out_ids=hids, out_scores=hsc)
         e2e_times.append(time.perf_counter() - t0)
-    e2e_s = sum(e2e_times)
-    if world > 1:
-        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(sum(e2e_times), dev, world)
     e2e_value = world * w.nq * args.e2e_steps / e2e_s
 
     if rank == 0:

@@ -2,7 +2,7 @@
 //
 // Path (ScaNN blog post, "Three stages of a search"):
 //   centroid_scores_kernel   s[q][c] = q . centroid_c                 (partitioning)
-//   top_leaves_kernel        best L leaves per query
+//   top_leaves_*_kernel      best L leaves per query
 //   invert_*                 query->leaf lists become leaf->query lists, so a
 //                            leaf's codes are read once per query group
 //   lut_*_kernel             lut[q][b][j] = q_b . center[b][j]        (AH table)
@@ -11,9 +11,11 @@
 //   scan_kernel              leaf-major 4-bit code scan: per slot, the sum of
 //                            table entries for every query of the group;
 //                            scores at or above the bound are kept
+//   tau_update_kernel        between scan phases, raises each bound to the R-th
+//                            best point kept so far
 //   redo_scan_kernel         query-major rescan for the rare query whose kept
 //                            set overflowed its buffer (with a tighter bound)
-//   rerank_kernel            best R by approximate score, exact fp32 dot
+//   finish_kernel            best R by approximate score, exact fp32 dot
 //                            products for them (reordering), best k
 #include <cuda_runtime.h>
 
@@ -1111,7 +1113,7 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
 }
 
 // ---------------------------------------------------------------------------
-// bound refinement between the two scan phases
+// bound refinement between scan phases
 // ---------------------------------------------------------------------------
 
 // One CTA per query, between scan phases: every point of the leaves scanned so
@@ -1265,9 +1267,9 @@ size_t finish_smem_bytes(int R, int d) {
 //     round an overflow is reported through the error word and the stored
 //     subset is used.
 //  2. Without reorder, the best k of those are the result.  With reorder,
-//     8-lane groups compute the exact fp32 dot product of each candidate's
-//     stored vector (float, or bfloat16 upcast) with the query, and one warp
-//     keeps the best k by (exact score, id).
+//     groups of 2..32 lanes (by d) compute the exact fp32 dot product of each
+//     candidate's stored vector (float, or bfloat16 upcast) with the query,
+//     and one warp keeps the best k by (exact score, id).
 template <int MODE>
 __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round, int q,
                              unsigned char* smem, SelectScratch& scr,
