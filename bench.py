@@ -37,6 +37,10 @@ L2_BYTES = 126 * 1024 * 1024
 SM_COUNT = 148
 SMEM_BYTES_PER_CLK = 128          # per SM: 32 banks x 4 B
 SM_MAX_MHZ_FALLBACK = 1965.0
+# DRAM bytes (read + write) that one ncu capture counted for one scan launch, per
+# (workload, table mode) at the workload's default batch; None where no capture
+# of the current scan kernel exists.
+SCAN_TRAFFIC_BYTES = {("glove", 0): 35.81e6}
 
 
 def parse():
@@ -344,16 +348,31 @@ def run_ours(args):
         smem_peak_gbs = SM_COUNT * SMEM_BYTES_PER_CLK * mhz * 1e6 / 1e9
         achieved = lut_bytes / (scan_ms * 1e-3) / 1e9
         roofline = {"bound": "smem", "achieved": achieved, "peak": smem_peak_gbs, "unit": "GB/s",
-                    "frac": achieved / smem_peak_gbs, "traffic": None,
+                    "frac": achieved / smem_peak_gbs,
+                    "traffic": (SCAN_TRAFFIC_BYTES.get((args.workload, mode))
+                                if args.nq is None and args.leaves is None else None),
                     "kernel": "scan_kernel", "unit_bytes": f"{bytes_per_lookup} B per table lookup",
                     "lookups_per_launch": lookups,
                     "peak_source": f"derived: {SM_COUNT} SMs x {SMEM_BYTES_PER_CLK} B/clk x {mhz:.0f} MHz"}
+        # the step against the sum of its stages' roofline times: centroid GEMM at
+        # the SIMT fp32 FMA peak, the scan at the larger of its SMEM-lookup and
+        # unique-code HBM times, the reorder gather at the HBM copy rate
+        hbm = hbm_peak or 6650.0
+        fp32_tflops = SM_COUNT * 128 * 2 * mhz * 1e6 / 1e12
+        elt = 2 if w.reorder_dtype == "bf16" else 4
+        parts = {"centroid_scores": 2.0 * w.nq * w.num_leaves * w.d / (fp32_tflops * 1e12) * 1e3,
+                 "scan": max(lut_bytes / (smem_peak_gbs * 1e9), unique_code_bytes / (hbm * 1e9)) * 1e3,
+                 "reorder_gather": (w.nq * w.reorder_num * w.d * elt / (hbm * 1e9) * 1e3) if w.reorder_num else 0.0}
+        roof_ms = sum(parts.values())
+        step_roofline = {"ms": roof_ms, "frac": roof_ms / ms_per_step, "parts_ms": parts,
+                         "peaks": f"fp32 FMA {fp32_tflops:.1f} TFLOP/s derived, SMEM {smem_peak_gbs:.0f} GB/s derived, "
+                                  f"HBM {hbm:.0f} GB/s " + ("measured" if hbm_peak else "fallback")}
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32" if mode == 0 else "u8",
                 "data": "synthetic (seeded Gaussian mixture, GloVe-shaped; index trained on it)",
                 "config": config_dict(w, args),
-                "roofline": roofline,
+                "roofline": roofline, "step_roofline": step_roofline,
                 "scan": {"ms": scan_ms, "hbm_unique_code_gbs": unique_code_bytes / (scan_ms * 1e-3) / 1e9,
                          "unique_code_bytes": unique_code_bytes, "hbm_peak_gbs": hbm_peak,
                          "lookups_per_s": lookups / (scan_ms * 1e-3)},

@@ -276,6 +276,44 @@ AH_API ah_status ah_search_leaves_noalloc(ah_index *ix, const float *queries, in
                                           float *out_leaf_scores, void *cuda_stream);
 
 /* Release everything the index owns.  Does not touch the borrowed views. */
+/*
+ * Index directories (ScaNN blog, "Using the library": a built searcher is
+ * written to a directory and loaded back later).  ah_save writes the index's
+ * arrays into the existing directory `dir` as NumPy .npy files (format 1.0,
+ * little endian, C order; numpy.load reads each one), overwriting them:
+ *   centroids.npy     <f4 [num_leaves, d]
+ *   leaf_offsets.npy  <i8 [num_leaves + 1]
+ *   slot_ids.npy      <i4 [n]
+ *   codes.npy         |u1 [n, d / dims_per_block / 2]
+ *   codebook.npy      <f4 [d / dims_per_block, 16, dims_per_block]
+ *   reorder_vecs.npy  <f4 [n, d], or <u2 [n, d] holding bfloat16 bit
+ *                     patterns (absent when the index has no reorder copy)
+ *   ah_index.txt      first line "ah-index 1", then "reorder_dtype f32",
+ *                     "reorder_dtype bf16" or "reorder_dtype none"
+ * Synchronous (device-to-host copies).  Errors: AH_ERR_INVALID_ARG (NULL
+ * argument, a file that cannot be written: the message names it),
+ * AH_ERR_CUDA.
+ */
+AH_API ah_status ah_save(ah_index *ix, const char *dir);
+
+/*
+ * Reads the sizes of an index directory without using the GPU: fills n, d,
+ * num_leaves, dims_per_block and reorder_dtype of *out (-1 for no reorder
+ * copy) and sets its pointers to NULL.  Every file's header is checked
+ * against the others' and against the file's length.  Errors:
+ * AH_ERR_INVALID_ARG (a missing or malformed file; the message names it).
+ */
+AH_API ah_status ah_inspect(const char *dir, ah_index_views *out);
+
+/*
+ * Loads an index directory onto the current device: the arrays are copied
+ * into device memory that the index owns (counted by ah_index_memory, freed
+ * by ah_destroy), then the index is built as by ah_build_index_views on
+ * cuda_stream.  Synchronous.  Errors: those of ah_inspect, AH_ERR_OOM,
+ * AH_ERR_CUDA, and those of ah_build_index_views.  *out is NULL on error.
+ */
+AH_API ah_status ah_load(const char *dir, void *cuda_stream, ah_index **out);
+
 AH_API void ah_destroy(ah_index *ix);
 
 /* Static text for a status code. */

@@ -16,6 +16,7 @@
 
 #include "ah.h"
 #include "kernels.h"
+#include "npy_io.h"
 
 namespace {
 
@@ -78,6 +79,7 @@ struct ah_index {
     int opt_threshold_leaves = 1;
     int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
+    void* loaded[6] = {};            // index arrays owned by an index from ah_load
 };
 
 namespace {
@@ -581,6 +583,8 @@ void ah_destroy(ah_index* ix) {
     if (ix->offs32) cudaFree(ix->offs32);
     if (ix->ptile) cudaFree(ix->ptile);
     if (ix->err) cudaFree(ix->err);
+    for (void* p : ix->loaded)
+        if (p) cudaFree(p);
     if (ix->ev_ready)
         for (int i = 0; i < ah_index::kMaxMarks; ++i) cudaEventDestroy(ix->ev[i]);
     delete ix;
@@ -659,3 +663,203 @@ ah_status ah_search_leaves_noalloc(ah_index* ix, const float* queries, int32_t n
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// index directories
+// ---------------------------------------------------------------------------
+
+namespace {
+
+const char* const kIndexFiles[6] = {"centroids.npy", "leaf_offsets.npy", "slot_ids.npy",
+                                    "codes.npy",     "codebook.npy",     "reorder_vecs.npy"};
+const char* const kMetaFile = "ah_index.txt";
+constexpr size_t kStageBytes = size_t(64) << 20;      // host staging for the copies
+
+std::string path_in(const char* dir, const char* file) {
+    std::string s(dir);
+    if (!s.empty() && s.back() != '/') s += '/';
+    return s + file;
+}
+
+// array i of the views: device pointer, dtype text, shape
+struct ArraySpec {
+    const void* ptr;
+    std::string descr;
+    std::vector<int64_t> shape;
+};
+
+std::vector<ArraySpec> array_specs(const ah_index_views& v) {
+    const int64_t B = v.d / v.dims_per_block;
+    std::vector<ArraySpec> a(6);
+    a[0] = {v.centroids, "<f4", {v.num_leaves, v.d}};
+    a[1] = {v.leaf_offsets, "<i8", {int64_t(v.num_leaves) + 1}};
+    a[2] = {v.slot_ids, "<i4", {v.n}};
+    a[3] = {v.codes, "|u1", {v.n, B / 2}};
+    a[4] = {v.codebook, "<f4", {B, 16, v.dims_per_block}};
+    a[5] = {v.reorder_vecs, v.reorder_dtype == AH_BF16 ? "<u2" : "<f4", {v.n, v.d}};
+    return a;
+}
+
+ah_status write_array(const std::string& path, const ArraySpec& a, std::vector<char>& stage) {
+    FILE* f = std::fopen(path.c_str(), "wb");
+    if (!f) return fail(AH_ERR_INVALID_ARG, ("cannot write " + path).c_str());
+    const std::string h = ah::npy::make_header(a.descr, a.shape);
+    bool ok = std::fwrite(h.data(), 1, h.size(), f) == h.size();
+    const int64_t bytes = ah::npy::count(a.shape) * ah::npy::item_size(a.descr);
+    for (int64_t off = 0; ok && off < bytes; off += static_cast<int64_t>(stage.size())) {
+        const size_t len = static_cast<size_t>(std::min<int64_t>(bytes - off, static_cast<int64_t>(stage.size())));
+        cudaError_t e = cudaMemcpy(stage.data(), static_cast<const char*>(a.ptr) + off, len, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) {
+            std::fclose(f);
+            return cuda_fail(e, "index array read");
+        }
+        ok = std::fwrite(stage.data(), 1, len, f) == len;
+    }
+    ok = (std::fclose(f) == 0) && ok;
+    return ok ? AH_OK : fail(AH_ERR_INVALID_ARG, ("short write to " + path).c_str());
+}
+
+}  // namespace
+
+ah_status ah_save(ah_index* ix, const char* dir) {
+    if (!ix || !dir) return fail(AH_ERR_INVALID_ARG, "NULL argument");
+    const ah_index_views& v = ix->views;
+    std::vector<ArraySpec> a = array_specs(v);
+    std::vector<char> stage(kStageBytes);
+    for (int i = 0; i < 6; ++i) {
+        if (i == 5 && !v.reorder_vecs) continue;
+        const ah_status st = write_array(path_in(dir, kIndexFiles[i]), a[i], stage);
+        if (st != AH_OK) return st;
+    }
+    if (!v.reorder_vecs) std::remove(path_in(dir, kIndexFiles[5]).c_str());
+    const std::string meta = path_in(dir, kMetaFile);
+    FILE* f = std::fopen(meta.c_str(), "w");
+    if (!f) return fail(AH_ERR_INVALID_ARG, ("cannot write " + meta).c_str());
+    const char* dt = !v.reorder_vecs ? "none" : (v.reorder_dtype == AH_BF16 ? "bf16" : "f32");
+    const bool ok = std::fprintf(f, "ah-index 1\nreorder_dtype %s\n", dt) > 0;
+    if (std::fclose(f) != 0 || !ok) return fail(AH_ERR_INVALID_ARG, ("short write to " + meta).c_str());
+    return AH_OK;
+}
+
+namespace {
+
+ah_status inspect_dir(const char* dir, ah_index_views* out, ah::npy::Header hdr[6], bool* has_reorder) {
+    // meta: version and the reorder copy's type
+    const std::string meta = path_in(dir, kMetaFile);
+    FILE* f = std::fopen(meta.c_str(), "r");
+    if (!f) return fail(AH_ERR_INVALID_ARG, ("cannot open " + meta).c_str());
+    char l1[64] = {0}, key[64] = {0}, val[64] = {0};
+    const bool ok = std::fgets(l1, sizeof(l1), f) && std::fscanf(f, "%63s %63s", key, val) == 2;
+    std::fclose(f);
+    if (!ok || std::strncmp(l1, "ah-index 1", 10) != 0 || std::strcmp(key, "reorder_dtype") != 0)
+        return fail(AH_ERR_INVALID_ARG, (meta + ": expected \"ah-index 1\" then \"reorder_dtype <f32|bf16|none>\"").c_str());
+    int rdt;
+    if (!std::strcmp(val, "f32")) rdt = AH_F32;
+    else if (!std::strcmp(val, "bf16")) rdt = AH_BF16;
+    else if (!std::strcmp(val, "none")) rdt = -1;
+    else return fail(AH_ERR_INVALID_ARG, (meta + ": unknown reorder_dtype").c_str());
+    *has_reorder = rdt >= 0;
+    for (int i = 0; i < 6; ++i) {
+        if (i == 5 && !*has_reorder) continue;
+        const std::string p = path_in(dir, kIndexFiles[i]);
+        const std::string why = ah::npy::read_header(p.c_str(), &hdr[i]);
+        if (!why.empty()) return fail(AH_ERR_INVALID_ARG, (p + ": " + why).c_str());
+    }
+    auto bad = [&](int i, const char* what) { return fail(AH_ERR_INVALID_ARG, (path_in(dir, kIndexFiles[i]) + ": " + what).c_str()); };
+    const auto& c = hdr[0].shape;
+    if (hdr[0].descr != "<f4" || c.size() != 2) return bad(0, "need <f4 [num_leaves, d]");
+    const int64_t NL = c[0], d = c[1];
+    if (hdr[1].descr != "<i8" || hdr[1].shape != std::vector<int64_t>{NL + 1}) return bad(1, "need <i8 [num_leaves + 1]");
+    if (hdr[2].descr != "<i4" || hdr[2].shape.size() != 1) return bad(2, "need <i4 [n]");
+    const int64_t n = hdr[2].shape[0];
+    const auto& cb = hdr[4].shape;
+    if (hdr[4].descr != "<f4" || cb.size() != 3 || cb[1] != 16 || cb[0] <= 0 || cb[2] <= 0 || cb[0] * cb[2] != d || cb[0] % 2)
+        return bad(4, "need <f4 [B, 16, dims_per_block] with B even and B * dims_per_block = d");
+    const int64_t B = cb[0];
+    if ((hdr[3].descr != "|u1" && hdr[3].descr != "<u1") || hdr[3].shape != std::vector<int64_t>{n, B / 2})
+        return bad(3, "need |u1 [n, B / 2]");
+    if (*has_reorder) {
+        const char* want = rdt == AH_BF16 ? "<u2" : "<f4";
+        if (hdr[5].descr != want || hdr[5].shape != std::vector<int64_t>{n, d})
+            return bad(5, rdt == AH_BF16 ? "need <u2 [n, d] (bfloat16 bits)" : "need <f4 [n, d]");
+    }
+    if (NL <= 0 || NL > INT32_MAX || d <= 0 || d > INT32_MAX || n <= 0) return bad(0, "sizes out of range");
+    *out = ah_index_views{};
+    out->n = n;
+    out->d = static_cast<int32_t>(d);
+    out->num_leaves = static_cast<int32_t>(NL);
+    out->dims_per_block = static_cast<int32_t>(cb[2]);
+    out->reorder_dtype = rdt;
+    return AH_OK;
+}
+
+}  // namespace
+
+ah_status ah_inspect(const char* dir, ah_index_views* out) {
+    if (!dir || !out) return fail(AH_ERR_INVALID_ARG, "NULL argument");
+    ah::npy::Header hdr[6];
+    bool has_reorder = false;
+    return inspect_dir(dir, out, hdr, &has_reorder);
+}
+
+ah_status ah_load(const char* dir, void* cuda_stream, ah_index** out) {
+    if (!out) return fail(AH_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    if (!dir) return fail(AH_ERR_INVALID_ARG, "dir is NULL");
+    ah_index_views v;
+    ah::npy::Header hdr[6];
+    bool has_reorder = false;
+    ah_status st = inspect_dir(dir, &v, hdr, &has_reorder);
+    if (st != AH_OK) return st;
+    void* dev[6] = {};
+    size_t total = 0;
+    auto release = [&]() {
+        for (void*& p : dev)
+            if (p) cudaFree(p);
+    };
+    std::vector<char> stage(kStageBytes);
+    for (int i = 0; i < 6; ++i) {
+        if (i == 5 && !has_reorder) continue;
+        const int64_t bytes = ah::npy::count(hdr[i].shape) * ah::npy::item_size(hdr[i].descr);
+        cudaError_t e = cudaMalloc(&dev[i], static_cast<size_t>(std::max<int64_t>(bytes, 1)));
+        if (e != cudaSuccess) {
+            release();
+            return e == cudaErrorMemoryAllocation ? fail(AH_ERR_OOM, "index arrays") : cuda_fail(e, "index arrays");
+        }
+        total += static_cast<size_t>(bytes);
+        const std::string p = path_in(dir, kIndexFiles[i]);
+        FILE* f = std::fopen(p.c_str(), "rb");
+        bool ok = f && std::fseek(f, static_cast<long>(hdr[i].data_offset), SEEK_SET) == 0;
+        for (int64_t off = 0; ok && off < bytes; off += static_cast<int64_t>(stage.size())) {
+            const size_t len = static_cast<size_t>(std::min<int64_t>(bytes - off, static_cast<int64_t>(stage.size())));
+            ok = std::fread(stage.data(), 1, len, f) == len;
+            if (ok && (e = cudaMemcpy(static_cast<char*>(dev[i]) + off, stage.data(), len, cudaMemcpyHostToDevice)) != cudaSuccess) {
+                std::fclose(f);
+                release();
+                return cuda_fail(e, "index array copy");
+            }
+        }
+        if (f) std::fclose(f);
+        if (!ok) {
+            release();
+            return fail(AH_ERR_INVALID_ARG, ("cannot read " + p).c_str());
+        }
+    }
+    v.centroids = static_cast<const float*>(dev[0]);
+    v.leaf_offsets = static_cast<const int64_t*>(dev[1]);
+    v.slot_ids = static_cast<const int32_t*>(dev[2]);
+    v.codes = static_cast<const uint8_t*>(dev[3]);
+    v.codebook = static_cast<const float*>(dev[4]);
+    v.reorder_vecs = dev[5];
+    if (!has_reorder) v.reorder_dtype = AH_F32;
+    ah_index* ix = nullptr;
+    st = ah_build_index_views(&v, cuda_stream, &ix);
+    if (st != AH_OK) {
+        release();
+        return st;
+    }
+    for (int i = 0; i < 6; ++i) ix->loaded[i] = dev[i];
+    ix->owned_bytes += total;
+    *out = ix;
+    return AH_OK;
+}

@@ -79,6 +79,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_status_string": (ctypes.c_char_p, [I32]),
         "ah_last_error": (ctypes.c_char_p, []),
         "ah_search_leaves_noalloc": (I32, [P, P, I32, I32, P, P, P]),
+        "ah_save": (I32, [P, ctypes.c_char_p]),
+        "ah_inspect": (I32, [ctypes.c_char_p, P]),
+        "ah_load": (I32, [ctypes.c_char_p, P, ctypes.POINTER(P)]),
         "ah_set_option": (I32, [P, I32, I64]),
     }
     for name, (res, args) in sig.items():
@@ -102,6 +105,16 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def inspect(path: str) -> dict:
+    """Sizes of an index directory written by ``Index.save`` (no GPU needed):
+    n, d, num_leaves, dims_per_block, reorder_dtype ("f32", "bf16" or None)."""
+    lib = load_library()
+    v = Views()
+    _check(lib, lib.ah_inspect(os.fsencode(path), ctypes.byref(v)))
+    rdt = {AH_F32: "f32", AH_BF16: "bf16"}.get(v.reorder_dtype)
+    return dict(n=v.n, d=v.d, num_leaves=v.num_leaves, dims_per_block=v.dims_per_block, reorder_dtype=rdt)
 
 
 class Index:
@@ -143,6 +156,34 @@ class Index:
         with torch.cuda.device(dev):
             _check(self._lib, self._lib.ah_build_index_views(ctypes.byref(v), _stream(stream), ctypes.byref(h)))
         self._h = h
+
+    # -- index directories -----------------------------------------------------
+    def save(self, path: str):
+        """Write the index arrays to directory ``path`` (created if missing) as
+        .npy files plus ``ah_index.txt``; synchronous."""
+        os.makedirs(path, exist_ok=True)
+        with torch.cuda.device(self.device):
+            _check(self._lib, self._lib.ah_save(self._h, os.fsencode(path)))
+
+    @classmethod
+    def load(cls, path: str, device=None, stream=None) -> "Index":
+        """An index loaded from a directory written by ``save``; its arrays are
+        owned by the library (device memory freed by ``close``)."""
+        self = cls.__new__(cls)
+        self._lib = load_library()
+        if not torch.cuda.is_available():
+            raise AhError(4, "no CUDA device")
+        info = inspect(path)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        h = ctypes.c_void_p()
+        with torch.cuda.device(dev):
+            _check(self._lib, self._lib.ah_load(os.fsencode(path), _stream(stream), ctypes.byref(h)))
+        self._h = h
+        self.arrays = None
+        self.device = dev
+        self.n, self.d = info["n"], info["d"]
+        self.num_leaves, self.dims_per_block = info["num_leaves"], info["dims_per_block"]
+        return self
 
     # -- search ---------------------------------------------------------------
     def search(self, queries: torch.Tensor, k: int, num_leaves_to_search: int, reorder_num: int,
