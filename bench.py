@@ -437,6 +437,7 @@ def run_sweep(args):
                 index.search(qg, w.k, L, w.reorder_num, args.lut_mode)
                 e1.record(stream)
                 st = index.stage_times()
+                e1.synchronize()
                 ms.append(e0.elapsed_time(e1))
                 scan.append(st["scan"] + st.get("scan_rest", 0.0))
             index.set_profiling(True)       # per-stage breakdown, a few untimed steps

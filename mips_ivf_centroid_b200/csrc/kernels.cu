@@ -675,6 +675,8 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 
 // Slots sampled per query for the bound: the requested sample, at least 8R
 // (so about R/8 of the sample's points pass), at most kMaxThresholdSample.
+constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
+
 __host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
     return min(kMaxThresholdSample, max(max(R, requested), 8 * R));
 }
@@ -691,6 +693,8 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kSelThreads> rs;
+    __shared__ int seg_end[kThresholdSegs], seg_pos[kThresholdSegs], seg_slot[kThresholdSegs];
+    __shared__ int s_nseg, s_taken;
     const int q = blockIdx.x;
     const int R = a.R;
     unsigned char* lut = smem;
@@ -699,46 +703,106 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
     load_query_table<MODE>(ix, b, q, lut);
     __syncthreads();
     const int M = threshold_sample(R, a.threshold_sample);
-    // score slots [start, start + m) of the query's leaf of rank i into vals
-    int taken = 0;
-    auto score_range = [&](int i, int start, int m) {
-        const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
-        const int s0 = ix.offs[leaf] + start;
-        const int p0 = ix.ptile[leaf] * 32 + start;
-        for (int t0 = 0; t0 < m; t0 += 4 * kSelThreads) {
-            int32_t ps[4];
-            bool ok[4];
-            uint32_t v[4];
+    // The sample as segments (leaf, first slot, count) in order: the first
+    // M/S slots of each of the S best leaves, then the remaining slots of the
+    // leaves in rank order until M.  One warp builds the table with prefix
+    // sums; every thread then scores its sample indices in one pass, so a
+    // sample that spans several small leaves costs no extra passes.  A table
+    // that would exceed kThresholdSegs entries ends the sample early (a smaller
+    // subset still gives a valid bound).
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int64_t lrow = static_cast<int64_t>(q) * a.L;
+        const int S = max(1, min(a.L, a.threshold_leaves));
+        const int per = M / S;
+        int nseg = 0, taken = 0;
+        bool full = false;
+        // append this warp round's segments (cnt > 0) in lane order
+        auto append = [&](int cnt, int leaf, int start) {
+            int incl = cnt;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = t0 + u * kSelThreads + threadIdx.x;
-                ok[u] = t < m;
-                ps[u] = p0 + t;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += v;
             }
-            int32_t sid[4];              // loaded ahead, to overlap the code loads
-#pragma unroll
-            for (int u = 0; u < 4; ++u) sid[u] = ok[u] ? ix.slot_ids[s0 + t0 + u * kSelThreads + threadIdx.x] : 0;
-            slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, v);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = t0 + u * kSelThreads + threadIdx.x;
-                if (ok[u]) vals[taken + t] = make_key(v[u], sid[u]);
+            const unsigned m = __ballot_sync(0xFFFFFFFFu, cnt > 0);
+            const int idx = nseg + __popc(m & ((1u << lane) - 1u));
+            if (cnt > 0 && idx < kThresholdSegs) {
+                seg_end[idx] = taken + incl;
+                seg_pos[idx] = ix.ptile[leaf] * 32 + start;
+                seg_slot[idx] = ix.offs[leaf] + start;
             }
+            const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            const int n = __popc(m);
+            if (nseg + n > kThresholdSegs) {
+                // keep the first kThresholdSegs segments only
+                const unsigned lm = __ballot_sync(0xFFFFFFFFu, cnt > 0 && idx == kThresholdSegs - 1);
+                taken += __shfl_sync(0xFFFFFFFFu, incl, __ffs(lm) - 1);   // end of the last kept segment
+                nseg = kThresholdSegs;
+                full = true;
+            } else {
+                taken += total;
+                nseg += n;
+            }
+        };
+        for (int i0 = 0; i0 < S && !full; i0 += 32) {
+            const int i = i0 + lane;
+            int cnt = 0, leaf = 0;
+            if (i < S) {
+                leaf = b.leaves[lrow + i];
+                cnt = min(ix.offs[leaf + 1] - ix.offs[leaf], per);
+            }
+            append(cnt, leaf, 0);
         }
-        taken += m;
-    };
-    auto leaf_size = [&](int i) {
-        const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
-        return ix.offs[leaf + 1] - ix.offs[leaf];
-    };
-    // the first M/S slots of each of the S best leaves, then (if short) the
-    // remaining slots of the leaves in rank order
-    const int S = max(1, min(a.L, a.threshold_leaves));
-    const int per = M / S;
-    for (int i = 0; i < S; ++i) score_range(i, 0, min(leaf_size(i), per));
-    for (int i = 0; i < a.L && taken < M; ++i) {
-        const int start = (i < S) ? min(leaf_size(i), per) : 0;
-        score_range(i, start, min(leaf_size(i) - start, M - taken));
+        for (int i0 = 0; i0 < a.L && taken < M && !full; i0 += 32) {
+            const int i = i0 + lane;
+            int avail = 0, leaf = 0, start = 0;
+            if (i < a.L) {
+                leaf = b.leaves[lrow + i];
+                const int size = ix.offs[leaf + 1] - ix.offs[leaf];
+                start = (i < S) ? min(size, per) : 0;
+                avail = size - start;
+            }
+            int excl = avail;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, excl, off);
+                if (lane >= off) excl += v;
+            }
+            excl -= avail;
+            const int cnt = max(0, min(avail, M - taken - excl));
+            append(cnt, leaf, start);
+        }
+        if (lane == 0) {
+            s_nseg = nseg;
+            s_taken = taken;
+        }
+    }
+    __syncthreads();
+    const int nseg = s_nseg, taken = s_taken;
+    for (int t0 = 0; t0 < taken; t0 += 4 * kSelThreads) {
+        int32_t ps[4], sid[4];
+        bool ok[4];
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t0 + u * kSelThreads + threadIdx.x;
+            ok[u] = i < taken;
+            int lo = 0, hi = nseg - 1;                 // first segment whose end is above i
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (seg_end[mid] > i) hi = mid; else lo = mid + 1;
+            }
+            const int off = i - (lo > 0 ? seg_end[lo - 1] : 0);
+            ps[u] = seg_pos[lo] + off;
+            sid[u] = ok[u] ? ix.slot_ids[seg_slot[lo] + off] : 0;
+        }
+        slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t0 + u * kSelThreads + threadIdx.x;
+            if (ok[u]) vals[i] = make_key(v[u], sid[u]);
+        }
     }
     __syncthreads();
     if (taken <= 4 * kSelThreads) {
