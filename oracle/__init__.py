@@ -9,12 +9,15 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 * ``avq.py``: the training-side formulas the pages print: the eta ratio, the
   anisotropic loss and its closed-form center update ("The loss in one
   paragraph", "Training an anisotropic codebook yourself").
+* ``encode`` (``orc_encode`` in ah_oracle.c): anisotropic code assignment by
+  coordinate descent, the index-build step before the search.
 
 Parity pins: every function here is checked against something other than
-itself in ``tests/test_oracle_pins.py`` and ``tests/test_avq_pins.py``.  The
-one part without an independent pin is the choice of anisotropic codes by
-coordinate descent, which lives in the input generator, not here (parity
-unpinned there beyond the descent invariant).
+itself in ``tests/test_oracle_pins.py``, ``tests/test_avq_pins.py`` and
+``tests/test_encode_pins.py`` (the code assignment: eta = 1 gives the
+per-block nearest centers, the result is a coordinate-wise minimum of the
+loss computed independently, the loss never rises above the L2 codes' and
+exhaustive search on two blocks bounds it).
 """
 from __future__ import annotations
 
@@ -74,6 +77,8 @@ def _load():
         lib.orc_u8_table.argtypes = [P, P, P, P, P]
         lib.orc_u8_sums.argtypes = [P, P, ctypes.c_int64, P, P]
         lib.orc_max_threads.restype = ctypes.c_int
+        lib.orc_encode.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_double,
+                                   ctypes.c_int, P, P]
         _lib = lib
     return _lib
 
@@ -172,6 +177,24 @@ class OracleIndex:
         out = np.empty(slots.shape[0], np.uint32)
         _load().orc_u8_sums(self.ref, _ptr(q), slots.shape[0], _ptr(slots), _ptr(out))
         return out
+
+
+def encode(X, codebook, T: float, passes: int):
+    """Anisotropic code assignment (index build), ``orc_encode`` in ah_oracle.c.
+
+    X [n, d] float32, codebook [B, 16, dpb] float32; eta per point from T and
+    the point's norm (T <= 0: plain L2 codes).  Returns (codes [n, B/2] uint8
+    nibble-packed, passes_used [n] int32)."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    cb = np.ascontiguousarray(codebook, dtype=np.float32)
+    n, d = X.shape
+    B, _, dpb = cb.shape
+    if B * dpb != d or B % 2:
+        raise ValueError("codebook shape does not match d (B must be even)")
+    codes = np.empty((n, B // 2), np.uint8)
+    used = np.empty(n, np.int32)
+    _load().orc_encode(_ptr(X), n, d, dpb, _ptr(cb), float(T), int(passes), _ptr(codes), _ptr(used))
+    return codes, used
 
 
 def max_threads() -> int:

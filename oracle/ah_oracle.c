@@ -365,3 +365,128 @@ int orc_max_threads(void) {
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * Anisotropic code assignment (index build; ScaNN blog, "Training an
+ * anisotropic codebook yourself": codes minimise the anisotropic loss, and
+ * since blocks couple through r . u the assignment is refined iteratively).
+ *
+ * Reading used (one point x, B = d / dpb blocks of 16 centers):
+ *   norm = sqrt(sum_t x_t^2); u_t = x_t / norm; t_ = (T / norm)^2 and
+ *   eta = (d - 1) t_ / (1 - t_) ("The loss in one paragraph"), or eta = 1
+ *   when T <= 0, norm = 0 or t_ >= 1 (no valid anisotropic weight).
+ *   Loss of a reconstruction x~: (eta - 1) (r . u)^2 + ||r||^2, r = x - x~.
+ *   Start: per block the center of least squared error (ties: lower index).
+ *   Then up to `passes` passes over b = 0..B-1; per block, with the other
+ *   blocks fixed, the center of least loss (ties: lower index) replaces the
+ *   current one only if its loss is strictly lower; a pass without a change
+ *   ends the descent.
+ * Arithmetic in fp64, every sum over a block's coordinates in ascending
+ * order, multiplications and additions rounded separately (no fused
+ * multiply-add), in this order:
+ *   rpar = sum_t (x_t - x~_t) u_t, rn2 = sum_t (x_t - x~_t)^2 over all t;
+ *   per block: wp = rpar - sum_s (x_s - c_cur,s) u_s, wn = rn2 - sum_s
+ *   (x_s - c_cur,s)^2; per center j: p_j = wp + sum_s (x_s - c_j,s) u_s,
+ *   n_j = wn + sum_s (x_s - c_j,s)^2, loss_j = (eta - 1) (p_j p_j) + n_j;
+ *   on a change rpar = p_best, rn2 = n_best.
+ * Output: codes [n][B/2] nibble-packed (block 2i low nibble of byte i);
+ * passes_used[i] = passes run for point i (0 when none was needed).
+ * ------------------------------------------------------------------------ */
+void orc_encode(const float *X, int64_t n, int d, int dpb, const float *codebook, double T, int passes,
+                uint8_t *codes, int32_t *passes_used) {
+    const int B = d / dpb;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t i = 0; i < n; ++i) {
+        const float *xr = X + i * (int64_t)d;
+        int code[4096];
+        double nrm2 = 0.0;
+        for (int t = 0; t < d; ++t) nrm2 = nrm2 + (double)xr[t] * (double)xr[t];
+        const double norm = sqrt(nrm2);
+        double eta = 1.0;
+        if (T > 0.0 && norm > 0.0) {
+            const double tt = (T / norm) * (T / norm);
+            if (tt < 1.0) eta = ((double)(d - 1) * tt) / (1.0 - tt);
+        }
+        const double e1 = eta - 1.0;
+        /* L2 start */
+        for (int b = 0; b < B; ++b) {
+            int best = 0;
+            double bestv = 0.0;
+            for (int j = 0; j < 16; ++j) {
+                double e = 0.0;
+                for (int s = 0; s < dpb; ++s) {
+                    const double df = (double)xr[b * dpb + s] - (double)codebook[((int64_t)b * 16 + j) * dpb + s];
+                    e = e + df * df;
+                }
+                if (j == 0 || e < bestv) {
+                    bestv = e;
+                    best = j;
+                }
+            }
+            code[b] = best;
+        }
+        double rpar = 0.0, rn2 = 0.0;
+        for (int b = 0; b < B; ++b)
+            for (int s = 0; s < dpb; ++s) {
+                const int t = b * dpb + s;
+                const double x = (double)xr[t];
+                const double u = norm > 0.0 ? x / norm : 0.0;
+                const double r = x - (double)codebook[((int64_t)b * 16 + code[b]) * dpb + s];
+                rpar = rpar + r * u;
+                rn2 = rn2 + r * r;
+            }
+        int used = 0;
+        for (int p = 0; p < passes; ++p) {
+            int changed = 0;
+            for (int b = 0; b < B; ++b) {
+                const float *cb = codebook + (int64_t)b * 16 * dpb;
+                const int cur = code[b];
+                double wp = rpar, wn = rn2;
+                {
+                    double sp = 0.0, sn = 0.0;
+                    for (int s = 0; s < dpb; ++s) {
+                        const double x = (double)xr[b * dpb + s];
+                        const double u = norm > 0.0 ? x / norm : 0.0;
+                        const double r = x - (double)cb[cur * dpb + s];
+                        sp = sp + r * u;
+                        sn = sn + r * r;
+                    }
+                    wp = wp - sp;
+                    wn = wn - sn;
+                }
+                int best = 0;
+                double bl = 0.0, bp = 0.0, bn = 0.0, lcur = 0.0;
+                for (int j = 0; j < 16; ++j) {
+                    double sp = 0.0, sn = 0.0;
+                    for (int s = 0; s < dpb; ++s) {
+                        const double x = (double)xr[b * dpb + s];
+                        const double u = norm > 0.0 ? x / norm : 0.0;
+                        const double r = x - (double)cb[j * dpb + s];
+                        sp = sp + r * u;
+                        sn = sn + r * r;
+                    }
+                    const double pj = wp + sp, nj = wn + sn;
+                    const double l = e1 * (pj * pj) + nj;
+                    if (j == cur) lcur = l;
+                    if (j == 0 || l < bl) {
+                        bl = l;
+                        best = j;
+                        bp = pj;
+                        bn = nj;
+                    }
+                }
+                if (bl < lcur) {
+                    code[b] = best;
+                    rpar = bp;
+                    rn2 = bn;
+                    ++changed;
+                }
+            }
+            used = p + 1;
+            if (changed == 0) break;
+        }
+        if (passes_used) passes_used[i] = used;
+        uint8_t *out = codes + i * (int64_t)(B / 2);
+        for (int b = 0; b < B; b += 2) out[b / 2] = (uint8_t)(code[b] | (code[b + 1] << 4));
+    }
+}
