@@ -58,6 +58,9 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=100)
     p.add_argument("--sweep", action="store_true",
                    help="sweep workload: one JSON line per (batch, leaves) point instead of the single line")
+    p.add_argument("--encode", action="store_true",
+                   help="index build: time the anisotropic code assignment over the workload's points")
+    p.add_argument("--passes", type=int, default=10)
     return p.parse_args()
 
 
@@ -463,10 +466,69 @@ def run_sweep(args):
     index.close()
 
 
+def run_encode(args):
+    """One JSON line: anisotropic code assignment (ah_encode) of the workload's
+    n points against its trained codebook, points/s on the device (inputs
+    resident), with the oracle's restatement timed on a sample of points."""
+    import torch
+    from mips_ivf_centroid_b200 import build as ahbuild, datagen
+    ahbuild.build()
+    from mips_ivf_centroid_b200 import encode
+    import oracle
+    w = workload_spec(args)
+    T = w.threshold_T or 0.0
+    X = datagen.make_data(w)
+    ix = datagen.build_index(w, X, "cuda")
+    Xg = torch.from_numpy(X).cuda()
+    cb = ix.codebook
+    stream = torch.cuda.current_stream()
+    codes, used = encode(Xg, cb, T, args.passes)
+    for _ in range(args.warmup):
+        encode(Xg, cb, T, args.passes, out=codes, passes_used=used)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            encode(Xg, cb, T, args.passes, out=codes, passes_used=used)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    up = used.cpu().numpy().astype(np.int64)
+    B, dpb = w.blocks, w.dims_per_block
+    # fp64 operations the descent performs: start (16 centers x dpb x 3 per
+    # block), residual sums (dpb x 5 per block), and per pass and block 16
+    # centers x (dpb x 6 + 5) plus the current center's dpb x 6
+    ops = float(w.n) * (2 * w.d + B * (16 * dpb * 3 + dpb * 5)) + float(up.sum()) * B * (16 * (6 * dpb + 5) + 6 * dpb)
+    mhz = SM_MAX_MHZ_FALLBACK
+    peak = SM_COUNT * 64 * mhz * 1e6          # fp64 ops per second, one per lane per clock
+    # oracle on a sample of points
+    ns = min(w.n, 20000)
+    t0 = time.perf_counter()
+    ocodes, oused = oracle.encode(X[:ns], cb.cpu().numpy(), T, args.passes)
+    ot = time.perf_counter() - t0
+    same = bool(np.array_equal(ocodes, codes[:ns].cpu().numpy()))
+    line = {"metric": "anisotropic code assignment points/s (1 B200)", "value": w.n / (ms * 1e-3),
+            "unit": "points/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Gaussian mixture; codebook trained on it)",
+            "config": {"workload": f"{w.name}-shaped: n={w.n:,} d={w.d} dims_per_block={dpb} T={T} passes<={args.passes}"},
+            "passes_mean": float(up.mean()),
+            "roofline": {"bound": "alu", "achieved": ops / (ms * 1e-3) / 1e12, "peak": peak / 1e12,
+                         "unit": "Tops/s (fp64)", "frac": ops / (ms * 1e-3) / peak, "traffic": None,
+                         "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 lanes x {mhz:.0f} MHz (nominal rate)"},
+            "cpu_baseline": {"value": ns / ot, "unit": "points/s", "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": f"first {ns} points"},
+            "oracle_match_on_sample": same, "clocks": clk.summary(), "gpu_launches": args.steps + args.warmup + 1}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.encode:
+        run_encode(args)
     elif args.sweep:
         run_sweep(args)
     else:

@@ -314,6 +314,33 @@ AH_API ah_status ah_inspect(const char *dir, ah_index_views *out);
  */
 AH_API ah_status ah_load(const char *dir, void *cuda_stream, ah_index **out);
 
+/*
+ * Anisotropic code assignment, the index-build step before the search (ScaNN
+ * blog, "Training an anisotropic codebook yourself": codes minimise the
+ * anisotropic loss; blocks couple through r . u, so the assignment is refined
+ * iteratively).  For each point x (row of X):
+ *   eta = (d - 1) t / (1 - t), t = (T / ||x||)^2 ("The loss in one
+ *   paragraph"); eta = 1 when T <= 0, ||x|| = 0 or t >= 1;
+ *   loss(x~) = (eta - 1) ((x - x~) . x / ||x||)^2 + ||x - x~||^2;
+ *   start from the nearest center of every block (ties: lower index), then up
+ *   to `passes` passes over blocks 0..B-1, each replacing a block's center by
+ *   the one of least loss with the other blocks fixed when that is strictly
+ *   lower (ties: lower index); a pass without a change ends the descent.
+ * fp64 arithmetic, each product and sum rounded separately, sums over a
+ * block's coordinates in ascending order (the order is part of the result).
+ *   X           [n][d] float, device
+ *   codebook    [d/dims_per_block][16][dims_per_block] float, device
+ *   codes       [n][d/dims_per_block/2] uint8 out, device: block 2i in the
+ *               low nibble of byte i
+ *   passes_used [n] int32 out, device, or NULL: passes run per point
+ * Asynchronous on cuda_stream; nothing is allocated.  Errors:
+ * AH_ERR_INVALID_ARG (NULL array, n < 0, d not divisible by
+ * 2 * dims_per_block, passes outside [0, 1000]), AH_ERR_UNSUPPORTED (more
+ * than AH_MAX_BLOCKS blocks), AH_ERR_CUDA.
+ */
+AH_API ah_status ah_encode(const float *X, int64_t n, int32_t d, int32_t dims_per_block, const float *codebook,
+                           double T, int32_t passes, uint8_t *codes, int32_t *passes_used, void *cuda_stream);
+
 AH_API void ah_destroy(ah_index *ix);
 
 /* Static text for a status code. */

@@ -251,7 +251,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     // is raised to the R-th best point kept (and its buffer compacted).
     std::vector<int> bounds{0};
     {
-        const int M = std::min(4096, std::max(std::max(a.R, ix->opt_threshold_sample), 8 * a.R));
+        const int M = ah::threshold_sample(a.R, ix->opt_threshold_sample);
         const double avg_leaf = static_cast<double>(dix.n) / dix.nl;
         const double expect_one_pass = 0.25 * a.R * L * avg_leaf / M;   // points kept by the sample's bound
         int first = L;
@@ -862,4 +862,26 @@ ah_status ah_load(const char* dir, void* cuda_stream, ah_index** out) {
     ix->owned_bytes += total;
     *out = ix;
     return AH_OK;
+}
+
+// ---------------------------------------------------------------------------
+// anisotropic code assignment
+// ---------------------------------------------------------------------------
+
+ah_status ah_encode(const float* X, int64_t n, int32_t d, int32_t dims_per_block, const float* codebook, double T,
+                    int32_t passes, uint8_t* codes, int32_t* passes_used, void* cuda_stream) {
+    if (n < 0) return fail(AH_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return AH_OK;
+    if (!X || !codebook || !codes) return fail(AH_ERR_INVALID_ARG, "NULL array");
+    if (d <= 0 || dims_per_block <= 0 || d % (2 * dims_per_block) != 0)
+        return fail(AH_ERR_INVALID_ARG, "d not a positive multiple of 2 * dims_per_block");
+    if (d / dims_per_block > AH_MAX_BLOCKS) return fail(AH_ERR_UNSUPPORTED, "blocks above AH_MAX_BLOCKS");
+    if (passes < 0 || passes > 1000) return fail(AH_ERR_INVALID_ARG, "passes outside [0, 1000]");
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = ah::launch_encode(X, n, d, dims_per_block, codebook, T, passes, codes, passes_used, sms,
+                              static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? AH_OK : cuda_fail(e, "encode");
 }

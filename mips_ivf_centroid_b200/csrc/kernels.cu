@@ -187,10 +187,112 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __res
     }
 }
 
-// 64x64 tiles, 32x32 for very small problems (more CTAs in flight).
+// 128x128 output tile per CTA of 256 threads, 8x8 outputs per thread (two
+// 4-wide fragments per dimension, read as float4 from shared memory), k in
+// steps of 8 with the next step's operands loaded from global memory while
+// the current one is multiplied.  Each output accumulates over k in ascending
+// order with fmaf, as the 64-wide kernel does, so both give identical scores.
+// VEC: d % 4 == 0 and 16-byte aligned rows, so operands load as float4.
+template <bool VEC>
+__global__ void __launch_bounds__(256, 2) centroid_scores128_kernel(const float* __restrict__ Q,
+                                                                    const float* __restrict__ C,
+                                                                    float* __restrict__ S, int nq, int nl, int d) {
+    chain_entry();
+    constexpr int T = 128, BK = 8, P = T + 4;
+    __shared__ __align__(16) float As[2][BK][P];
+    __shared__ __align__(16) float Bs[2][BK][P];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int m0 = blockIdx.y * T, n0 = blockIdx.x * T;
+    const int lrow = tid >> 1, lk = (tid & 1) * 4;      // operand row and first k this thread loads
+    float ra[4], rb[4];
+    auto gload = [&](int k0) {
+        const int gk = k0 + lk, gm = m0 + lrow, gn = n0 + lrow;
+        if (VEC) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), c = a;
+            if (gm < nq && gk < d) a = *reinterpret_cast<const float4*>(Q + static_cast<int64_t>(gm) * d + gk);
+            if (gn < nl && gk < d) c = *reinterpret_cast<const float4*>(C + static_cast<int64_t>(gn) * d + gk);
+            ra[0] = a.x; ra[1] = a.y; ra[2] = a.z; ra[3] = a.w;
+            rb[0] = c.x; rb[1] = c.y; rb[2] = c.z; rb[3] = c.w;
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                ra[t] = (gm < nq && gk + t < d) ? Q[static_cast<int64_t>(gm) * d + gk + t] : 0.0f;
+                rb[t] = (gn < nl && gk + t < d) ? C[static_cast<int64_t>(gn) * d + gk + t] : 0.0f;
+            }
+        }
+    };
+    auto sstore = [&](int buf) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            As[buf][lk + t][lrow] = ra[t];
+            Bs[buf][lk + t][lrow] = rb[t];
+        }
+    };
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    gload(0);
+    sstore(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += BK) {
+        const bool more = k0 + BK < d;
+        if (more) gload(k0 + BK);
+#pragma unroll
+        for (int kk = 0; kk < BK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        if (more) sstore(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+    }
+    const bool vstore = VEC && (nl % 4 == 0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+        if (gm >= nq) continue;
+        float* row = S + static_cast<int64_t>(gm) * nl;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int gn = n0 + 64 * h + tx * 4;
+            if (vstore && gn + 3 < nl) {
+                *reinterpret_cast<float4*>(row + gn) =
+                    make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    if (gn + t < nl) row[gn + t] = acc[i][4 * h + t];
+            }
+        }
+    }
+}
+
+// 128x128 tiles for large batches, 64x64 for mid-size ones, 32x32 for very
+// small problems (more CTAs in flight).
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
     const int64_t big = static_cast<int64_t>((ix.nl + 63) / 64) * ((a.nq + 63) / 64);
-    if (big >= 64) {
+    const int64_t tiles128 = static_cast<int64_t>((ix.nl + 127) / 128) * ((a.nq + 127) / 128);
+    if (tiles128 >= 256) {                   // enough 128-wide tiles to fill every SM twice
+        dim3 grid((ix.nl + 127) / 128, (a.nq + 127) / 128);
+        const bool vec = ix.d % 4 == 0 && reinterpret_cast<uintptr_t>(a.queries) % 16 == 0 &&
+                         reinterpret_cast<uintptr_t>(ix.centroids) % 16 == 0;
+        const cudaError_t le = vec ? launch_chained(centroid_scores128_kernel<true>, grid, dim3(256), 0, s, a.queries,
+                                                    ix.centroids, b.cscore, a.nq, ix.nl, ix.d)
+                                   : launch_chained(centroid_scores128_kernel<false>, grid, dim3(256), 0, s, a.queries,
+                                                    ix.centroids, b.cscore, a.nq, ix.nl, ix.d);
+        if (le != cudaSuccess) return le;
+    } else if (big >= 64) {
         dim3 grid((ix.nl + 63) / 64, (a.nq + 63) / 64);
         if (const cudaError_t le = launch_chained(centroid_scores_kernel<64>, dim3(grid), dim3(256), 0, s, a.queries, ix.centroids, b.cscore, a.nq, ix.nl, ix.d); le != cudaSuccess) return le;
     } else {
@@ -329,6 +431,65 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_reg_kernel(DeviceIndex
 }
 
 constexpr int kReorderBatch = AH_REORDER_BATCH;
+// One CTA per query, two warp-level stages: warp w keeps the best L of its
+// slice of the score row (KPL keys per lane, in registers), then warp 0 keeps
+// the best L of the 8 slices' survivors (at most 8 L <= 512 keys).  One
+// barrier in all.  For 1024 < centroids <= 8 * 32 * KPL and L <= 64.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads) top_leaves_2stage_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
+    __shared__ uint64_t cand[8 * 64];
+    __shared__ uint64_t keys[64];
+    __shared__ int s_count;
+    const int q = blockIdx.x;
+    const int L = a.L, nl = ix.nl;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* row = b.cscore + static_cast<int64_t>(q) * nl;
+    const int per = (nl + 7) / 8;
+    const int lo = warp * per, n = max(0, min(per, nl - lo));
+    if (threadIdx.x == 0) s_count = 0;
+    __syncthreads();
+    {
+        uint64_t k[KPL];
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+            const int i = lane + 32 * j;
+            k[j] = (i < n) ? make_key(float_key(row[lo + i]), lo + i) : 0ull;
+        }
+        const int keep = min(L, n);
+        if (keep > 0) {
+            const uint64_t thr = (keep < n) ? warp_kth_reg<KPL>(k, n, keep) : 1ull;
+            int base = 0;
+            if (lane == 0) base = atomicAdd(&s_count, keep);
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) {
+                const bool sel = k[j] != 0ull && k[j] >= thr;
+                const unsigned m = __ballot_sync(0xFFFFFFFFu, sel);
+                if (sel) cand[base + __popc(m & ((1u << lane) - 1u))] = k[j];
+                base += __popc(m);
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int tot = s_count;
+        warp_topk_src<16>(cand, static_cast<const int32_t*>(nullptr), tot, L, keys, static_cast<int32_t*>(nullptr), true);
+        long long local = 0;
+        for (int i = lane; i < L; i += 32) {
+            const uint64_t key = keys[i];
+            const int leaf = key_id(key);
+            b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
+            b.leaf_scores[static_cast<int64_t>(q) * L + i] = key_float(key_score(key));
+            if (i < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);
+            local += ix.offs[leaf + 1] - ix.offs[leaf];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, off);
+        if (lane == 0) b.scanned[q] = local;
+    }
+}
+
 constexpr int kTopWarps = 8;
 
 // One warp per query when the centroids fit 32 per lane: the scores stay in
@@ -365,6 +526,13 @@ cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchB
         cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_warp_kernel), smem, false);
         if (e != cudaSuccess) return e;
         if (const cudaError_t le = launch_chained(top_leaves_warp_kernel, dim3((a.nq + kTopWarps - 1) / kTopWarps), dim3(kTopWarps * 32), smem, s, ix, a, b); le != cudaSuccess) return le;
+        return cudaGetLastError();
+    }
+    if (ix.nl <= 16 * kSelThreads && a.L <= 64) {
+        const cudaError_t le = (ix.nl <= 8 * kSelThreads)
+            ? launch_chained(top_leaves_2stage_kernel<8>, dim3(a.nq), dim3(kSelThreads), 0, s, ix, a, b)
+            : launch_chained(top_leaves_2stage_kernel<16>, dim3(a.nq), dim3(kSelThreads), 0, s, ix, a, b);
+        if (le != cudaSuccess) return le;
         return cudaGetLastError();
     }
     if (ix.nl <= 16 * kSelThreads) {
@@ -478,7 +646,7 @@ cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const Sear
         if (e != cudaSuccess) return e;
         if (const cudaError_t le = launch_chained(invert_count_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     }
-    if (const cudaError_t le = launch_chained(invert_offsets_kernel, dim3(1), dim3(kScanBlock), 0, s, ix, b, scan_group(a.lut_mode), a.chunk); le != cudaSuccess) return le;
+    if (const cudaError_t le = launch_chained(invert_offsets_kernel, dim3(1), dim3(kScanBlock), 0, s, ix, b, scan_group(ix, a.lut_mode), a.chunk); le != cudaSuccess) return le;
     if (const cudaError_t le = launch_chained(invert_scatter_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
@@ -673,13 +841,8 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 // threshold: R-th best approximate score over a prefix of the best leaves
 // ---------------------------------------------------------------------------
 
-// Slots sampled per query for the bound: the requested sample, at least 8R
-// (so about R/8 of the sample's points pass), at most kMaxThresholdSample.
-constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
 
-__host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
-    return min(kMaxThresholdSample, max(max(R, requested), 8 * R));
-}
+constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
 
 // One CTA per query.  Scores a sample of M = min(points, threshold_sample)
 // slots of the query's best leaves (an even share of the S best, topped up in
@@ -1034,11 +1197,10 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
 
-template <int MODE, int NT>
-__global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : 1)) scan_kernel(DeviceIndex ix, SearchArgs a,
-                                                                                         SearchBuffers b) {
+template <int MODE, int NT, int GMAX>
+__global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 512 ? 2 : 1)))
+    scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
-    constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
     constexpr int GSTEP = (MODE == 0) ? 2 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_item, s_leaf;
@@ -1148,32 +1310,64 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : 1)) scan
     }
 }
 
-int scan_group(int lut_mode) { return lut_mode == 0 ? kGroupF32 : kGroupU8; }
+// Scan CTA shape: threads per CTA and queries per group.  Narrow tables
+// (a full group's tables within 64 KB): 256 threads, groups of 8 (fp32) or
+// 16 (uint8) queries, several CTAs per SM.  Wide tables: two CTAs of 512
+// threads per SM with half-size groups, so one CTA's table staging and
+// item-end barrier overlap the other's scanning.
+#ifndef AH_WIDE_SPLIT
+#define AH_WIDE_SPLIT 1
+#endif
+void scan_shape(const DeviceIndex& ix, int lut_mode, int* nt, int* gmax) {
+    const int g = lut_mode == 0 ? kGroupF32 : kGroupU8;
+    const size_t table = static_cast<size_t>(ix.B) * kCenters * (lut_mode == 0 ? 4 : 1) * g;
+    if (table <= 64 * 1024) {
+        *nt = 256;
+        *gmax = g;
+    } else if (AH_WIDE_SPLIT && table / 2 <= 100 * 1024) {
+        *nt = 512;
+        *gmax = g / 2;
+    } else {
+        *nt = 1024;
+        *gmax = g;
+    }
+}
 
-template <int MODE, int NT>
+int scan_group(const DeviceIndex& ix, int lut_mode) {
+    int nt, g;
+    scan_shape(ix, lut_mode, &nt, &g);
+    return g;
+}
+
+template <int MODE, int NT, int GMAX>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
-    constexpr int GMAX = (MODE == 0) ? kGroupF32 : kGroupU8;
     size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
-    a.scan_item_off_smem = (smem + off_bytes <= 200 * 1024 && off_bytes <= 64 * 1024) ? 1 : 0;
+    const size_t room = (NT == 512) ? 110 * 1024 : 200 * 1024;
+    a.scan_item_off_smem = (smem + off_bytes <= room && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT>), smem, true);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT, GMAX>), smem, true);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT>, NT, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT, GMAX>, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
+    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT, GMAX>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
-// Wide tables leave room for one CTA per SM: use 1024 threads then.
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s) {
-    const size_t table = static_cast<size_t>(ix.B) * (a.lut_mode == 0 ? kGroupF32 * kCenters * 4 : kGroupU8 * kCenters);
-    const bool wide = table > 64 * 1024;
-    if (a.lut_mode == 0) return wide ? launch_scan_t<0, 1024>(ix, a, b, num_sms, s) : launch_scan_t<0, 256>(ix, a, b, num_sms, s);
-    return wide ? launch_scan_t<1, 1024>(ix, a, b, num_sms, s) : launch_scan_t<1, 256>(ix, a, b, num_sms, s);
+    int nt, g;
+    scan_shape(ix, a.lut_mode, &nt, &g);
+    if (a.lut_mode == 0) {
+        if (nt == 256) return launch_scan_t<0, 256, kGroupF32>(ix, a, b, num_sms, s);
+        if (nt == 512) return launch_scan_t<0, 512, kGroupF32 / 2>(ix, a, b, num_sms, s);
+        return launch_scan_t<0, 1024, kGroupF32>(ix, a, b, num_sms, s);
+    }
+    if (nt == 256) return launch_scan_t<1, 256, kGroupU8>(ix, a, b, num_sms, s);
+    if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2>(ix, a, b, num_sms, s);
+    return launch_scan_t<1, 1024, kGroupU8>(ix, a, b, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------

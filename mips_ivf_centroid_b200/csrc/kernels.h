@@ -12,7 +12,20 @@ namespace ah {
 constexpr int kGroupF32 = 8;
 constexpr int kGroupU8 = 16;
 constexpr int kScanThreads = 256;
+#ifndef AH_SAMPLE_MULT
+#define AH_SAMPLE_MULT 8
+#endif
+constexpr int kSampleMult = AH_SAMPLE_MULT;       // the threshold sample holds at least this many times R slots
 constexpr int kMaxThresholdSample = 4096;   // slots scored per query for the threshold
+
+// Slots sampled per query for the filter bound: the requested sample, at
+// least kSampleMult R (so a small share of them passes), at most
+// kMaxThresholdSample.
+__host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
+    const int m = (R > requested ? R : requested);
+    const int want = m > kSampleMult * R ? m : kSampleMult * R;
+    return want < kMaxThresholdSample ? want : kMaxThresholdSample;
+}
 
 struct DeviceIndex {
     int64_t n;
@@ -100,7 +113,12 @@ cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffe
 cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int round,
                              int num_sms, cudaStream_t s);
 
-int scan_group(int lut_mode);
+int scan_group(const DeviceIndex& ix, int lut_mode);
 size_t finish_smem_bytes(int R, int d);
+
+// anisotropic code assignment (encode.cu)
+size_t encode_smem_bytes(int d, int dpb, bool* cb_in_smem);
+cudaError_t launch_encode(const float* X, int64_t n, int d, int dpb, const float* codebook, double T, int passes,
+                          uint8_t* codes, int32_t* passes_used, int num_sms, cudaStream_t s);
 
 }  // namespace ah

@@ -79,6 +79,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_status_string": (ctypes.c_char_p, [I32]),
         "ah_last_error": (ctypes.c_char_p, []),
         "ah_search_leaves_noalloc": (I32, [P, P, I32, I32, P, P, P]),
+        "ah_encode": (I32, [P, I64, I32, I32, P, ctypes.c_double, I32, P, P, P]),
         "ah_save": (I32, [P, ctypes.c_char_p]),
         "ah_inspect": (I32, [ctypes.c_char_p, P]),
         "ah_load": (I32, [ctypes.c_char_p, P, ctypes.POINTER(P)]),
@@ -105,6 +106,33 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def encode(X: torch.Tensor, codebook: torch.Tensor, T: float, passes: int = 10, stream=None,
+           out: Optional[torch.Tensor] = None, passes_used: Optional[torch.Tensor] = None):
+    """Anisotropic codes of the rows of X (index build, ``ah_encode``).
+
+    X [n, d] float32 and codebook [B, 16, dpb] float32 on one CUDA device.
+    Returns (codes [n, B/2] uint8, passes_used [n] int32), asynchronous on the
+    stream."""
+    lib = load_library()
+    if X.dtype != torch.float32 or X.dim() != 2 or not X.is_contiguous() or X.device.type != "cuda":
+        raise AhError(1, "X: need contiguous float32 [n, d] on a CUDA device")
+    if codebook.dtype != torch.float32 or codebook.dim() != 3 or not codebook.is_contiguous() \
+            or codebook.device != X.device:
+        raise AhError(1, "codebook: need contiguous float32 [B, 16, dpb] on X's device")
+    n, d = X.shape
+    B, _, dpb = codebook.shape
+    if B * dpb != d or codebook.shape[1] != 16:
+        raise AhError(1, "codebook: need [d / dims_per_block, 16, dims_per_block]")
+    if out is None:
+        out = torch.empty((n, B // 2), dtype=torch.uint8, device=X.device)
+    if passes_used is None:
+        passes_used = torch.empty((n,), dtype=torch.int32, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib, lib.ah_encode(_ptr(X), n, d, dpb, _ptr(codebook), float(T), int(passes), _ptr(out),
+                                  _ptr(passes_used), _stream(stream)))
+    return out, passes_used
 
 
 def inspect(path: str) -> dict:

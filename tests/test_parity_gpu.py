@@ -46,6 +46,11 @@ def _workload(name):
                                          n_means=100, training_sample_size=30_000),
         "leaves-5000": W["glove"].scaled(n=50_000, d=32, num_leaves=5000, num_leaves_to_search=16, nq=128,
                                          n_means=100, training_sample_size=50_000),
+        "gemm128-vec": W["glove"].scaled(n=40_000, d=64, num_leaves=2048, num_leaves_to_search=8, nq=2048,
+                                         n_means=100, training_sample_size=40_000),
+        "gemm128-scalar": W["glove"].scaled(n=40_000, d=34, dims_per_block=1, num_leaves=2048,
+                                            num_leaves_to_search=8, nq=2048, n_means=100,
+                                            training_sample_size=40_000),
         "small-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=600, num_leaves_to_search=2, nq=64,
                                           n_means=10, training_sample_size=3_000, code_loss="l2",
                                           threshold_T=None),
@@ -163,12 +168,25 @@ def test_sweep_mini(Index):
     compare(Index, "sweep-mini", 10, 64, 100, 0)
 
 
-@pytest.mark.parametrize("name", ["leaves-1500", "leaves-3000", "leaves-5000"])
-def test_many_centroids(Index, name):
-    # more centroids than one warp holds in registers (two register widths)
-    # and more than the block's register form holds (shared-memory radix)
-    w = _workload(name)[0]
-    compare(Index, name, 10, w.num_leaves_to_search, 100, 0)
+@pytest.mark.parametrize("name,L", [("leaves-1500", 40), ("leaves-3000", 64), ("leaves-3000", 100),
+                                    ("leaves-5000", 16)])
+def test_many_centroids(Index, name, L):
+    # more centroids than one warp holds in registers: two-stage warp selection
+    # (two register widths, L <= 64), the block's register form (L > 64), and
+    # beyond 4096 centroids the shared-memory radix
+    compare(Index, name, 10, L, 100, 0)
+
+
+@pytest.mark.parametrize("name", ["gemm128-vec", "gemm128-scalar"])
+def test_large_batch_centroid_tiles(Index, name):
+    # 2048 queries x 2048 centroids: the 128-wide centroid tiles (float4 operand
+    # loads when d % 4 == 0, scalar ones otherwise); the whole batch is searched,
+    # a sample of queries is checked stage by stage
+    from parity import compare_search
+    w, X, Q, ix, arr = _workload(name)
+    index = Index(ix)
+    compare_search(index, arr, Q, 10, w.num_leaves_to_search, 100, 0, qsel=np.arange(0, w.nq, 16))
+    index.close()
 
 
 def test_all_leaves(Index):
