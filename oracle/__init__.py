@@ -11,10 +11,12 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
   paragraph", "Training an anisotropic codebook yourself").
 * ``encode`` (``orc_encode`` in ah_oracle.c): anisotropic code assignment by
   coordinate descent, the index-build step before the search.
+* ``kmeans_assign`` / ``kmeans_update``: partition training (nearest centroid,
+  centroid means), the other index-build step.
 
 Parity pins: every function here is checked against something other than
 itself in ``tests/test_oracle_pins.py``, ``tests/test_avq_pins.py`` and
-``tests/test_encode_pins.py`` (the code assignment: eta = 1 gives the
+``tests/test_encode_pins.py``, ``tests/test_kmeans_pins.py`` (the code assignment: eta = 1 gives the
 per-block nearest centers, the result is a coordinate-wise minimum of the
 loss computed independently, the loss never rises above the L2 codes' and
 exhaustive search on two blocks bounds it).
@@ -79,6 +81,8 @@ def _load():
         lib.orc_max_threads.restype = ctypes.c_int
         lib.orc_encode.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, ctypes.c_double,
                                    ctypes.c_int, P, P]
+        lib.orc_kmeans_assign.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, ctypes.c_int, P, P]
+        lib.orc_kmeans_update.argtypes = [P, ctypes.c_int64, ctypes.c_int, P, ctypes.c_int, P, P, P]
         _lib = lib
     return _lib
 
@@ -195,6 +199,31 @@ def encode(X, codebook, T: float, passes: int):
     used = np.empty(n, np.int32)
     _load().orc_encode(_ptr(X), n, d, dpb, _ptr(cb), float(T), int(passes), _ptr(codes), _ptr(used))
     return codes, used
+
+
+def kmeans_assign(X, C):
+    """Nearest centroid of every row of X (``orc_kmeans_assign``): (assign [n]
+    int32, squared distance [n] float64)."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    C = np.ascontiguousarray(C, dtype=np.float32)
+    n, d = X.shape
+    a = np.empty(n, np.int32)
+    dist = np.empty(n, np.float64)
+    _load().orc_kmeans_assign(_ptr(X), n, d, _ptr(C), C.shape[0], _ptr(a), _ptr(dist))
+    return a, dist
+
+
+def kmeans_update(X, assign, C_old):
+    """Centroid means (``orc_kmeans_update``): (C_new [nl, d] float32, counts [nl] int64)."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    a = np.ascontiguousarray(assign, dtype=np.int32)
+    C_old = np.ascontiguousarray(C_old, dtype=np.float32)
+    n, d = X.shape
+    nl = C_old.shape[0]
+    C_new = np.empty_like(C_old)
+    counts = np.empty(nl, np.int64)
+    _load().orc_kmeans_update(_ptr(X), n, d, _ptr(a), nl, _ptr(C_old), _ptr(C_new), _ptr(counts))
+    return C_new, counts
 
 
 def max_threads() -> int:

@@ -490,3 +490,59 @@ void orc_encode(const float *X, int64_t n, int d, int dpb, const float *codebook
         for (int b = 0; b < B; b += 2) out[b / 2] = (uint8_t)(code[b] | (code[b + 1] << 4));
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Partition training (index build; ScaNN blog, "Using the library": the
+ * tree's leaves are trained by k-means on a sample of the data, and every
+ * point goes to its nearest leaf).
+ *
+ * Reading used:
+ *   assignment  a_i = argmin_c sum_t (x_it - c_t)^2, fp64, t ascending, each
+ *               difference, square and sum rounded separately; ties go to
+ *               the lower centroid index; dist_i = that minimum.
+ *   update      for each centroid c with members (a_i = c, i ascending):
+ *               s_t = sum_i x_it in fp64 in ascending i, new c_t = s_t / m
+ *               (fp64 division) rounded to float; a centroid without
+ *               members keeps its value; counts_c = m.
+ * ------------------------------------------------------------------------ */
+void orc_kmeans_assign(const float *X, int64_t n, int d, const float *C, int nl, int32_t *assign, double *dist) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const float *x = X + i * (int64_t)d;
+        int best = 0;
+        double bd = 0.0;
+        for (int c = 0; c < nl; ++c) {
+            const float *cr = C + (int64_t)c * d;
+            double acc = 0.0;
+            for (int t = 0; t < d; ++t) {
+                const double df = (double)x[t] - (double)cr[t];
+                acc = acc + df * df;
+            }
+            if (c == 0 || acc < bd) {
+                bd = acc;
+                best = c;
+            }
+        }
+        assign[i] = best;
+        if (dist) dist[i] = bd;
+    }
+}
+
+void orc_kmeans_update(const float *X, int64_t n, int d, const int32_t *assign, int nl, const float *C_old,
+                       float *C_new, int64_t *counts) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int c = 0; c < nl; ++c) {
+        double *s = (double *)calloc((size_t)d, sizeof(double));
+        int64_t m = 0;
+        for (int64_t i = 0; i < n; ++i) {
+            if (assign[i] != c) continue;
+            const float *x = X + i * (int64_t)d;
+            for (int t = 0; t < d; ++t) s[t] = s[t] + (double)x[t];
+            ++m;
+        }
+        for (int t = 0; t < d; ++t)
+            C_new[(int64_t)c * d + t] = m ? (float)(s[t] / (double)m) : C_old[(int64_t)c * d + t];
+        if (counts) counts[c] = m;
+        free(s);
+    }
+}
