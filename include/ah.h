@@ -196,7 +196,7 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
  *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves, to
  *                            bound its R-th best approximate score before the
  *                            scan (default 1024; the bound uses
- *                            max(value, 8 R) points, at most 4096)
+ *                            max(value, 4 R) points, at most 4096)
  *   AH_OPT_THRESHOLD_LEAVES  how many of the best leaves that sample is spread
  *                            over, evenly; the rest of the sample follows
  *                            rank order (default 1: a prefix in rank order)
@@ -340,6 +340,33 @@ AH_API ah_status ah_load(const char *dir, void *cuda_stream, ah_index **out);
  */
 AH_API ah_status ah_encode(const float *X, int64_t n, int32_t d, int32_t dims_per_block, const float *codebook,
                            double T, int32_t passes, uint8_t *codes, int32_t *passes_used, void *cuda_stream);
+
+/*
+ * Partition training, the other index-build step (ScaNN blog, "Using the
+ * library": the tree's leaves are k-means centroids trained on a sample, and
+ * every point goes to its nearest leaf).  One Lloyd iteration is
+ * ah_kmeans_assign followed by ah_kmeans_update.
+ *
+ * ah_kmeans_assign: assign[i] = argmin_c sum_t (X[i][t] - C[c][t])^2 over
+ * c < nl, fp64 with every difference, square and sum rounded separately,
+ * coordinates in ascending order, ties to the lower c; dist[i] (may be NULL)
+ * = that minimum.  X [n][d], C [nl][d] float; assign [n] int32, dist [n]
+ * double; all device memory.
+ *
+ * ah_kmeans_update: for every centroid c, its members i (assign[i] == c) in
+ * ascending order are summed per coordinate in fp64 and C_new[c] = sum / m
+ * (fp64 division, rounded to float); a centroid without members keeps
+ * C_old[c]; counts[c] (may be NULL) = m.  Entries of assign outside [0, nl)
+ * belong to no centroid.  C_new must not overlap C_old.
+ *
+ * Both asynchronous on cuda_stream; nothing is allocated.  Errors:
+ * AH_ERR_INVALID_ARG (NULL array, n < 0, d < 1, nl < 1), AH_ERR_UNSUPPORTED
+ * (d above AH_MAX_D; for the update, d above 3200), AH_ERR_CUDA.
+ */
+AH_API ah_status ah_kmeans_assign(const float *X, int64_t n, int32_t d, const float *C, int32_t nl, int32_t *assign,
+                                  double *dist, void *cuda_stream);
+AH_API ah_status ah_kmeans_update(const float *X, int64_t n, int32_t d, const int32_t *assign, int32_t nl,
+                                  const float *C_old, float *C_new, int64_t *counts, void *cuda_stream);
 
 AH_API void ah_destroy(ah_index *ix);
 

@@ -17,6 +17,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstddef>
 
 #include "kernels.h"
 
@@ -37,6 +38,10 @@ __device__ __forceinline__ void half_argmin(double& l, int& j, unsigned mask) {
     }
 }
 
+// USE_U: the point's unit vector u = x / ||x|| is computed once (each element
+// by one lane, the same correctly rounded division) into shared memory;
+// otherwise every use recomputes it, with identical values.
+template <bool USE_U>
 __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X, int64_t n, int d, int dpb,
                                                      const float* __restrict__ codebook, double T, int passes,
                                                      int cb_in_smem, uint8_t* __restrict__ codes,
@@ -46,6 +51,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X
     float* scb = reinterpret_cast<float*>(smem);
     const int cb_elems = B * 16 * dpb;
     uint8_t* scode = smem + (cb_in_smem ? static_cast<size_t>(cb_elems) * sizeof(float) : 0);
+    double* su_all = reinterpret_cast<double*>(
+        (reinterpret_cast<uintptr_t>(scode + static_cast<size_t>(16) * B) + 15) & ~static_cast<uintptr_t>(15));
     if (cb_in_smem) {
         for (int e = threadIdx.x; e < cb_elems; e += blockDim.x) scb[e] = codebook[e];
         __syncthreads();
@@ -70,6 +77,15 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X
             if (tt < 1.0) eta = __ddiv_rn(__dmul_rn(static_cast<double>(d - 1), tt), __dadd_rn(1.0, -tt));
         }
         const double e1 = __dadd_rn(eta, -1.0);
+        double* su = su_all + static_cast<size_t>(half) * d;
+        if (USE_U) {
+            for (int t = j; t < d; t += 16) {
+                const double x = static_cast<double>(xr[t]);
+                su[t] = norm > 0.0 ? __ddiv_rn(x, norm) : 0.0;
+            }
+            __syncwarp(mask);
+        }
+        auto unit = [&](int t, double x) { return USE_U ? su[t] : (norm > 0.0 ? __ddiv_rn(x, norm) : 0.0); };
         // start: per block the nearest center
         for (int b = 0; b < B; ++b) {
             double e = 0.0;
@@ -88,7 +104,7 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X
             const int c = code[b];
             for (int s = 0; s < dpb; ++s) {
                 const double x = static_cast<double>(xr[b * dpb + s]);
-                const double u = norm > 0.0 ? __ddiv_rn(x, norm) : 0.0;
+                const double u = unit(b * dpb + s, x);
                 const double r = __dadd_rn(x, -static_cast<double>(cb[(b * 16 + c) * dpb + s]));
                 rpar = __dadd_rn(rpar, __dmul_rn(r, u));
                 rn2 = __dadd_rn(rn2, __dmul_rn(r, r));
@@ -99,17 +115,16 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X
             int changed = 0;
             for (int b = 0; b < B; ++b) {
                 const int cur = code[b];
-                double sp = 0.0, sn = 0.0, cp = 0.0, cn = 0.0;
+                double sp = 0.0, sn = 0.0;
                 for (int s = 0; s < dpb; ++s) {
                     const double x = static_cast<double>(xr[b * dpb + s]);
-                    const double u = norm > 0.0 ? __ddiv_rn(x, norm) : 0.0;
-                    const double rc = __dadd_rn(x, -static_cast<double>(cb[(b * 16 + cur) * dpb + s]));
-                    cp = __dadd_rn(cp, __dmul_rn(rc, u));
-                    cn = __dadd_rn(cn, __dmul_rn(rc, rc));
+                    const double u = unit(b * dpb + s, x);
                     const double r = __dadd_rn(x, -static_cast<double>(cb[(b * 16 + j) * dpb + s]));
                     sp = __dadd_rn(sp, __dmul_rn(r, u));
                     sn = __dadd_rn(sn, __dmul_rn(r, r));
                 }
+                // the current center's sums are lane cur's own (same operations)
+                const double cp = __shfl_sync(mask, sp, cur, 16), cn = __shfl_sync(mask, sn, cur, 16);
                 const double wp = __dadd_rn(rpar, -cp), wn = __dadd_rn(rn2, -cn);
                 const double pj = __dadd_rn(wp, sp), nj = __dadd_rn(wn, sn);
                 const double l = __dadd_rn(__dmul_rn(e1, __dmul_rn(pj, pj)), nj);
@@ -137,30 +152,35 @@ __global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X
 
 }  // namespace
 
-size_t encode_smem_bytes(int d, int dpb, bool* cb_in_smem) {
+// Dynamic shared memory: the codebook (when it fits), 16 half-warps' codes
+// and, when it fits, 16 half-warps' unit vectors.
+size_t encode_smem_bytes(int d, int dpb, bool* cb_in_smem, bool* use_u) {
     const size_t B = static_cast<size_t>(d / dpb);
     const size_t cb = B * 16 * dpb * sizeof(float);
     const size_t codes = 16 * B;
-    *cb_in_smem = cb + codes <= 160 * 1024;
-    return (*cb_in_smem ? cb : 0) + codes;
+    const size_t u = 16 * static_cast<size_t>(d) * sizeof(double) + 16;
+    *cb_in_smem = cb + codes <= 100 * 1024;
+    const size_t base = (*cb_in_smem ? cb : 0) + codes;
+    *use_u = base + u <= 200 * 1024;
+    return base + (*use_u ? u : 0);
 }
 
 cudaError_t launch_encode(const float* X, int64_t n, int d, int dpb, const float* codebook, double T, int passes,
                           uint8_t* codes, int32_t* passes_used, int num_sms, cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
-    bool in_smem = false;
-    const size_t smem = encode_smem_bytes(d, dpb, &in_smem);
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    bool in_smem = false, use_u = false;
+    const size_t smem = encode_smem_bytes(d, dpb, &in_smem, &use_u);
+    auto kern = use_u ? encode_kernel<true> : encode_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel, 256, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t need = (n + 15) / 16;
     const int64_t grid = std::min<int64_t>(need, static_cast<int64_t>(num_sms) * per_sm);
-    encode_kernel<<<static_cast<unsigned>(grid), 256, smem, s>>>(X, n, d, dpb, codebook, T, passes, in_smem ? 1 : 0,
-                                                                 codes, passes_used);
+    kern<<<static_cast<unsigned>(grid), 256, smem, s>>>(X, n, d, dpb, codebook, T, passes, in_smem ? 1 : 0, codes,
+                                                        passes_used);
     return cudaGetLastError();
 }
 

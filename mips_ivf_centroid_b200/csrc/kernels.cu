@@ -1634,10 +1634,11 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
     }
     if (staged == -2) {
         K = scr.count;
-    } else if (staged >= 0 && staged <= 4 * kFinishThreads) {
+    } else if (staged >= 0 && staged <= kStageCap) {
         auto get = [&](int i) { return skeys[i]; };
         auto pay = [&](int i) { return sslots[i]; };
-        K = block_topk_reg<4, kFinishThreads>(get, pay, staged, R, rs, &scr.count, okeys, oslots, sorted);
+        K = block_topk_reg<kStageCap / kFinishThreads, kFinishThreads>(get, pay, staged, R, rs, &scr.count, okeys,
+                                                                       oslots, sorted);
     } else if (staged >= 0) {
         auto get = [&](int i) { return skeys[i]; };
         auto pay = [&](int i) { return sslots[i]; };

@@ -13,7 +13,7 @@ constexpr int kGroupF32 = 8;
 constexpr int kGroupU8 = 16;
 constexpr int kScanThreads = 256;
 #ifndef AH_SAMPLE_MULT
-#define AH_SAMPLE_MULT 8
+#define AH_SAMPLE_MULT 4
 #endif
 constexpr int kSampleMult = AH_SAMPLE_MULT;       // the threshold sample holds at least this many times R slots
 constexpr int kMaxThresholdSample = 4096;   // slots scored per query for the threshold
@@ -117,8 +117,15 @@ int scan_group(const DeviceIndex& ix, int lut_mode);
 size_t finish_smem_bytes(int R, int d);
 
 // anisotropic code assignment (encode.cu)
-size_t encode_smem_bytes(int d, int dpb, bool* cb_in_smem);
+size_t encode_smem_bytes(int d, int dpb, bool* cb_in_smem, bool* use_u);
 cudaError_t launch_encode(const float* X, int64_t n, int d, int dpb, const float* codebook, double T, int passes,
                           uint8_t* codes, int32_t* passes_used, int num_sms, cudaStream_t s);
+
+// partition training (kmeans.cu)
+cudaError_t launch_kmeans_assign(const float* X, int64_t n, int d, const float* C, int nl, int32_t* assign,
+                                 double* dist, cudaStream_t s);
+size_t kmeans_update_smem_bytes(int d);
+cudaError_t launch_kmeans_update(const float* X, int64_t n, int d, const int32_t* assign, int nl, const float* C_old,
+                                 float* C_new, int64_t* counts, cudaStream_t s);
 
 }  // namespace ah

@@ -34,6 +34,7 @@ def _case(n, d, dpb, seed, unit=True, scale=0.3):
     (2000, 64, 2, 0.0, 10, True),       # T = 0: L2 codes
     (1000, 32, 2, 0.5, 0, True),        # no descent
     (1000, 48, 2, 0.2, 100, True),      # to convergence
+    (400, 1536, 4, 0.05, 10, True),     # OpenAI-shaped: codebook and unit vectors outside shared memory
 ])
 def test_codes_match_oracle(enc, n, d, dpb, T, passes, unit):
     X, cb = _case(n, d, dpb, seed=n + d + dpb, unit=unit)
