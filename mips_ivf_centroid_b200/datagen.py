@@ -72,6 +72,7 @@ class Workload:
     training_sample_size: int = 250_000
     lloyd_iters: int = 10
     aniso_passes: int = 10
+    residual: bool = False                # codes of x - (its leaf's centroid) instead of x
 
     @property
     def blocks(self) -> int:
@@ -234,6 +235,7 @@ class IndexArrays:
     codes: torch.Tensor
     codebook: torch.Tensor
     reorder_vecs: torch.Tensor
+    residual: bool = False
 
     def to(self, device) -> "IndexArrays":
         f = {k: (v.to(device) if isinstance(v, torch.Tensor) else v)
@@ -252,6 +254,7 @@ class IndexArrays:
         else:
             out["reorder_vecs"] = rv.numpy()
             out["reorder_dtype"] = "f32"
+        out["residual"] = bool(self.residual)
         return out
 
 
@@ -419,16 +422,20 @@ def build_index(w: Workload, X: np.ndarray, device="cpu") -> IndexArrays:
     offs[1:] = torch.cumsum(counts, 0)
     Xs = Xt[order]
     del Xt
-    cb = _train_codebook(w, Xs)
-    codes = _l2_codes(Xs, cb)
+    # residual codes quantise x minus its leaf's centroid (one codebook for all
+    # leaves); the approximate score then adds q . centroid to the table sum
+    Ys = Xs - cent[assign[order]] if w.residual else Xs
+    cb = _train_codebook(w, Ys)
+    codes = _l2_codes(Ys, cb)
     if w.code_loss == "anisotropic":
-        codes = _anisotropic_codes(Xs, cb, codes, w.eta, w.aniso_passes)
+        codes = _anisotropic_codes(Ys, cb, codes, w.eta, w.aniso_passes)
+    del Ys
     packed = pack_codes(codes)
     del codes
     rv = Xs.to(torch.bfloat16) if w.reorder_dtype == "bf16" else Xs
     return IndexArrays(workload=w, centroids=cent.contiguous(), leaf_offsets=offs,
                        slot_ids=order.to(torch.int32), codes=packed, codebook=cb.contiguous(),
-                       reorder_vecs=rv.contiguous())
+                       reorder_vecs=rv.contiguous(), residual=w.residual)
 
 
 def make_workload(w: Workload, device="cpu", nq: Optional[int] = None):

@@ -62,6 +62,7 @@ class _Index(ctypes.Structure):
         ("codebook", ctypes.c_void_p),
         ("reorder_vecs", ctypes.c_void_p),
         ("reorder_is_bf16", ctypes.c_int32),
+        ("residual", ctypes.c_int32),
     ]
 
 
@@ -96,8 +97,9 @@ class OracleIndex:
 
     ``arrays``: dict with centroids [NL,d] f32, leaf_offsets [NL+1] i64,
     slot_ids [n] i32, codes [n,B/2] u8, codebook [B,16,dpb] f32,
-    reorder_vecs [n,d] (f32, or bf16 bits as u16; None if never reordered)
-    and reorder_dtype.
+    reorder_vecs [n,d] (f32, or bf16 bits as u16; None if never reordered),
+    reorder_dtype and residual (codes of x minus its leaf's centroid; the
+    approximate score then adds q . centroid to the table sum).
     """
 
     def __init__(self, arrays: dict):
@@ -118,7 +120,7 @@ class OracleIndex:
         self.n, self.d, self.num_leaves, self.dpb, self.blocks = a["slot_ids"].shape[0], d, nl, dpb, B
         self._s = _Index(self.n, d, nl, dpb, _ptr(a["centroids"]), _ptr(a["leaf_offsets"]),
                          _ptr(a["slot_ids"]), _ptr(a["codes"]), _ptr(a["codebook"]),
-                         _ptr(a["reorder_vecs"]), 1 if bf16 else 0)
+                         _ptr(a["reorder_vecs"]), 1 if bf16 else 0, 1 if arrays.get("residual") else 0)
 
     @property
     def ref(self):

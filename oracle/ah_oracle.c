@@ -47,6 +47,7 @@ typedef struct {
     const float *codebook;        /* [B][16][dims_per_block] */
     const void *reorder_vecs;     /* [n][d], float32 or bfloat16 bits */
     int32_t reorder_is_bf16;
+    int32_t residual;             /* codes quantise x - centroid of its leaf */
 } orc_index;
 
 typedef struct {
@@ -206,7 +207,7 @@ int orc_search(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32
                int32_t *out_ncand, int64_t *out_scanned) {
     if (!ix || !Q || !out_ids || !out_scores || nq < 0 || k <= 0 || L < 1 ||
         L > ix->num_leaves || reorder_num < 0 || (reorder_num > 0 && reorder_num < k) ||
-        (lut_mode != 0 && lut_mode != 1))
+        (lut_mode != 0 && lut_mode != 1) || (lut_mode == 1 && ix->residual))
         return -1;
     const int B = blocks_of(ix);
     const int32_t R = reorder_num > k ? reorder_num : k;
@@ -259,7 +260,8 @@ int orc_search(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32
             int c = leaves[i].slot;
             for (int64_t p = ix->leaf_offsets[c]; p < ix->leaf_offsets[c + 1]; ++p, ++m) {
                 if (lut_mode == 0) {
-                    cand[m].score = ah_score_f64(ix, lut, p);
+                    /* residual codes: q . x~ = q . centroid + table sum */
+                    cand[m].score = ix->residual ? ah_score_f64(ix, lut, p) + s[c] : ah_score_f64(ix, lut, p);
                     cand[m].id = ix->slot_ids[p];
                     cand[m].slot = (int32_t)p;
                 } else {
@@ -335,10 +337,24 @@ void orc_point_scores(const orc_index *ix, const float *q, int64_t nslots, const
     int B = blocks_of(ix);
     double *lut = (double *)malloc(sizeof(double) * (size_t)B * ORC_CENTERS);
     lut_f64(ix, q, lut);
+    double *s = ix->residual ? (double *)malloc(sizeof(double) * ix->num_leaves) : NULL;
+    if (s) centroid_scores(ix, q, s);
     for (int64_t i = 0; i < nslots; ++i) {
-        if (out_ah) out_ah[i] = ah_score_f64(ix, lut, slots[i]);
+        if (out_ah) {
+            out_ah[i] = ah_score_f64(ix, lut, slots[i]);
+            if (s) {
+                /* the slot's leaf: the last c with leaf_offsets[c] <= slot */
+                int lo = 0, hi = ix->num_leaves - 1;
+                while (lo < hi) {
+                    int mid = (lo + hi + 1) / 2;
+                    if (ix->leaf_offsets[mid] <= slots[i]) lo = mid; else hi = mid - 1;
+                }
+                out_ah[i] = out_ah[i] + s[lo];
+            }
+        }
         if (out_exact) out_exact[i] = exact_score(ix, q, slots[i]);
     }
+    free(s);
     free(lut);
 }
 

@@ -89,6 +89,45 @@ def test_approximate_score_is_dot_with_reconstruction():
         assert out["scanned"][qi] == scanned.shape[0]
 
 
+def test_residual_score_is_dot_with_centroid_plus_reconstruction():
+    # residual codes quantise x - c(leaf): the approximate point is c(leaf) + r~,
+    # so the score is q . c(leaf) + the table sum over the residual codebook
+    w, X, Q, ix, arr = _mini(aniso=True, residual=True)
+    assert arr["residual"]
+    orc = OracleIndex(arr)
+    out = orc.search(Q, w.k, w.num_leaves_to_search, w.reorder_num)
+    rt = _reconstruct(arr)
+    leaf_of = np.repeat(np.arange(w.num_leaves), np.diff(arr["leaf_offsets"]))
+    xt = rt + arr["centroids"].astype(np.float64)[leaf_of]
+    inv = np.empty(w.n, np.int64)
+    inv[arr["slot_ids"]] = np.arange(w.n)
+    for qi in range(Q.shape[0]):
+        nc = out["ncand"][qi]
+        slots = inv[out["cand_ids"][qi][:nc]]
+        expect = xt[slots] @ Q[qi].astype(np.float64)
+        np.testing.assert_allclose(out["cand_scores"][qi][:nc], expect, rtol=0, atol=1e-12)
+        lv = out["leaves"][qi]
+        scanned = np.concatenate([np.arange(arr["leaf_offsets"][c], arr["leaf_offsets"][c + 1])
+                                  for c in lv])
+        sc = xt[scanned] @ Q[qi].astype(np.float64)
+        best = scanned[_order(sc, arr["slot_ids"][scanned])][:nc]
+        np.testing.assert_array_equal(arr["slot_ids"][best], out["cand_ids"][qi][:nc])
+        a, _ = orc.point_scores(Q[qi], slots)
+        np.testing.assert_allclose(a, expect, rtol=0, atol=1e-12)
+    # the residual reconstruction is closer to the data than the plain one
+    wp, Xp, _, _, arrp = _mini(aniso=True)
+    err_res = np.linalg.norm(X[arr["slot_ids"]] - xt, axis=1).mean()
+    err_plain = np.linalg.norm(Xp[arrp["slot_ids"]] - _reconstruct(arrp), axis=1).mean()
+    assert err_res < err_plain
+
+
+def test_residual_codes_reject_uint8_tables():
+    w, X, Q, ix, arr = _mini(residual=True)
+    orc = OracleIndex(arr)
+    with pytest.raises(Exception):
+        orc.search(Q, w.k, w.num_leaves_to_search, w.reorder_num, lut_mode=1)
+
+
 def test_hand_worked_nibble_example():
     # One point, d = 4, dims_per_block = 1 (B = 4 blocks); codes bytes 0x21, 0x43
     # mean block 0 -> center 1, block 1 -> 2, block 2 -> 3, block 3 -> 4
