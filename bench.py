@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--encode", action="store_true",
                    help="index build: time the anisotropic code assignment over the workload's points")
     p.add_argument("--passes", type=int, default=10)
+    p.add_argument("--kmeans", action="store_true",
+                   help="index build: time one k-means iteration (assignment + update) over the workload's points")
     return p.parse_args()
 
 
@@ -523,10 +525,68 @@ def run_encode(args):
     print(json.dumps(line), flush=True)
 
 
+def run_kmeans(args):
+    """One JSON line: one Lloyd iteration (ah_kmeans_assign + ah_kmeans_update)
+    of the workload's n points against its num_leaves centroids, points/s on
+    the device, with the oracle timed on a sample of points."""
+    import torch
+    from mips_ivf_centroid_b200 import build as ahbuild, datagen
+    ahbuild.build()
+    from mips_ivf_centroid_b200 import kmeans_assign, kmeans_update
+    import oracle
+    w = workload_spec(args)
+    X = datagen.make_data(w)
+    rng = np.random.default_rng(1)
+    C = X[rng.choice(w.n, size=w.num_leaves, replace=False)].copy()
+    Xg, Cg = torch.from_numpy(X).cuda(), torch.from_numpy(C).cuda()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        a, _ = kmeans_assign(Xg, Cg)
+        kmeans_update(Xg, a, Cg)
+    torch.cuda.synchronize()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    ta = tu = 0.0
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            e0.record(stream)
+            a, _ = kmeans_assign(Xg, Cg)
+            e1.record(stream)
+            Cn, cnt = kmeans_update(Xg, a, Cg)
+            e2.record(stream)
+            torch.cuda.synchronize()
+            ta += e0.elapsed_time(e1)
+            tu += e1.elapsed_time(e2)
+    ta, tu = ta / args.steps, tu / args.steps
+    ops = 3.0 * w.n * w.num_leaves * w.d           # difference, square, sum per (point, centroid, coordinate)
+    mhz = SM_MAX_MHZ_FALLBACK
+    peak = SM_COUNT * 64 * mhz * 1e6
+    ns = min(w.n, 2000)
+    t0 = time.perf_counter()
+    ao, _ = oracle.kmeans_assign(X[:ns], C)
+    ot = time.perf_counter() - t0
+    same = bool(np.array_equal(ao, a[:ns].cpu().numpy()))
+    line = {"metric": "k-means iteration points/s (1 B200)", "value": w.n / ((ta + tu) * 1e-3), "unit": "points/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ta + tu,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Gaussian mixture)",
+            "config": {"workload": f"{w.name}-shaped: n={w.n:,} d={w.d} centroids={w.num_leaves}"},
+            "assign_ms": ta, "update_ms": tu,
+            "roofline": {"bound": "alu", "kernel": "kmeans_assign", "achieved": ops / (ta * 1e-3) / 1e12,
+                         "peak": peak / 1e12, "unit": "Tops/s (fp64)", "frac": ops / (ta * 1e-3) / peak,
+                         "traffic": None,
+                         "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 lanes x {mhz:.0f} MHz (nominal rate)"},
+            "cpu_baseline": {"value": ns / ot, "unit": "points/s (assignment)", "cores": oracle.max_threads(),
+                             "kind": "oracle", "sample": f"first {ns} points"},
+            "oracle_match_on_sample": same, "clocks": clk.summary(), "gpu_launches": 2 * (args.steps + args.warmup)}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.kmeans:
+        run_kmeans(args)
     elif args.encode:
         run_encode(args)
     elif args.sweep:

@@ -86,6 +86,12 @@ enum { AH_LUT_F32 = 0, AH_LUT_U8 = 1 };
  *   reorder_vecs    [n][d] slot order, float (AH_F32) or bfloat16 (AH_BF16);
  *                   may be NULL if the index is only searched with
  *                   reorder_num = 0
+ *   residual        0: codes quantise each point; 1: codes quantise the
+ *                   point minus its leaf's centroid (one codebook for all
+ *                   leaves), so a point's approximate score is the query's
+ *                   centroid score of that leaf plus its table sum (added
+ *                   after the sum, in fp32).  Residual indexes support fp32
+ *                   tables only (AH_LUT_U8 is AH_ERR_UNSUPPORTED).
  */
 typedef struct {
     int64_t n;
@@ -99,6 +105,7 @@ typedef struct {
     const float *codebook;
     const void *reorder_vecs;
     int32_t reorder_dtype;
+    int32_t residual;
 } ah_index_views;
 
 typedef struct ah_index ah_index;
@@ -289,7 +296,8 @@ AH_API ah_status ah_search_leaves_noalloc(ah_index *ix, const float *queries, in
  *   reorder_vecs.npy  <f4 [n, d], or <u2 [n, d] holding bfloat16 bit
  *                     patterns (absent when the index has no reorder copy)
  *   ah_index.txt      first line "ah-index 1", then "reorder_dtype f32",
- *                     "reorder_dtype bf16" or "reorder_dtype none"
+ *                     "reorder_dtype bf16" or "reorder_dtype none", then
+ *                     "residual 0" or "residual 1" (absent: 0)
  * Synchronous (device-to-host copies).  Errors: AH_ERR_INVALID_ARG (NULL
  * argument, a file that cannot be written: the message names it),
  * AH_ERR_CUDA.
@@ -361,7 +369,7 @@ AH_API ah_status ah_encode(const float *X, int64_t n, int32_t d, int32_t dims_pe
  *
  * Both asynchronous on cuda_stream; nothing is allocated.  Errors:
  * AH_ERR_INVALID_ARG (NULL array, n < 0, d < 1, nl < 1), AH_ERR_UNSUPPORTED
- * (d above AH_MAX_D; for the update, d above 3200), AH_ERR_CUDA.
+ * (d above AH_MAX_D; for the update, d above 6400), AH_ERR_CUDA.
  */
 AH_API ah_status ah_kmeans_assign(const float *X, int64_t n, int32_t d, const float *C, int32_t nl, int32_t *assign,
                                   double *dist, void *cuda_stream);

@@ -189,6 +189,8 @@ ah_status validate_search(ah_index* ix, const void* queries, int32_t nq, int32_t
     if (reorder_num > 0 && !ix->views.reorder_vecs)
         return fail(AH_ERR_INVALID_ARG, "reorder_num > 0 but the index has no reorder vectors");
     if (lut_mode != AH_LUT_F32 && lut_mode != AH_LUT_U8) return fail(AH_ERR_INVALID_ARG, "unknown lut_mode");
+    if (lut_mode == AH_LUT_U8 && ix->views.residual)
+        return fail(AH_ERR_UNSUPPORTED, "uint8 tables need codes of the points, not residuals");
     const int64_t per_query_cand = static_cast<int64_t>(cap_for(std::max(reorder_num, k)));
     if (static_cast<int64_t>(nq) * per_query_cand > (int64_t(1) << 40)) return fail(AH_ERR_UNSUPPORTED, "batch too large");
     return AH_OK;
@@ -354,6 +356,10 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     ah_index* ix = new (std::nothrow) ah_index();
     if (!ix) return fail(AH_ERR_OOM, "host allocation");
+    if (v->residual != 0 && v->residual != 1) {
+        delete ix;
+        return fail(AH_ERR_INVALID_ARG, "residual must be 0 or 1");
+    }
     ix->views = *v;
     cudaError_t e = cudaGetDevice(&ix->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ix->num_sms, cudaDevAttrMultiProcessorCount, ix->device);
@@ -424,6 +430,7 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
     d.codebook = v->codebook;
     d.reorder_vecs = v->reorder_vecs;
     d.reorder_bf16 = v->reorder_dtype == AH_BF16 ? 1 : 0;
+    d.residual = v->residual;
     *out = ix;
     return AH_OK;
 }
@@ -736,7 +743,7 @@ ah_status ah_save(ah_index* ix, const char* dir) {
     FILE* f = std::fopen(meta.c_str(), "w");
     if (!f) return fail(AH_ERR_INVALID_ARG, ("cannot write " + meta).c_str());
     const char* dt = !v.reorder_vecs ? "none" : (v.reorder_dtype == AH_BF16 ? "bf16" : "f32");
-    const bool ok = std::fprintf(f, "ah-index 1\nreorder_dtype %s\n", dt) > 0;
+    const bool ok = std::fprintf(f, "ah-index 1\nreorder_dtype %s\nresidual %d\n", dt, v.residual ? 1 : 0) > 0;
     if (std::fclose(f) != 0 || !ok) return fail(AH_ERR_INVALID_ARG, ("short write to " + meta).c_str());
     return AH_OK;
 }
@@ -748,9 +755,14 @@ ah_status inspect_dir(const char* dir, ah_index_views* out, ah::npy::Header hdr[
     const std::string meta = path_in(dir, kMetaFile);
     FILE* f = std::fopen(meta.c_str(), "r");
     if (!f) return fail(AH_ERR_INVALID_ARG, ("cannot open " + meta).c_str());
-    char l1[64] = {0}, key[64] = {0}, val[64] = {0};
+    char l1[64] = {0}, key[64] = {0}, val[64] = {0}, key2[64] = {0};
+    int resid = 0;
     const bool ok = std::fgets(l1, sizeof(l1), f) && std::fscanf(f, "%63s %63s", key, val) == 2;
+    const int got2 = ok ? std::fscanf(f, "%63s %d", key2, &resid) : 0;
     std::fclose(f);
+    if (got2 == 2 && (std::strcmp(key2, "residual") != 0 || (resid != 0 && resid != 1)))
+        return fail(AH_ERR_INVALID_ARG, (meta + ": third line must be \"residual 0\" or \"residual 1\"").c_str());
+    if (got2 != 2) resid = 0;
     if (!ok || std::strncmp(l1, "ah-index 1", 10) != 0 || std::strcmp(key, "reorder_dtype") != 0)
         return fail(AH_ERR_INVALID_ARG, (meta + ": expected \"ah-index 1\" then \"reorder_dtype <f32|bf16|none>\"").c_str());
     int rdt;
@@ -790,6 +802,7 @@ ah_status inspect_dir(const char* dir, ah_index_views* out, ah::npy::Header hdr[
     out->num_leaves = static_cast<int32_t>(NL);
     out->dims_per_block = static_cast<int32_t>(cb[2]);
     out->reorder_dtype = rdt;
+    out->residual = resid;
     return AH_OK;
 }
 
@@ -884,4 +897,28 @@ ah_status ah_encode(const float* X, int64_t n, int32_t d, int32_t dims_per_block
         e = ah::launch_encode(X, n, d, dims_per_block, codebook, T, passes, codes, passes_used, sms,
                               static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? AH_OK : cuda_fail(e, "encode");
+}
+
+// ---------------------------------------------------------------------------
+// partition training
+// ---------------------------------------------------------------------------
+
+ah_status ah_kmeans_assign(const float* X, int64_t n, int32_t d, const float* C, int32_t nl, int32_t* assign,
+                           double* dist, void* cuda_stream) {
+    if (n < 0 || d < 1 || nl < 1) return fail(AH_ERR_INVALID_ARG, "n < 0, d < 1 or nl < 1");
+    if (n == 0) return AH_OK;
+    if (!X || !C || !assign) return fail(AH_ERR_INVALID_ARG, "NULL array");
+    if (d > AH_MAX_D) return fail(AH_ERR_UNSUPPORTED, "d above AH_MAX_D");
+    const cudaError_t e = ah::launch_kmeans_assign(X, n, d, C, nl, assign, dist, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? AH_OK : cuda_fail(e, "k-means assignment");
+}
+
+ah_status ah_kmeans_update(const float* X, int64_t n, int32_t d, const int32_t* assign, int32_t nl, const float* C_old,
+                           float* C_new, int64_t* counts, void* cuda_stream) {
+    if (n < 0 || d < 1 || nl < 1) return fail(AH_ERR_INVALID_ARG, "n < 0, d < 1 or nl < 1");
+    if ((n > 0 && (!X || !assign)) || !C_old || !C_new) return fail(AH_ERR_INVALID_ARG, "NULL array");
+    if (ah::kmeans_update_smem_bytes(d) > 200 * 1024) return fail(AH_ERR_UNSUPPORTED, "d above 6400 for the update");
+    const cudaError_t e = ah::launch_kmeans_update(X, n, d, assign, nl, C_old, C_new, counts,
+                                                   static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? AH_OK : cuda_fail(e, "k-means update");
 }

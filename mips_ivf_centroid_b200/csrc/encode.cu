@@ -25,28 +25,27 @@ namespace ah {
 
 namespace {
 
-// (loss, center) minimum over the half-warp, ties to the lower center
+// (loss, center) minimum over the half-warp, ties to the lower center: the
+// minimum value by a shuffle reduction, then the lowest lane holding it.
 __device__ __forceinline__ void half_argmin(double& l, int& j, unsigned mask) {
+    double m = l;
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) {
-        const double lo = __shfl_xor_sync(mask, l, off, 16);
-        const int jo = __shfl_xor_sync(mask, j, off, 16);
-        if (lo < l || (lo == l && jo < j)) {
-            l = lo;
-            j = jo;
-        }
-    }
+    for (int off = 8; off > 0; off >>= 1) m = fmin(m, __shfl_xor_sync(mask, m, off, 16));
+    const unsigned hit = __ballot_sync(mask, l == m) & mask;
+    j = (__ffs(hit) - 1) & 15;
+    l = m;
 }
 
 // USE_U: the point's unit vector u = x / ||x|| is computed once (each element
 // by one lane, the same correctly rounded division) into shared memory;
 // otherwise every use recomputes it, with identical values.
-template <bool USE_U>
-__global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X, int64_t n, int d, int dpb,
+template <bool USE_U, int DPB>
+__global__ void __launch_bounds__(256) encode_kernel(const float* __restrict__ X, int64_t n, int d, int dpb_rt,
                                                      const float* __restrict__ codebook, double T, int passes,
                                                      int cb_in_smem, uint8_t* __restrict__ codes,
                                                      int32_t* __restrict__ passes_used) {
     extern __shared__ __align__(16) unsigned char smem[];
+    const int dpb = DPB > 0 ? DPB : dpb_rt;      // compile-time for the common block widths
     const int B = d / dpb;
     float* scb = reinterpret_cast<float*>(smem);
     const int cb_elems = B * 16 * dpb;
@@ -170,7 +169,14 @@ cudaError_t launch_encode(const float* X, int64_t n, int d, int dpb, const float
     if (n <= 0) return cudaSuccess;
     bool in_smem = false, use_u = false;
     const size_t smem = encode_smem_bytes(d, dpb, &in_smem, &use_u);
-    auto kern = use_u ? encode_kernel<true> : encode_kernel<false>;
+    void (*kern)(const float*, int64_t, int, int, const float*, double, int, int, uint8_t*, int32_t*);
+    switch (dpb) {
+        case 1: kern = use_u ? encode_kernel<true, 1> : encode_kernel<false, 1>; break;
+        case 2: kern = use_u ? encode_kernel<true, 2> : encode_kernel<false, 2>; break;
+        case 4: kern = use_u ? encode_kernel<true, 4> : encode_kernel<false, 4>; break;
+        case 8: kern = use_u ? encode_kernel<true, 8> : encode_kernel<false, 8>; break;
+        default: kern = use_u ? encode_kernel<true, 0> : encode_kernel<false, 0>; break;
+    }
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     int per_sm = 0;

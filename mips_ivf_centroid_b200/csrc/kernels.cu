@@ -735,9 +735,10 @@ cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchB
 // fp32: table in shared memory as [B][16] floats; returns the score key.
 // uint8: table as [B][16] bytes; returns the integer sum.
 // `pos` is the slot's position in the leaf-padded code copy.
+// With residual codes the leaf's centroid score `off` is added after the sum.
 template <int MODE>
 __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int B,
-                                               const unsigned char* lut, int32_t pos) {
+                                               const unsigned char* lut, int32_t pos, bool add_off, float off) {
     const uint32_t* cw = codes_il + (static_cast<int64_t>(pos >> 5) * W) * 32 + (pos & 31);
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
@@ -747,7 +748,7 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
             int nb = min(8, B - 8 * w);
             for (int i = 0; i < nb; ++i) acc = __fadd_rn(acc, lf[(8 * w + i) * kCenters + ((c >> (4 * i)) & 15u)]);
         }
-        return float_key(acc);
+        return float_key(add_off ? __fadd_rn(acc, off) : acc);
     } else {
         uint32_t acc = 0;
         for (int w = 0; w < W; ++w) {
@@ -764,7 +765,7 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
 template <int MODE>
 __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int B,
                                              const unsigned char* lut, const int32_t* pos, const bool* valid,
-                                             uint32_t* out) {
+                                             const float* off, uint32_t* out) {
     const uint32_t* cw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -799,7 +800,7 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) out[u] = float_key(acc[u]);
+        for (int u = 0; u < 4; ++u) out[u] = float_key(off ? __fadd_rn(acc[u], off[u]) : acc[u]);
     } else {
         uint32_t acc[4] = {0u, 0u, 0u, 0u};
         for (int w = 0; w < W; ++w) {
@@ -857,6 +858,7 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kSelThreads> rs;
     __shared__ int seg_end[kThresholdSegs], seg_pos[kThresholdSegs], seg_slot[kThresholdSegs];
+    __shared__ float seg_off[kThresholdSegs];       // residual codes: the leaf's centroid score
     __shared__ int s_nseg, s_taken;
     const int q = blockIdx.x;
     const int R = a.R;
@@ -894,6 +896,7 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
                 seg_end[idx] = taken + incl;
                 seg_pos[idx] = ix.ptile[leaf] * 32 + start;
                 seg_slot[idx] = ix.offs[leaf] + start;
+                seg_off[idx] = ix.residual ? b.cscore[static_cast<int64_t>(q) * ix.nl + leaf] : 0.0f;
             }
             const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
             const int n = __popc(m);
@@ -947,6 +950,7 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
         int32_t ps[4], sid[4];
         bool ok[4];
         uint32_t v[4];
+        float off4[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = t0 + u * kSelThreads + threadIdx.x;
@@ -959,8 +963,9 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
             const int off = i - (lo > 0 ? seg_end[lo - 1] : 0);
             ps[u] = seg_pos[lo] + off;
             sid[u] = ok[u] ? ix.slot_ids[seg_slot[lo] + off] : 0;
+            off4[u] = seg_off[lo];
         }
-        slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, v);
+        slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, ix.residual ? off4 : nullptr, v);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = t0 + u * kSelThreads + threadIdx.x;
@@ -1107,7 +1112,7 @@ struct TileJob {
 template <int G, int NT>
 __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                                const TileJob& job, const int* s_q, const uint32_t* s_th,
-                                               const uint32_t* s_tl) {
+                                               const uint32_t* s_tl, const float* s_off) {
     constexpr int BS = (G / 2) * kCenters;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
@@ -1133,7 +1138,8 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize) {
-                const float sc = (qi & 1) ? acc[qi >> 1].y : acc[qi >> 1].x;
+                const float sum = (qi & 1) ? acc[qi >> 1].y : acc[qi >> 1].x;
+                const float sc = ix.residual ? __fadd_rn(sum, s_off[qi]) : sum;
                 const uint32_t key = float_key(sc);
                 append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot, s_q[qi], ix, b);
             }
@@ -1206,6 +1212,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 5
     __shared__ int s_item, s_leaf;
     __shared__ int s_q[GMAX];
     __shared__ uint32_t s_th[GMAX], s_tl[GMAX];
+    __shared__ float s_off[GMAX];            // residual codes: each query's score of this leaf
     const int B = ix.B;
     const int total_items = b.item_off[ix.nl];
     const size_t lut_bytes = static_cast<size_t>(B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
@@ -1251,6 +1258,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 5
             uint64_t t = (qq >= 0) ? b.tau[qq] : ~0ull;
             s_th[threadIdx.x] = static_cast<uint32_t>(t >> 32);
             s_tl[threadIdx.x] = static_cast<uint32_t>(t);
+            s_off[threadIdx.x] = (ix.residual && qq >= 0) ? b.cscore[static_cast<int64_t>(qq) * ix.nl + leaf] : 0.0f;
         }
         __syncthreads();
         // stage the group's tables
@@ -1294,10 +1302,10 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 5
         __syncthreads();
         if (MODE == 0) {
             switch (G) {
-                case 8: scan_tiles_f32<8, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 6: scan_tiles_f32<6, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 4: scan_tiles_f32<4, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                default: scan_tiles_f32<2, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
+                case 8: scan_tiles_f32<8, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                case 6: scan_tiles_f32<6, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                case 4: scan_tiles_f32<4, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                default: scan_tiles_f32<2, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
             }
         } else {
             switch (G) {
@@ -1477,10 +1485,12 @@ __global__ void __launch_bounds__(kSelThreads) redo_scan_kernel(DeviceIndex ix, 
         const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + i];
         const int s0 = ix.offs[leaf], s1 = ix.offs[leaf + 1];
         const int p0 = ix.ptile[leaf] * 32 - s0;            // padded position = slot + p0
+        const float off = ix.residual ? b.cscore[static_cast<int64_t>(q) * ix.nl + leaf] : 0.0f;
         for (int base = s0; base < s1; base += kSelThreads) {
             const int slot = base + threadIdx.x;
             const bool in = slot < s1;
-            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot + p0) : 0u;
+            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot + p0, ix.residual != 0, off)
+                                  : 0u;
             append_candidates(in && reaches(v, th, tl, ix.slot_ids, slot), v, slot, q, ix, b);
         }
     }

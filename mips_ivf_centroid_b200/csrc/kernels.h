@@ -38,6 +38,7 @@ struct DeviceIndex {
     const float* codebook;                // [B][16][dpb]
     const void* reorder_vecs;             // [n][d]
     int reorder_bf16;
+    int residual;                         // codes quantise x - its leaf's centroid: scores add q . centroid
 };
 
 struct SearchBuffers {

@@ -44,6 +44,7 @@ class Views(ctypes.Structure):
         ("codebook", ctypes.c_void_p),
         ("reorder_vecs", ctypes.c_void_p),
         ("reorder_dtype", ctypes.c_int32),
+        ("residual", ctypes.c_int32),
     ]
 
 
@@ -80,6 +81,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_last_error": (ctypes.c_char_p, []),
         "ah_search_leaves_noalloc": (I32, [P, P, I32, I32, P, P, P]),
         "ah_encode": (I32, [P, I64, I32, I32, P, ctypes.c_double, I32, P, P, P]),
+        "ah_kmeans_assign": (I32, [P, I64, I32, P, I32, P, P, P]),
+        "ah_kmeans_update": (I32, [P, I64, I32, P, I32, P, P, P, P]),
         "ah_save": (I32, [P, ctypes.c_char_p]),
         "ah_inspect": (I32, [ctypes.c_char_p, P]),
         "ah_load": (I32, [ctypes.c_char_p, P, ctypes.POINTER(P)]),
@@ -135,6 +138,47 @@ def encode(X: torch.Tensor, codebook: torch.Tensor, T: float, passes: int = 10, 
     return out, passes_used
 
 
+def _f32_2d(t: torch.Tensor, name: str, dev=None):
+    if t.dtype != torch.float32 or t.dim() != 2 or not t.is_contiguous() or t.device.type != "cuda" \
+            or (dev is not None and t.device != dev):
+        raise AhError(1, f"{name}: need contiguous float32 2-D CUDA tensor" + (f" on {dev}" if dev else ""))
+
+
+def kmeans_assign(X: torch.Tensor, C: torch.Tensor, stream=None):
+    """Nearest centroid of every row of X (``ah_kmeans_assign``): (assign [n]
+    int32, squared distance [n] float64), asynchronous on the stream."""
+    lib = load_library()
+    _f32_2d(X, "X")
+    _f32_2d(C, "C", X.device)
+    if C.shape[1] != X.shape[1]:
+        raise AhError(1, "C: need [nl, d] with X's d")
+    n, d = X.shape
+    a = torch.empty((n,), dtype=torch.int32, device=X.device)
+    dist = torch.empty((n,), dtype=torch.float64, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib, lib.ah_kmeans_assign(_ptr(X), n, d, _ptr(C), C.shape[0], _ptr(a), _ptr(dist), _stream(stream)))
+    return a, dist
+
+
+def kmeans_update(X: torch.Tensor, assign: torch.Tensor, C_old: torch.Tensor, stream=None):
+    """Centroid means over each centroid's members (``ah_kmeans_update``):
+    (C_new [nl, d] float32, counts [nl] int64), asynchronous on the stream."""
+    lib = load_library()
+    _f32_2d(X, "X")
+    _f32_2d(C_old, "C_old", X.device)
+    if assign.dtype != torch.int32 or assign.dim() != 1 or assign.shape[0] != X.shape[0] \
+            or assign.device != X.device or not assign.is_contiguous():
+        raise AhError(1, "assign: need contiguous int32 [n] on X's device")
+    n, d = X.shape
+    nl = C_old.shape[0]
+    C_new = torch.empty_like(C_old)
+    counts = torch.empty((nl,), dtype=torch.int64, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib, lib.ah_kmeans_update(_ptr(X), n, d, _ptr(assign), nl, _ptr(C_old), _ptr(C_new), _ptr(counts),
+                                         _stream(stream)))
+    return C_new, counts
+
+
 def inspect(path: str) -> dict:
     """Sizes of an index directory written by ``Index.save`` (no GPU needed):
     n, d, num_leaves, dims_per_block, reorder_dtype ("f32", "bf16" or None)."""
@@ -142,7 +186,8 @@ def inspect(path: str) -> dict:
     v = Views()
     _check(lib, lib.ah_inspect(os.fsencode(path), ctypes.byref(v)))
     rdt = {AH_F32: "f32", AH_BF16: "bf16"}.get(v.reorder_dtype)
-    return dict(n=v.n, d=v.d, num_leaves=v.num_leaves, dims_per_block=v.dims_per_block, reorder_dtype=rdt)
+    return dict(n=v.n, d=v.d, num_leaves=v.num_leaves, dims_per_block=v.dims_per_block, reorder_dtype=rdt,
+                residual=bool(v.residual))
 
 
 class Index:
@@ -179,7 +224,8 @@ class Index:
         v = Views(self.n, self.d, self.num_leaves, self.dims_per_block, c.data_ptr(),
                   arrays.leaf_offsets.data_ptr(), arrays.slot_ids.data_ptr(), arrays.codes.data_ptr(),
                   arrays.codebook.data_ptr(), rv.data_ptr() if rv is not None else None,
-                  AH_BF16 if (rv is not None and rv.dtype == torch.bfloat16) else AH_F32)
+                  AH_BF16 if (rv is not None and rv.dtype == torch.bfloat16) else AH_F32,
+                  1 if getattr(arrays, "residual", False) else 0)
         h = ctypes.c_void_p()
         with torch.cuda.device(dev):
             _check(self._lib, self._lib.ah_build_index_views(ctypes.byref(v), _stream(stream), ctypes.byref(h)))

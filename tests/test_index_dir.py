@@ -11,7 +11,7 @@ import pytest
 from mips_ivf_centroid_b200 import datagen
 
 
-def _write(path, arr, reorder="f32"):
+def _write(path, arr, reorder="f32", residual=None):
     os.makedirs(path, exist_ok=True)
     for k in ("centroids", "leaf_offsets", "slot_ids", "codes", "codebook"):
         np.save(os.path.join(path, f"{k}.npy"), arr[k])
@@ -19,6 +19,8 @@ def _write(path, arr, reorder="f32"):
         np.save(os.path.join(path, "reorder_vecs.npy"), arr["reorder_vecs"])
     with open(os.path.join(path, "ah_index.txt"), "w") as f:
         f.write(f"ah-index 1\nreorder_dtype {reorder or 'none'}\n")
+        if residual is not None:
+            f.write(f"residual {residual}\n")
 
 
 @pytest.fixture(scope="module")
@@ -41,7 +43,7 @@ def test_inspect_reads_numpy_written_directory(tmp_path, arrays):
     w, arr = arrays
     _write(tmp_path, arr)
     info = inspect(str(tmp_path))
-    assert info == dict(n=3000, d=20, num_leaves=30, dims_per_block=2, reorder_dtype="f32")
+    assert info == dict(n=3000, d=20, num_leaves=30, dims_per_block=2, reorder_dtype="f32", residual=False)
 
 
 def test_inspect_bf16_and_no_reorder_copy(tmp_path, arrays):
@@ -54,6 +56,18 @@ def test_inspect_bf16_and_no_reorder_copy(tmp_path, arrays):
     assert inspect(str(tmp_path / "b"))["reorder_dtype"] == "bf16"
     _write(tmp_path / "n", arr, reorder=None)
     assert inspect(str(tmp_path / "n"))["reorder_dtype"] is None
+
+
+def test_inspect_residual_line(tmp_path, arrays):
+    from mips_ivf_centroid_b200 import inspect
+    w, arr = arrays
+    _write(tmp_path / "r1", arr, residual=1)
+    assert inspect(str(tmp_path / "r1"))["residual"] is True
+    _write(tmp_path / "r0", arr, residual=0)
+    assert inspect(str(tmp_path / "r0"))["residual"] is False
+    _write(tmp_path / "bad", arr, residual=2)
+    st, msg = _status(lambda: inspect(str(tmp_path / "bad")))
+    assert st == 1 and "ah_index.txt" in msg
 
 
 @pytest.mark.parametrize("case", ["missing", "dtype", "offsets", "codes", "truncated", "fortran", "meta",

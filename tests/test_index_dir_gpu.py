@@ -19,11 +19,12 @@ def lib():
     return Index
 
 
-@pytest.mark.parametrize("reorder_dtype", ["f32", "bf16"])
-def test_save_load_round_trip(tmp_path, lib, reorder_dtype):
+@pytest.mark.parametrize("reorder_dtype,residual", [("f32", False), ("bf16", False), ("f32", True)])
+def test_save_load_round_trip(tmp_path, lib, reorder_dtype, residual):
     Index = lib
     w = datagen.WORKLOADS["glove"].scaled(n=40_000, d=64, num_leaves=200, num_leaves_to_search=12, nq=128,
-                                          n_means=60, training_sample_size=40_000, reorder_dtype=reorder_dtype)
+                                          n_means=60, training_sample_size=40_000, reorder_dtype=reorder_dtype,
+                                          residual=residual)
     X = datagen.make_data(w)
     Q = torch.from_numpy(datagen.make_queries(w)).cuda()
     ix = datagen.build_index(w, X, "cuda")
@@ -39,7 +40,7 @@ def test_save_load_round_trip(tmp_path, lib, reorder_dtype):
     assert (b.n, b.d, b.num_leaves, b.dims_per_block) == (w.n, w.d, w.num_leaves, w.dims_per_block)
     assert b.memory_bytes() >= sum(arr[k].nbytes for k in ("centroids", "leaf_offsets", "slot_ids", "codes",
                                                              "codebook", "reorder_vecs"))
-    for mode in (0, 1):
+    for mode in ((0,) if residual else (0, 1)):
         for R in (100, 0):
             ia, sa = a.search(Q, 10, w.num_leaves_to_search, R, mode)
             ib, sb = b.search(Q, 10, w.num_leaves_to_search, R, mode)

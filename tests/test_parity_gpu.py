@@ -51,6 +51,8 @@ def _workload(name):
         "gemm128-scalar": W["glove"].scaled(n=40_000, d=34, dims_per_block=1, num_leaves=2048,
                                             num_leaves_to_search=8, nq=2048, n_means=100,
                                             training_sample_size=40_000),
+        "glove-mini-residual": W["glove"].scaled(n=60_000, num_leaves=300, num_leaves_to_search=24, nq=300,
+                                                 n_means=120, training_sample_size=60_000, residual=True),
         "small-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=600, num_leaves_to_search=2, nq=64,
                                           n_means=10, training_sample_size=3_000, code_loss="l2",
                                           threshold_T=None),
@@ -186,6 +188,22 @@ def test_large_batch_centroid_tiles(Index, name):
     w, X, Q, ix, arr = _workload(name)
     index = Index(ix)
     compare_search(index, arr, Q, 10, w.num_leaves_to_search, 100, 0, qsel=np.arange(0, w.nq, 16))
+    index.close()
+
+
+@pytest.mark.parametrize("reorder_num", [100, 0])
+def test_residual_codes(Index, reorder_num):
+    # codes of x minus its leaf's centroid: scores add the query's centroid score
+    compare(Index, "glove-mini-residual", 10, 24, reorder_num, 0)
+
+
+def test_residual_codes_reject_uint8_tables(Index):
+    from mips_ivf_centroid_b200 import AhError
+    w, X, Q, ix, arr = _workload("glove-mini-residual")
+    index = Index(ix)
+    with pytest.raises(AhError) as e:
+        index.search(torch.from_numpy(Q[:4]).cuda(), 10, 24, 100, 1)
+    assert e.value.status == 2
     index.close()
 
 
