@@ -46,17 +46,4 @@ __device__ __forceinline__ uint32_t key_score(uint64_t key) {
     return static_cast<uint32_t>(key >> 32);
 }
 
-// Packed fp32x2 add (sm_100): two independent IEEE round-to-nearest adds.
-__device__ __forceinline__ unsigned long long add_f32x2(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ float lo_f32(unsigned long long v) {
-    return __uint_as_float(static_cast<uint32_t>(v & 0xFFFFFFFFull));
-}
-__device__ __forceinline__ float hi_f32(unsigned long long v) {
-    return __uint_as_float(static_cast<uint32_t>(v >> 32));
-}
-
 }  // namespace ah

@@ -394,23 +394,6 @@ __device__ uint64_t block_kth_largest(GetKey get, int n, int K, SelectScratch& s
 
 namespace ah {
 
-// The K-th largest of n distinct keys (1 <= K <= n), computed by one warp
-// without sorting; all lanes return it.
-template <class GetKey>
-__device__ uint64_t warp_kth_largest(GetKey get, int n, int K, int* hist) {
-    uint64_t prefix = 0ull, mask = 0ull;
-    if (K < n) warp_select_threshold(get, n, K, hist, &prefix, &mask);
-    uint64_t mn = ~0ull;
-    for (int i = threadIdx.x & 31; i < n; i += 32) {
-        const uint64_t k = get(i);
-        if ((k & mask) >= prefix && k < mn) mn = k;
-    }
-    const unsigned hi = __reduce_min_sync(0xFFFFFFFFu, static_cast<unsigned>(mn >> 32));
-    const unsigned lo = __reduce_min_sync(0xFFFFFFFFu, (static_cast<unsigned>(mn >> 32) == hi)
-                                                           ? static_cast<unsigned>(mn) : 0xFFFFFFFFu);
-    return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
 }  // namespace ah
 
 // ---------------------------------------------------------------------------
