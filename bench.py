@@ -40,7 +40,7 @@ SM_MAX_MHZ_FALLBACK = 1965.0
 # DRAM bytes (read + write) that one ncu capture counted for one scan launch, per
 # (workload, table mode) at the workload's default batch; None where no capture
 # of the current scan kernel exists.
-SCAN_TRAFFIC_BYTES = {("glove", 0): 35.81e6}
+SCAN_TRAFFIC_BYTES = {("glove", 0): 35.79e6}
 
 
 def parse():
@@ -52,7 +52,10 @@ def parse():
     p.add_argument("--workload", default="glove")
     p.add_argument("--lut-mode", type=int, default=0, choices=[0, 1])
     p.add_argument("--nq", type=int, default=None)
-    p.add_argument("--leaves", type=int, default=None)
+    p.add_argument("--leaves", type=int, default=None, help="num_leaves_to_search")
+    p.add_argument("--n", type=int, default=None,
+                   help="reduced point count (profiling captures): means and training sample scale along")
+    p.add_argument("--num-leaves", type=int, default=None, help="partition size with --n")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--e2e-steps", type=int, default=100)
@@ -172,6 +175,10 @@ def workload_spec(args):
         w = w.scaled(nq=args.nq)
     if args.leaves:
         w = w.scaled(num_leaves_to_search=args.leaves)
+    if args.n:
+        nl = args.num_leaves or max(1, w.num_leaves * args.n // w.n)
+        w = w.scaled(n=args.n, num_leaves=nl, n_means=max(1, w.n_means * args.n // w.n),
+                     training_sample_size=min(w.training_sample_size, args.n))
     return w
 
 

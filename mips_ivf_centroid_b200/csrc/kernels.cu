@@ -1109,7 +1109,7 @@ struct TileJob {
 // The warps of a CTA split the item's tiles; a lane owns one slot.  Blocks are
 // summed in order 0..B-1 with IEEE fp32 adds (two queries per packed add), the
 // order every kernel that scores a slot uses.
-template <int G, int NT>
+template <int G, int NT, bool RES>
 __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                                const TileJob& job, const int* s_q, const uint32_t* s_th,
                                                const uint32_t* s_tl, const float* s_off) {
@@ -1139,7 +1139,7 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize) {
                 const float sum = (qi & 1) ? acc[qi >> 1].y : acc[qi >> 1].x;
-                const float sc = ix.residual ? __fadd_rn(sum, s_off[qi]) : sum;
+                const float sc = RES ? __fadd_rn(sum, s_off[qi]) : sum;
                 const uint32_t key = float_key(sc);
                 append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot, s_q[qi], ix, b);
             }
@@ -1202,9 +1202,17 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #ifndef AH_SCAN_MIN_BLOCKS
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
+// uint8 groups of 16 queries keep 24 accumulator registers per lane: 48
+// registers (5 CTAs per SM) hold them without spilling
+#ifndef AH_SCAN_MIN_BLOCKS_U8
+#define AH_SCAN_MIN_BLOCKS_U8 5
+#endif
 
-template <int MODE, int NT, int GMAX>
-__global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 512 ? 2 : 1)))
+// RES: residual codes (each query's centroid score of the leaf is added to its
+// sums); a separate instantiation so plain indexes pay nothing for it.
+template <int MODE, int NT, int GMAX, bool RES>
+__global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOCKS : AH_SCAN_MIN_BLOCKS_U8)
+                                                 : (NT == 512 ? 2 : 1)))
     scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
     constexpr int GSTEP = (MODE == 0) ? 2 : 4;
@@ -1258,7 +1266,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 5
             uint64_t t = (qq >= 0) ? b.tau[qq] : ~0ull;
             s_th[threadIdx.x] = static_cast<uint32_t>(t >> 32);
             s_tl[threadIdx.x] = static_cast<uint32_t>(t);
-            s_off[threadIdx.x] = (ix.residual && qq >= 0) ? b.cscore[static_cast<int64_t>(qq) * ix.nl + leaf] : 0.0f;
+            if (RES) s_off[threadIdx.x] = (qq >= 0) ? b.cscore[static_cast<int64_t>(qq) * ix.nl + leaf] : 0.0f;
         }
         __syncthreads();
         // stage the group's tables
@@ -1302,10 +1310,10 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? AH_SCAN_MIN_BLOCKS : (NT == 5
         __syncthreads();
         if (MODE == 0) {
             switch (G) {
-                case 8: scan_tiles_f32<8, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
-                case 6: scan_tiles_f32<6, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
-                case 4: scan_tiles_f32<4, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
-                default: scan_tiles_f32<2, NT>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                case 8: scan_tiles_f32<8, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                case 6: scan_tiles_f32<6, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                case 4: scan_tiles_f32<4, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
+                default: scan_tiles_f32<2, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
             }
         } else {
             switch (G) {
@@ -1347,7 +1355,7 @@ int scan_group(const DeviceIndex& ix, int lut_mode) {
     return g;
 }
 
-template <int MODE, int NT, int GMAX>
+template <int MODE, int NT, int GMAX, bool RES>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
     size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
@@ -1355,13 +1363,13 @@ static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const Sear
     const size_t room = (NT == 512) ? 110 * 1024 : 200 * 1024;
     a.scan_item_off_smem = (smem + off_bytes <= room && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT, GMAX>), smem, true);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT, GMAX, RES>), smem, true);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT, GMAX>, NT, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT, GMAX, RES>, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT, GMAX>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
+    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT, GMAX, RES>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -1369,13 +1377,19 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
     int nt, g;
     scan_shape(ix, a.lut_mode, &nt, &g);
     if (a.lut_mode == 0) {
-        if (nt == 256) return launch_scan_t<0, 256, kGroupF32>(ix, a, b, num_sms, s);
-        if (nt == 512) return launch_scan_t<0, 512, kGroupF32 / 2>(ix, a, b, num_sms, s);
-        return launch_scan_t<0, 1024, kGroupF32>(ix, a, b, num_sms, s);
+        if (ix.residual) {
+            if (nt == 256) return launch_scan_t<0, 256, kGroupF32, true>(ix, a, b, num_sms, s);
+            if (nt == 512) return launch_scan_t<0, 512, kGroupF32 / 2, true>(ix, a, b, num_sms, s);
+            return launch_scan_t<0, 1024, kGroupF32, true>(ix, a, b, num_sms, s);
+        }
+        if (nt == 256) return launch_scan_t<0, 256, kGroupF32, false>(ix, a, b, num_sms, s);
+        if (nt == 512) return launch_scan_t<0, 512, kGroupF32 / 2, false>(ix, a, b, num_sms, s);
+        return launch_scan_t<0, 1024, kGroupF32, false>(ix, a, b, num_sms, s);
     }
-    if (nt == 256) return launch_scan_t<1, 256, kGroupU8>(ix, a, b, num_sms, s);
-    if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2>(ix, a, b, num_sms, s);
-    return launch_scan_t<1, 1024, kGroupU8>(ix, a, b, num_sms, s);
+    // uint8 tables are refused for residual codes before any launch
+    if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
+    if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
+    return launch_scan_t<1, 1024, kGroupU8, false>(ix, a, b, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------
