@@ -48,16 +48,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
+    srcs = _sources()
+    objs = [os.path.join(BUILD, os.path.basename(src)[:-3] + ".o") for src in srcs]
+    # one nvcc per source, all at once
+    procs = [subprocess.Popen([nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj],
+                              stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+             for src, obj in zip(srcs, objs)]
     logs = []
-    for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        logs.append(r.stdout + r.stderr)
-        if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
-        objs.append(obj)
+    failed = []
+    for src, pr in zip(srcs, procs):
+        out, _ = pr.communicate()
+        logs.append(out)
+        if pr.returncode != 0:
+            failed.append(f"nvcc failed for {src}:\n{out}")
+    if failed:
+        raise RuntimeError("\n".join(failed))
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
            "-Xcompiler", "-fPIC"]
