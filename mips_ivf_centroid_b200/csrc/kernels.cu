@@ -1202,10 +1202,11 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #ifndef AH_SCAN_MIN_BLOCKS
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
-// uint8 groups of 16 queries keep 24 accumulator registers per lane: 48
-// registers (5 CTAs per SM) hold them without spilling
+// uint8 groups of 16 queries keep 24 accumulator registers per lane; at 6
+// CTAs per SM (40 registers) a few spill to L1, which measured slightly faster
+// than 5 or 4 CTAs without spills
 #ifndef AH_SCAN_MIN_BLOCKS_U8
-#define AH_SCAN_MIN_BLOCKS_U8 5
+#define AH_SCAN_MIN_BLOCKS_U8 6
 #endif
 
 // RES: residual codes (each query's centroid score of the leaf is added to its
