@@ -141,8 +141,8 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __res
     chain_entry();
     constexpr int PT = TM / 16;              // outputs per thread per dimension
     constexpr int LOADS = TM * kGemmBK / 256;
-    __shared__ float As[kGemmBK][TM + 4];
-    __shared__ float Bs[kGemmBK][TM + 4];
+    __shared__ float As[2][kGemmBK][TM + 4];
+    __shared__ float Bs[2][kGemmBK][TM + 4];
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TM;
     float acc[PT][PT];
@@ -150,30 +150,50 @@ __global__ void __launch_bounds__(256) centroid_scores_kernel(const float* __res
     for (int i = 0; i < PT; ++i)
 #pragma unroll
         for (int j = 0; j < PT; ++j) acc[i][j] = 0.0f;
-    for (int k0 = 0; k0 < d; k0 += kGemmBK) {
+    // the next k step's operands are loaded into registers while the current
+    // one is multiplied (each output still accumulates over k in order)
+    float ra[LOADS], rb[LOADS];
+    auto gload = [&](int k0) {
 #pragma unroll
         for (int r = 0; r < LOADS; ++r) {
-            int e = threadIdx.x + 256 * r;
-            int row = e >> 4, col = e & 15;
-            int gk = k0 + col;
-            int gm = m0 + row, gn = n0 + row;
-            As[col][row] = (gm < nq && gk < d) ? Q[static_cast<int64_t>(gm) * d + gk] : 0.0f;
-            Bs[col][row] = (gn < nl && gk < d) ? C[static_cast<int64_t>(gn) * d + gk] : 0.0f;
+            const int e = threadIdx.x + 256 * r;
+            const int row = e >> 4, col = e & 15;
+            const int gk = k0 + col, gm = m0 + row, gn = n0 + row;
+            ra[r] = (gm < nq && gk < d) ? Q[static_cast<int64_t>(gm) * d + gk] : 0.0f;
+            rb[r] = (gn < nl && gk < d) ? C[static_cast<int64_t>(gn) * d + gk] : 0.0f;
         }
-        __syncthreads();
+    };
+    auto sstore = [&](int buf) {
+#pragma unroll
+        for (int r = 0; r < LOADS; ++r) {
+            const int e = threadIdx.x + 256 * r;
+            const int row = e >> 4, col = e & 15;
+            As[buf][col][row] = ra[r];
+            Bs[buf][col][row] = rb[r];
+        }
+    };
+    gload(0);
+    sstore(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < d; k0 += kGemmBK) {
+        const bool more = k0 + kGemmBK < d;
+        if (more) gload(k0 + kGemmBK);
 #pragma unroll
         for (int kk = 0; kk < kGemmBK; ++kk) {
             float av[PT], bv[PT];
 #pragma unroll
-            for (int i = 0; i < PT; ++i) av[i] = As[kk][ty + 16 * i];
+            for (int i = 0; i < PT; ++i) av[i] = As[buf][kk][ty + 16 * i];
 #pragma unroll
-            for (int j = 0; j < PT; ++j) bv[j] = Bs[kk][tx + 16 * j];
+            for (int j = 0; j < PT; ++j) bv[j] = Bs[buf][kk][tx + 16 * j];
 #pragma unroll
             for (int i = 0; i < PT; ++i)
 #pragma unroll
                 for (int j = 0; j < PT; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
+        if (more) sstore(buf ^ 1);
         __syncthreads();
+        buf ^= 1;
     }
 #pragma unroll
     for (int i = 0; i < PT; ++i) {
