@@ -80,6 +80,10 @@ struct ah_index {
     int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
     void* loaded[6] = {};            // index arrays owned by an index from ah_load
+    // side stream for the stages that do not depend on the partition stage
+    // (lookup tables; the query->leaf inversion once top-L is known)
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_tl = nullptr, ev_lut = nullptr, ev_inv = nullptr;
 };
 
 namespace {
@@ -243,6 +247,24 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     };
     e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)(2 * dix.nl + ix->ws.nq + 8), s);
     if (e != cudaSuccess) return cuda_fail(e, "memset");
+    // With per-stage profiling everything runs in order on s (clean stage
+    // times); otherwise the tables and the inversion run on the side stream,
+    // joined back before the threshold and the scan.
+    const bool fork = ix->profiling != 1;
+    if (fork && !ix->side) {
+        if ((e = cudaStreamCreateWithFlags(&ix->side, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "side stream");
+        for (cudaEvent_t* ev : {&ix->ev_fork, &ix->ev_tl, &ix->ev_lut, &ix->ev_inv})
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess)
+                return cuda_fail(e, "side stream events");
+    }
+    const cudaStream_t s2 = fork ? ix->side : s;
+    if (fork) {
+        if ((e = cudaEventRecord(ix->ev_fork, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s2, ix->ev_fork, 0)) != cudaSuccess)
+            return cuda_fail(e, "fork");
+        if ((e = ah::launch_lut(dix, a, b, s2)) != cudaSuccess) return cuda_fail(e, "lut");
+        if ((e = cudaEventRecord(ix->ev_lut, s2)) != cudaSuccess) return cuda_fail(e, "fork");
+    }
     mark(-1);
     if ((e = ah::launch_centroid_scores(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "centroid scores");
     launches += 1;
@@ -270,14 +292,24 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
     launches += 1;
     mark(1);
-    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], true, s)) != cudaSuccess) return cuda_fail(e, "invert");
+    if (fork) {
+        if ((e = cudaEventRecord(ix->ev_tl, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s2, ix->ev_tl, 0)) != cudaSuccess)
+            return cuda_fail(e, "fork");
+    }
+    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], true, s2)) != cudaSuccess) return cuda_fail(e, "invert");
     launches += 2;
     mark(2);
-    if ((e = ah::launch_lut(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "lut");
+    if (fork) {
+        if ((e = cudaEventRecord(ix->ev_inv, s2)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ix->ev_lut, 0)) != cudaSuccess)
+            return cuda_fail(e, "join");
+    } else if ((e = ah::launch_lut(dix, a, b, s)) != cudaSuccess) {
+        return cuda_fail(e, "lut");
+    }
     launches += 1;
     mark(3);
     if ((e = ah::launch_threshold(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "threshold");
     launches += 1;
+    if (fork && (e = cudaStreamWaitEvent(s, ix->ev_inv, 0)) != cudaSuccess) return cuda_fail(e, "join");
     mark(4);
     for (size_t p = 0; p + 1 < bounds.size(); ++p) {
         if (p > 0) {
@@ -592,6 +624,9 @@ void ah_destroy(ah_index* ix) {
     if (ix->err) cudaFree(ix->err);
     for (void* p : ix->loaded)
         if (p) cudaFree(p);
+    for (cudaEvent_t ev : {ix->ev_fork, ix->ev_tl, ix->ev_lut, ix->ev_inv})
+        if (ev) cudaEventDestroy(ev);
+    if (ix->side) cudaStreamDestroy(ix->side);
     if (ix->ev_ready)
         for (int i = 0; i < ah_index::kMaxMarks; ++i) cudaEventDestroy(ix->ev[i]);
     delete ix;
