@@ -64,6 +64,9 @@ def parse():
     p.add_argument("--encode", action="store_true",
                    help="index build: time the anisotropic code assignment over the workload's points")
     p.add_argument("--passes", type=int, default=10)
+    p.add_argument("--leaf-shards", action="store_true",
+                   help="leaf-partitioned search: rank r scans the leaves c with c % N == r for the whole batch; "
+                        "candidates are gathered and merged exactly (strong scaling)")
     p.add_argument("--kmeans", action="store_true",
                    help="index build: time one k-means iteration (assignment + update) over the workload's points")
     return p.parse_args()
@@ -588,10 +591,74 @@ def run_kmeans(args):
     print(json.dumps(line), flush=True)
 
 
+def run_leaf_shards(args):
+    """One JSON line: the leaf-partitioned search.  Every rank holds all
+    centroids and the codebook and the points of its own leaves, searches the
+    same batch, and the ranks' best R (with exact scores) are gathered and
+    merged; value = queries / the slowest rank's device time per step."""
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_ranks(world, dev)
+    from mips_ivf_centroid_b200 import Index, build as ahbuild, datagen, shard
+    ahbuild.build()
+    w = workload_spec(args)
+    X = datagen.make_data(w)
+    Q = datagen.make_queries(w)
+    full = datagen.build_index(w, X, dev)
+    del X
+    sh = shard.shard_arrays(full, world, rank)
+    del full
+    torch.cuda.empty_cache()
+    index = Index(sh)
+    qg = torch.from_numpy(Q).to(dev)
+    L, k, R, mode = w.num_leaves_to_search, w.k, w.reorder_num, args.lut_mode
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        local_c = shard.shard_candidates(index, qg, k, L, R, mode)
+        g = shard.gather_candidates(local_c) if world > 1 else tuple(
+            None if t is None else t.unsqueeze(0).contiguous() for t in local_c)
+        return shard.merge_gathered(g, k)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    total = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev, world)
+    ms = total / args.steps
+    if rank == 0:
+        line = {"metric": METRIC, "value": w.nq / (ms * 1e-3), "unit": "queries/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "f32" if mode == 0 else "u8",
+                "data": "synthetic (seeded Gaussian mixture; index trained on it)",
+                "config": dict(config_dict(w, args), parallelism=f"leaf-partitioned x{world}"),
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    index.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.leaf_shards:
+        run_leaf_shards(args)
     elif args.kmeans:
         run_kmeans(args)
     elif args.encode:

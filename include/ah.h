@@ -161,6 +161,8 @@ AH_API ah_status ah_search(ah_index *ix, const float *queries, int32_t nq, int32
  *   passed                 [nq]     points whose approximate score reached the
  *                                   query's filter bound in the first scan pass
  *   rescans                [1]      queries rescanned after a buffer overflow
+ *   cand_exact             [nq][R]  with reorder_num > 0: the exact score of
+ *                                   each of cand_ids (same order; padded -inf)
  */
 typedef struct {
     int32_t *leaf_ids;
@@ -172,6 +174,7 @@ typedef struct {
     int64_t *scanned;
     int32_t *passed;
     int32_t *rescans;
+    float *cand_exact;
 } ah_search_trace;
 
 /* ah_search plus the intermediate results named in *trace (may be NULL). */
@@ -375,6 +378,30 @@ AH_API ah_status ah_kmeans_assign(const float *X, int64_t n, int32_t d, const fl
                                   double *dist, void *cuda_stream);
 AH_API ah_status ah_kmeans_update(const float *X, int64_t n, int32_t d, const int32_t *assign, int32_t nl,
                                   const float *C_old, float *C_new, int64_t *counts, void *cuda_stream);
+
+/*
+ * Exact merge for a leaf-partitioned search.  G shards hold the same
+ * centroids and codebook and disjoint sets of leaves' points (the other
+ * leaves empty), so every shard picks the same L leaves and scans its own
+ * points of them; the union of the shards' best R by approximate score holds
+ * the best R of all points.  Per query this keeps the best R of the G * R
+ * entries by (approx desc, id asc) and returns the best k of those by
+ * (exact desc, id asc): the result one index over all points gives.
+ *   cand_ids     [G][nq][R] int32 (id < 0: padding)    device
+ *   cand_approx  [G][nq][R] float: descending order = approximate ranking
+ *                (ah_search_trace.cand_scores with fp32 tables; the integer
+ *                sums converted to float with uint8 tables)
+ *   cand_exact   [G][nq][R] float (ah_search_trace.cand_exact), or NULL when
+ *                searched without reorder: the best k by approx are returned
+ *   out_ids [nq][k] int32, out_scores [nq][k] float (exact, or approx without
+ *                reorder; padding -1 / -inf)            device
+ * Asynchronous on cuda_stream.  Errors: AH_ERR_INVALID_ARG (NULL array,
+ * G < 1, nq < 0, k < 1, R < k), AH_ERR_UNSUPPORTED (R above AH_MAX_R,
+ * G * R above 65536), AH_ERR_CUDA.
+ */
+AH_API ah_status ah_merge_shards(int32_t G, int32_t nq, int32_t R, int32_t k, const int32_t *cand_ids,
+                                 const float *cand_approx, const float *cand_exact, int32_t *out_ids,
+                                 float *out_scores, void *cuda_stream);
 
 AH_API void ah_destroy(ah_index *ix);
 

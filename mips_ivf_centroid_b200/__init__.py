@@ -9,14 +9,15 @@ the first ``Index`` does, and raises if the library is missing.
 """
 from __future__ import annotations
 
-__all__ = ["Index", "AhError", "load_library", "inspect", "encode", "kmeans_assign", "kmeans_update", "LUT_F32", "LUT_U8"]
+__all__ = ["Index", "AhError", "load_library", "inspect", "encode", "kmeans_assign", "kmeans_update", "merge_shards", "LUT_F32", "LUT_U8"]
 
 LUT_F32 = 0
 LUT_U8 = 1
 
 
 def __getattr__(name):
-    if name in ("Index", "AhError", "load_library", "inspect", "encode", "kmeans_assign", "kmeans_update"):
+    if name in ("Index", "AhError", "load_library", "inspect", "encode", "kmeans_assign", "kmeans_update",
+                "merge_shards"):
         from . import index as _index
         return getattr(_index, name)
     raise AttributeError(name)

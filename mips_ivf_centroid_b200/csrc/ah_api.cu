@@ -229,6 +229,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
         a.tr_ncand = tr->ncand;
         a.tr_scanned = tr->scanned;
         a.tr_passed = tr->passed;
+        a.tr_cand_exact = tr->cand_exact;
         a.tr_rescans = tr->rescans;
     }
     const ah::DeviceIndex& dix = ix->dix;
@@ -956,4 +957,21 @@ ah_status ah_kmeans_update(const float* X, int64_t n, int32_t d, const int32_t* 
     const cudaError_t e = ah::launch_kmeans_update(X, n, d, assign, nl, C_old, C_new, counts,
                                                    static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? AH_OK : cuda_fail(e, "k-means update");
+}
+
+// ---------------------------------------------------------------------------
+// leaf-partitioned search: exact merge of the shards' candidates
+// ---------------------------------------------------------------------------
+
+ah_status ah_merge_shards(int32_t G, int32_t nq, int32_t R, int32_t k, const int32_t* cand_ids,
+                          const float* cand_approx, const float* cand_exact, int32_t* out_ids, float* out_scores,
+                          void* cuda_stream) {
+    if (G < 1 || nq < 0 || k < 1 || R < k) return fail(AH_ERR_INVALID_ARG, "need G >= 1, nq >= 0, 1 <= k <= R");
+    if (R > AH_MAX_R) return fail(AH_ERR_UNSUPPORTED, "R above AH_MAX_R");
+    if (static_cast<int64_t>(G) * R > 65536) return fail(AH_ERR_UNSUPPORTED, "G * R above 65536");
+    if (nq == 0) return AH_OK;
+    if (!cand_ids || !cand_approx || !out_ids || !out_scores) return fail(AH_ERR_INVALID_ARG, "NULL array");
+    const cudaError_t e = ah::launch_merge_shards(G, nq, R, k, cand_ids, cand_approx, cand_exact, out_ids, out_scores,
+                                                  static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? AH_OK : cuda_fail(e, "shard merge");
 }

@@ -1789,6 +1789,9 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         if (i < K && gl == 0) ekeys[i] = make_key(float_key(acc), key_id(okeys[i]));
     }
     __syncthreads();
+    if (a.tr_cand_exact)
+        for (int i = threadIdx.x; i < R; i += kFinishThreads)
+            a.tr_cand_exact[ro + i] = (i < K) ? key_float(key_score(ekeys[i])) : -INFINITY;
     auto eget = [&](int i) { return ekeys[i]; };
     auto epay = [&](int i) { return i; };
     if (k <= kWarpMaxK) {

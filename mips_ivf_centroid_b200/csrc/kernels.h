@@ -84,6 +84,7 @@ struct SearchArgs {
     int32_t* tr_ncand;
     int64_t* tr_scanned;
     int32_t* tr_passed;
+    float* tr_cand_exact;       // [nq][R] exact scores of the traced candidates
     int32_t* tr_rescans;
     int scan_item_off_smem;     // set by the scan launcher
     int topl_row_smem;          // set by the top-leaves launcher
@@ -128,5 +129,9 @@ cudaError_t launch_kmeans_assign(const float* X, int64_t n, int d, const float* 
 size_t kmeans_update_smem_bytes(int d);
 cudaError_t launch_kmeans_update(const float* X, int64_t n, int d, const int32_t* assign, int nl, const float* C_old,
                                  float* C_new, int64_t* counts, cudaStream_t s);
+
+// exact merge of per-shard candidates (merge.cu)
+cudaError_t launch_merge_shards(int G, int nq, int R, int k, const int32_t* ids, const float* approx,
+                                const float* exact, int32_t* out_ids, float* out_scores, cudaStream_t s);
 
 }  // namespace ah

@@ -51,7 +51,7 @@ class Views(ctypes.Structure):
 class Trace(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("leaf_ids", "leaf_scores", "cand_ids", "cand_scores", "cand_sums", "ncand", "scanned",
-                 "passed", "rescans")]
+                 "passed", "rescans", "cand_exact")]
 
 
 def load_library(path: Optional[str] = None) -> ctypes.CDLL:
@@ -84,6 +84,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_kmeans_assign": (I32, [P, I64, I32, P, I32, P, P, P]),
         "ah_kmeans_update": (I32, [P, I64, I32, P, I32, P, P, P, P]),
         "ah_save": (I32, [P, ctypes.c_char_p]),
+        "ah_merge_shards": (I32, [I32, I32, I32, I32, P, P, P, P, P, P]),
         "ah_inspect": (I32, [ctypes.c_char_p, P]),
         "ah_load": (I32, [ctypes.c_char_p, P, ctypes.POINTER(P)]),
         "ah_set_option": (I32, [P, I32, I64]),
@@ -177,6 +178,31 @@ def kmeans_update(X: torch.Tensor, assign: torch.Tensor, C_old: torch.Tensor, st
         _check(lib, lib.ah_kmeans_update(_ptr(X), n, d, _ptr(assign), nl, _ptr(C_old), _ptr(C_new), _ptr(counts),
                                          _stream(stream)))
     return C_new, counts
+
+
+def merge_shards(cand_ids: torch.Tensor, cand_approx: torch.Tensor, cand_exact: Optional[torch.Tensor], k: int,
+                 stream=None):
+    """Exact merge of a leaf-partitioned search (``ah_merge_shards``).
+
+    cand_ids [G, nq, R] int32, cand_approx [G, nq, R] float32 (descending =
+    approximate ranking), cand_exact [G, nq, R] float32 or None (searched
+    without reorder), all on one CUDA device.  Returns (ids [nq, k] int32,
+    scores [nq, k] float32)."""
+    lib = load_library()
+    if cand_ids.dtype != torch.int32 or cand_ids.dim() != 3 or not cand_ids.is_contiguous() \
+            or cand_ids.device.type != "cuda":
+        raise AhError(1, "cand_ids: need contiguous int32 [G, nq, R] on a CUDA device")
+    for name, t in (("cand_approx", cand_approx), ("cand_exact", cand_exact)):
+        if t is not None and (t.dtype != torch.float32 or t.shape != cand_ids.shape or not t.is_contiguous()
+                              or t.device != cand_ids.device):
+            raise AhError(1, f"{name}: need contiguous float32 like cand_ids")
+    G, nq, R = cand_ids.shape
+    ids = torch.empty((nq, k), dtype=torch.int32, device=cand_ids.device)
+    scores = torch.empty((nq, k), dtype=torch.float32, device=cand_ids.device)
+    with torch.cuda.device(cand_ids.device):
+        _check(lib, lib.ah_merge_shards(G, nq, R, k, _ptr(cand_ids), _ptr(cand_approx), _ptr(cand_exact), _ptr(ids),
+                                        _ptr(scores), _stream(stream)))
+    return ids, scores
 
 
 def inspect(path: str) -> dict:
@@ -290,7 +316,8 @@ class Index:
                      ncand=torch.empty((nq,), dtype=torch.int32, device=self.device),
                      scanned=torch.empty((nq,), dtype=torch.int64, device=self.device),
                      passed=torch.empty((nq,), dtype=torch.int32, device=self.device),
-                     rescans=torch.zeros((1,), dtype=torch.int32, device=self.device))
+                     rescans=torch.zeros((1,), dtype=torch.int32, device=self.device),
+                     cand_exact=torch.full((nq, R), float("-inf"), dtype=torch.float32, device=self.device))
             tr = Trace(*[t[n].data_ptr() for n, _ in Trace._fields_])
             _check(self._lib, self._lib.ah_search_traced(self._h, _ptr(q), nq, k, num_leaves_to_search, reorder_num,
                                                          lut_mode, _ptr(ids), _ptr(scores), ctypes.byref(tr), s))
