@@ -322,6 +322,9 @@ cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, c
     return cudaGetLastError();
 }
 
+#ifndef AH_SCAN_LAST_BATCH
+#define AH_SCAN_LAST_BATCH 0
+#endif
 #ifndef AH_REORDER_BATCH
 #define AH_REORDER_BATCH 4
 #endif
@@ -1062,6 +1065,24 @@ __device__ __forceinline__ void append_candidates(bool pass, uint32_t key, int32
     }
 }
 
+// Keep (value, slot) for query qi of the group when it reaches the query's
+// bound.  Only the bound's score word is read for every slot: its id word is
+// read when some lane ties it exactly, and the query index when some lane
+// passes (both rare), each behind a warp vote so that no lane reads them
+// otherwise.
+__device__ __forceinline__ void keep_if_reaches(bool valid, uint32_t v, int32_t slot, int qi, const int* s_q,
+                                                const uint32_t* s_th, const uint32_t* s_tl, const DeviceIndex& ix,
+                                                const SearchBuffers& b) {
+    const uint32_t th = s_th[qi];
+    bool pass = valid && v >= th;
+    const bool tie = pass && v == th;
+    if (__any_sync(0xFFFFFFFFu, tie)) {
+        const uint32_t tl = s_tl[qi];
+        if (tie) pass = (0xFFFFFFFFu - static_cast<uint32_t>(ix.slot_ids[slot])) >= tl;
+    }
+    if (__any_sync(0xFFFFFFFFu, pass)) append_candidates(pass, v, slot, s_q[qi], ix, b);
+}
+
 // One code word (8 blocks) for a group of G queries, fp32 tables staged as
 // [b][G/2][16] float2: per nibble one 8-byte shared load per query pair, one
 // packed add.  `base` points at block 8w's tables.
@@ -1153,15 +1174,29 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
             f32_word<G>(c2, lut2 + (8 * w + 16) * BS, acc);
             f32_word<G>(c3, lut2 + (8 * w + 24) * BS, acc);
         }
+#if AH_SCAN_LAST_BATCH
+        // the remaining full words and the tail word (at most 4) in one batch
+        if (w < W) {
+            uint32_t c[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) c[i] = (w + i < W) ? cwp[(w + i) * 32] : 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (w + i < Wf) f32_word<G>(c[i], lut2 + 8 * (w + i) * BS, acc);
+                else if (w + i == Wf && tail) f32_tail<G>(c[i], tail, lut2 + 8 * Wf * BS, acc);
+            }
+        }
+#else
         for (; w < Wf; ++w) f32_word<G>(cwp[w * 32], lut2 + 8 * w * BS, acc);
         if (tail) f32_tail<G>(cwp[Wf * 32], tail, lut2 + 8 * Wf * BS, acc);
+#endif
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize) {
                 const float sum = (qi & 1) ? acc[qi >> 1].y : acc[qi >> 1].x;
                 const float sc = RES ? __fadd_rn(sum, s_off[qi]) : sum;
                 const uint32_t key = float_key(sc);
-                append_candidates(valid && reaches(key, s_th[qi], s_tl[qi], ix.slot_ids, slot), key, slot, s_q[qi], ix, b);
+                keep_if_reaches(valid, key, slot, qi, s_q, s_th, s_tl, ix, b);
             }
         }
     }
@@ -1207,8 +1242,7 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize)
-                append_candidates(valid && reaches(sums[qi], s_th[qi], s_tl[qi], ix.slot_ids, slot), sums[qi], slot,
-                                  s_q[qi], ix, b);
+                keep_if_reaches(valid, sums[qi], slot, qi, s_q, s_th, s_tl, ix, b);
         }
     }
 }
