@@ -322,9 +322,6 @@ cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, c
     return cudaGetLastError();
 }
 
-#ifndef AH_SCAN_LAST_BATCH
-#define AH_SCAN_LAST_BATCH 0
-#endif
 #ifndef AH_REORDER_BATCH
 #define AH_REORDER_BATCH 4
 #endif
@@ -1174,22 +1171,8 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
             f32_word<G>(c2, lut2 + (8 * w + 16) * BS, acc);
             f32_word<G>(c3, lut2 + (8 * w + 24) * BS, acc);
         }
-#if AH_SCAN_LAST_BATCH
-        // the remaining full words and the tail word (at most 4) in one batch
-        if (w < W) {
-            uint32_t c[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) c[i] = (w + i < W) ? cwp[(w + i) * 32] : 0u;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if (w + i < Wf) f32_word<G>(c[i], lut2 + 8 * (w + i) * BS, acc);
-                else if (w + i == Wf && tail) f32_tail<G>(c[i], tail, lut2 + 8 * Wf * BS, acc);
-            }
-        }
-#else
         for (; w < Wf; ++w) f32_word<G>(cwp[w * 32], lut2 + 8 * w * BS, acc);
         if (tail) f32_tail<G>(cwp[Wf * 32], tail, lut2 + 8 * Wf * BS, acc);
-#endif
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize) {
