@@ -3,9 +3,11 @@
 The search path (centroid scoring -> top-L leaves -> per-query lookup tables ->
 4-bit code scan -> top-R -> exact reorder -> top-k) runs in hand-written sm_100a
 CUDA kernels behind the C ABI declared in ``include/ah.h``; this package is the
-thin Python binding over that library (``Index``), plus the seeded input
-generator ``datagen``.  Importing the package does not load the CUDA library;
-the first ``Index`` does, and raises if the library is missing.
+thin Python binding over that library: ``Index`` (search, save/load),
+``encode`` and ``kmeans_assign``/``kmeans_update`` (index build),
+``merge_shards`` and the ``shard`` module (leaf-partitioned search), plus the
+seeded input generator ``datagen``.  Importing the package does not load the
+CUDA library; the first call that needs it does, and raises if it is missing.
 """
 from __future__ import annotations
 
