@@ -1239,9 +1239,8 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
 #ifndef AH_SCAN_MIN_BLOCKS
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
-// uint8 groups of 16 queries keep 24 accumulator registers per lane; at 6
-// CTAs per SM (40 registers) a few spill to L1, which measured slightly faster
-// than 5 or 4 CTAs without spills
+// uint8 scan: 6 CTAs per SM as for fp32 (groups of 8 queries keep 12
+// accumulator registers per lane, leaving room for loads in flight)
 #ifndef AH_SCAN_MIN_BLOCKS_U8
 #define AH_SCAN_MIN_BLOCKS_U8 6
 #endif

@@ -10,7 +10,7 @@ namespace ah {
 
 // Queries per scan work item (leaf, query group, slot chunk).
 constexpr int kGroupF32 = 8;
-constexpr int kGroupU8 = 16;
+constexpr int kGroupU8 = 8;
 constexpr int kScanThreads = 256;
 #ifndef AH_SAMPLE_MULT
 #define AH_SAMPLE_MULT 4
