@@ -15,8 +15,6 @@ run in the CUDA library.
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional
-
 import torch
 
 from .index import AhError, merge_shards

@@ -18,7 +18,7 @@ import torch
 from mips_ivf_centroid_b200 import datagen
 from oracle import OracleIndex
 
-from parity import ranked_match, same_set, tol
+from parity import ranked_match, same_set
 
 pytestmark = pytest.mark.gpu
 
