@@ -122,6 +122,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     add(stage ? sizeof(int32_t) * (size_t)cnq * ck : 0);        // 16 dids
     add(stage ? sizeof(float) * (size_t)cnq * ck : 0);          // 17 dscores
     add(sizeof(int32_t) * (size_t)cnq * cap);                   // 18 candidate slots
+    add(sizeof(int32_t) * (size_t)cnq);                         // 19 finish order
     size_t total = 0;
     for (int i = 0; i < n; ++i) total += sz[i];
     if (w.base) {
@@ -156,6 +157,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     b.tau = reinterpret_cast<uint64_t*>(part[8]);
     b.ckey = reinterpret_cast<uint64_t*>(part[9]);
     b.cslot = reinterpret_cast<int32_t*>(part[18]);
+    b.order = reinterpret_cast<int32_t*>(part[19]);
     int32_t* zr = reinterpret_cast<int32_t*>(part[10]);
     b.qcount = zr;
     b.qcursor = zr + NL;
@@ -327,7 +329,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
         mark(p == 0 ? 5 : 7);
     }
     if ((e = ah::launch_finish(dix, a, b, 0, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "finish");
-    launches += 1;
+    launches += 2;                                           // the finish order and the finish
     mark(8);
     for (int round = 1; round <= 2; ++round) {
         if ((e = ah::launch_redo_scan(dix, a, b, round, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "rescan");

@@ -1830,6 +1830,19 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
     }
 }
 
+// The finish's CTAs start in grid order, and a query with more than
+// kStageCap kept candidates takes about twice as long as the rest; listing
+// those first keeps them out of the grid's last, partial wave.  (Positions
+// come from atomics; each query's result does not depend on them.)
+__global__ void __launch_bounds__(256) finish_order_kernel(SearchArgs a, SearchBuffers b) {
+    chain_entry();
+    const int q = blockIdx.x * 256 + threadIdx.x;
+    if (q >= a.nq) return;
+    const bool heavy = b.count[q] > kStageCap;
+    const int pos = heavy ? atomicAdd(&b.counters[5], 1) : a.nq - 1 - atomicAdd(&b.counters[6], 1);
+    b.order[pos] = q;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kFinishThreads, AH_FINISH_MIN_BLOCKS) finish_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b, int round) {
     chain_entry();
@@ -1837,7 +1850,7 @@ __global__ void __launch_bounds__(kFinishThreads, AH_FINISH_MIN_BLOCKS) finish_k
     __shared__ SelectScratch scr;
     __shared__ RegSelectScratch<kFinishThreads> rs;
     if (round == 0) {
-        finish_query<MODE>(ix, a, b, 0, blockIdx.x, smem, scr, rs);
+        finish_query<MODE>(ix, a, b, 0, b.order[blockIdx.x], smem, scr, rs);
         return;
     }
     // rescan rounds: a small grid walks the previous round's redo list
@@ -1868,6 +1881,11 @@ cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffe
     const size_t smem = finish_smem_bytes(a.R, ix.d);
     const unsigned grid = (round == 0) ? static_cast<unsigned>(a.nq) : static_cast<unsigned>(std::min(a.nq, 2 * num_sms));
     cudaError_t e;
+    if (round == 0) {
+        if (const cudaError_t le = launch_chained(finish_order_kernel, dim3((a.nq + 255) / 256), dim3(256), 0, s, a, b);
+            le != cudaSuccess)
+            return le;
+    }
     if (a.lut_mode == 0) {
         if ((e = prefer_shared(finish_kernel<0>, smem)) != cudaSuccess) return e;
         if (const cudaError_t le = launch_chained(finish_kernel<0>, dim3(grid), dim3(kFinishThreads), smem, s, ix, a, b, round); le != cudaSuccess) return le;

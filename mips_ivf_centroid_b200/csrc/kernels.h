@@ -56,6 +56,7 @@ struct SearchBuffers {
     int32_t* cslot;         // [nq][cap] and their slots
     int32_t* count;         // [nq]          (zeroed per search)
     int32_t* redo;          // [2][nq]       queries to rescan after rounds 0 and 1
+    int32_t* order;         // [nq]          finish order: queries with many kept candidates first
     int32_t* counters;      // [8]           (zeroed per search): 0 scan work (first phase), 1..2 redo
                             //               list sizes, 3..4 rescan work of rounds 1..2, 5 scan work
                             //               (second phase)
