@@ -15,11 +15,15 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
   centroid means), the other index-build step.
 
 Parity pins: every function here is checked against something other than
-itself in ``tests/test_oracle_pins.py``, ``tests/test_avq_pins.py`` and
-``tests/test_encode_pins.py``, ``tests/test_kmeans_pins.py`` (the code assignment: eta = 1 gives the
-per-block nearest centers, the result is a coordinate-wise minimum of the
-loss computed independently, the loss never rises above the L2 codes' and
-exhaustive search on two blocks bounds it).
+itself: the search in ``tests/test_oracle_pins.py`` (numpy brute force, the
+reconstruction identity, residual codes, an integer special case, hand-worked
+values, the blog's operation counts), the training formulas in
+``tests/test_avq_pins.py``, the code assignment in ``tests/test_encode_pins.py``
+(eta = 1 gives the per-block nearest centers; with one live block the result is
+the exhaustive argmin of the loss as ``avq.py`` computes it; converged codes
+are coordinate-wise minima; never worse than the L2 codes) and partition
+training in ``tests/test_kmeans_pins.py`` (numpy argmin and means, exact ties,
+Lloyd monotonicity).
 """
 from __future__ import annotations
 
