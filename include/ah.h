@@ -13,7 +13,11 @@
  *                    dot products, and the best k are returned.
  * The search-time knobs follow the post's "Using the library" section
  * (search_batched with leaves_to_search and pre_reorder_num_neighbors, and
- * final_num_neighbors).  Training an index is not part of this library.
+ * final_num_neighbors).  Besides the search the library provides the steps
+ * that build an index (anisotropic code assignment, k-means partition
+ * training: ah_encode, ah_kmeans_assign, ah_kmeans_update), index directories
+ * (ah_save, ah_inspect, ah_load) and the exact merge of a leaf-partitioned
+ * search (ah_merge_shards).
  *
  * Conventions for every entry point:
  *  - Status codes only: no exceptions cross the ABI, nothing calls exit/abort.
@@ -28,7 +32,9 @@
  *    than k are padded with id -1 and score -INFINITY.
  *  - Ids are the original datapoint ids (int32).
  *  - An index may be searched from one stream at a time (it owns one
- *    workspace); different indexes are independent.
+ *    workspace, and a side stream for stages that do not depend on the
+ *    partition stage, joined back before the results are written); different
+ *    indexes are independent.
  */
 #ifndef AH_H_
 #define AH_H_
