@@ -64,7 +64,7 @@ def parse():
                    help="index build: time the anisotropic code assignment over the workload's points")
     p.add_argument("--passes", type=int, default=10)
     p.add_argument("--leaf-shards", action="store_true",
-                   help="leaf-partitioned search: rank r scans the leaves c with c % N == r for the whole batch; "
+                   help="leaf-partitioned search: rank r scans the leaves c with c %% N == r for the whole batch; "
                         "candidates are gathered and merged exactly (strong scaling)")
     p.add_argument("--kmeans", action="store_true",
                    help="index build: time one k-means iteration (assignment + update) over the workload's points")
