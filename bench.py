@@ -71,6 +71,18 @@ def parse():
     return p.parse_args()
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the oracle baseline's record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -246,7 +258,7 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64" if args.lut_mode == 0 else "u8",
             "data": "synthetic (seeded Gaussian mixture, GloVe-shaped)", "config": config_dict(w, args),
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": oracle.max_threads(), "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"{S} of {w.nq} queries per step, {len(times)} steps"},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -399,7 +411,7 @@ def run_ours(args):
             import oracle
             orc = oracle.OracleIndex(ix.numpy())
             rate, done, el, cores = oracle_rate(orc, Q, w, mode, args.cpu_seconds)
-            line["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            line["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                                     "sample": f"{done} queries of the batch in {el:.1f} s"}
         print(json.dumps(line), flush=True)
     index.close()
@@ -528,7 +540,7 @@ def run_encode(args):
             "roofline": {"bound": "alu", "achieved": ops / (ms * 1e-3) / 1e12, "peak": peak / 1e12,
                          "unit": "Tops/s (fp64)", "frac": ops / (ms * 1e-3) / peak, "traffic": None,
                          "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 lanes x {mhz:.0f} MHz (nominal rate)"},
-            "cpu_baseline": {"value": ns / ot, "unit": "points/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": ns / ot, "unit": "points/s", "cores": oracle.max_threads(), "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"first {ns} points"},
             "oracle_match_on_sample": same, "clocks": clk.summary(), "gpu_launches": args.steps + args.warmup + 1}
     print(json.dumps(line), flush=True)
@@ -585,7 +597,7 @@ def run_kmeans(args):
                          "traffic": None,
                          "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 lanes x {mhz:.0f} MHz (nominal rate)"},
             "cpu_baseline": {"value": ns / ot, "unit": "points/s (assignment)", "cores": oracle.max_threads(),
-                             "kind": "oracle", "sample": f"first {ns} points"},
+                             "kind": "oracle", "cpu_model": cpu_model(), "sample": f"first {ns} points"},
             "oracle_match_on_sample": same, "clocks": clk.summary(), "gpu_launches": 2 * (args.steps + args.warmup)}
     print(json.dumps(line), flush=True)
 
