@@ -58,6 +58,17 @@ def test_inspect_bf16_and_no_reorder_copy(tmp_path, arrays):
     assert inspect(str(tmp_path / "n"))["reorder_dtype"] is None
 
 
+def test_inspect_reads_format_2_headers(tmp_path, arrays):
+    # numpy writes format 2.0 (4-byte header length) when asked; the reader takes both
+    from mips_ivf_centroid_b200 import inspect
+    w, arr = arrays
+    _write(tmp_path, arr)
+    for k in ("centroids", "codes", "reorder_vecs"):
+        with open(os.path.join(tmp_path, f"{k}.npy"), "wb") as f:
+            np.lib.format.write_array(f, arr[k], version=(2, 0))
+    assert inspect(str(tmp_path))["n"] == 3000
+
+
 def test_inspect_residual_line(tmp_path, arrays):
     from mips_ivf_centroid_b200 import inspect
     w, arr = arrays
