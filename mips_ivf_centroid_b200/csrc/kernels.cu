@@ -920,8 +920,10 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
             }
             const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
             const int n = __popc(m);
-            if (nseg + n > kThresholdSegs) {
-                // keep the first kThresholdSegs segments only
+            if (nseg + n >= kThresholdSegs) {
+                // the table is full: keep its first kThresholdSegs segments and
+                // stop.  nseg < kThresholdSegs on entry (a full table ends both
+                // loops), so some lane holds index kThresholdSegs - 1 here
                 const unsigned lm = __ballot_sync(0xFFFFFFFFu, cnt > 0 && idx == kThresholdSegs - 1);
                 taken += __shfl_sync(0xFFFFFFFFu, incl, __ffs(lm) - 1);   // end of the last kept segment
                 nseg = kThresholdSegs;

@@ -53,6 +53,9 @@ def _workload(name):
                                             training_sample_size=40_000),
         "glove-mini-residual": W["glove"].scaled(n=60_000, num_leaves=300, num_leaves_to_search=24, nq=300,
                                                  n_means=120, training_sample_size=60_000, residual=True),
+        "tiny-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=2000, num_leaves_to_search=1500, nq=32,
+                                         n_means=10, training_sample_size=3_000, code_loss="l2",
+                                         threshold_T=None),
         "small-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=600, num_leaves_to_search=2, nq=64,
                                           n_means=10, training_sample_size=3_000, code_loss="l2",
                                           threshold_T=None),
@@ -205,6 +208,14 @@ def test_residual_codes_reject_uint8_tables(Index):
         index.search(torch.from_numpy(Q[:4]).cuda(), 10, 24, 100, 1)
     assert e.value.status == 2
     index.close()
+
+
+@pytest.mark.parametrize("lut_mode", [0, 1])
+def test_threshold_sample_over_hundreds_of_leaves(Index, lut_mode):
+    # leaves of about 1.5 points, none empty: the threshold sample's segment
+    # table fills (256 leaves, exactly at a warp round's end) before the
+    # sample does, and the bound comes from that subset alone
+    compare(Index, "tiny-leaves", 10, 1500, 100, lut_mode)
 
 
 def test_all_leaves(Index):
