@@ -218,6 +218,51 @@ def test_threshold_sample_over_hundreds_of_leaves(Index, lut_mode):
     compare(Index, "tiny-leaves", 10, 1500, 100, lut_mode)
 
 
+def _overflow_case():
+    """Two leaves.  The better one by centroid score holds 2,000 points whose
+    codes are all low (centers 0-3); the other holds 20,000 points whose codes
+    are all high (centers 8-15), with every center a positive multiple of the
+    all-ones vector and every query positive.  The filter bound comes from a
+    sample of the first leaf, so every point of the second reaches it: about
+    20,000 kept against a buffer of 8,192 (R = 100), and every query is
+    rescanned with the bound taken from its stored candidates."""
+    from mips_ivf_centroid_b200.datagen import IndexArrays
+    key = "overflow"
+    if key in _cache:
+        return _cache[key]
+    rng = np.random.default_rng(20261202)
+    d, n0, n1, nq = 16, 2_000, 20_000, 16
+    n = n0 + n1
+    w = datagen.WORKLOADS["glove"].scaled(n=n, d=d, num_leaves=2, num_leaves_to_search=2, nq=nq,
+                                          n_means=1, training_sample_size=n)
+    B = d // w.dims_per_block
+    nib = np.concatenate([rng.integers(0, 4, (n0, B)), rng.integers(8, 16, (n1, B))]).astype(np.uint8)
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    codebook = np.broadcast_to((np.arange(16, dtype=np.float32) / 15)[None, :, None],
+                               (B, 16, w.dims_per_block)).copy()
+    centroids = np.stack([np.full(d, 10.0, np.float32), np.ones(d, np.float32)])
+    X = rng.standard_normal((n, d)).astype(np.float32)
+    Q = rng.uniform(0.5, 1.5, (nq, d)).astype(np.float32)
+    slot_ids = rng.permutation(n).astype(np.int32)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    ix = IndexArrays(workload=w, centroids=t(centroids), leaf_offsets=t(np.array([0, n0, n], np.int64)),
+                     slot_ids=t(slot_ids), codes=t(codes), codebook=t(codebook), reorder_vecs=t(X[slot_ids]))
+    _cache[key] = (w, X, Q, ix, ix.numpy())
+    return _cache[key]
+
+
+@pytest.mark.parametrize("lut_mode", [0, 1])
+def test_candidate_buffer_overflow_rescans(Index, lut_mode):
+    w, X, Q, ix, arr = _overflow_case()
+    index = Index(ix)
+    _, _, tr = index.search(torch.from_numpy(Q).cuda(), 10, 2, 100, lut_mode, trace=True)
+    index.sync_status()
+    index.close()
+    assert int(tr["rescans"][0]) == w.nq
+    assert (tr["passed"].cpu() > 8192).all()
+    compare(Index, "overflow", 10, 2, 100, lut_mode, max_leaf_mismatch=0.0, max_cand_mismatch=0.0)
+
+
 def test_all_leaves(Index):
     compare(Index, "glove-mini", 10, 300, 100, 0, qsel=slice(0, 40))
 
