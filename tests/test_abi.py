@@ -87,3 +87,11 @@ def test_library_is_sm100a_only():
     log = open(os.path.join(ahbuild.BUILD, "ptxas.log")).read()
     assert "sm_100a" in log
     assert "compute_100a,code=sm_100a" in " ".join(ahbuild.NVCC_FLAGS)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # the package has no other way to search: without the CUDA library it raises
+    with pytest.raises(ahindex.AhError) as e:
+        ahindex.load_library(str(tmp_path / "libah.so"))
+    assert e.value.status == 4
+    assert "not built" in str(e.value)
