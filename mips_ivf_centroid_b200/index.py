@@ -112,6 +112,47 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _need(t, name: str, dtype, shape, device=None):
+    """AhError(1) unless ``t`` is a contiguous ``dtype`` tensor of ``shape``
+    (None matches any extent), on ``device`` when one is given.  The library
+    receives pointers and sizes only, so extents are checked here."""
+    ok = (isinstance(t, torch.Tensor) and t.dtype == dtype and t.is_contiguous() and t.dim() == len(shape)
+          and all(e is None or t.shape[i] == e for i, e in enumerate(shape))
+          and (device is None or t.device == device))
+    if not ok:
+        want = "[" + ", ".join("*" if e is None else str(e) for e in shape) + "]"
+        raise AhError(1, f"{name}: need contiguous {dtype} {want}" + ("" if device is None else f" on {device}"))
+
+
+def _check_index_arrays(arrays):
+    """Extents of the index arrays against one another: centroids [NL, d],
+    leaf_offsets [NL + 1], slot_ids [n], codes [n, B / 2], codebook [B, 16,
+    dpb] with B * dpb = d and B even, reorder_vecs [n, d] or None.  Returns
+    (n, d, NL, dpb)."""
+    c, cb = arrays.centroids, arrays.codebook
+    if not isinstance(c, torch.Tensor) or c.dim() != 2:
+        raise AhError(1, "centroids: need [num_leaves, d]")
+    nl, d = c.shape
+    if not isinstance(cb, torch.Tensor) or cb.dim() != 3 or cb.shape[1] != 16 or cb.shape[0] * cb.shape[2] != d:
+        raise AhError(1, "codebook: need [d / dims_per_block, 16, dims_per_block]")
+    B, dpb = cb.shape[0], cb.shape[2]
+    if B % 2:
+        raise AhError(1, "codebook: need an even number of blocks (d a multiple of 2 * dims_per_block)")
+    dev = c.device
+    _need(c, "centroids", torch.float32, (nl, d))
+    _need(arrays.leaf_offsets, "leaf_offsets", torch.int64, (nl + 1,), dev)
+    _need(arrays.slot_ids, "slot_ids", torch.int32, (None,), dev)
+    n = arrays.slot_ids.shape[0]
+    _need(arrays.codes, "codes", torch.uint8, (n, B // 2), dev)
+    _need(cb, "codebook", torch.float32, (B, 16, dpb), dev)
+    rv = arrays.reorder_vecs
+    if rv is not None:
+        if not isinstance(rv, torch.Tensor) or rv.dtype not in (torch.float32, torch.bfloat16):
+            raise AhError(1, "reorder_vecs: need float32 or bfloat16")
+        _need(rv, "reorder_vecs", rv.dtype, (n, d), dev)
+    return n, d, nl, dpb
+
+
 def encode(X: torch.Tensor, codebook: torch.Tensor, T: float, passes: int = 10, stream=None,
            out: Optional[torch.Tensor] = None, passes_used: Optional[torch.Tensor] = None):
     """Anisotropic codes of the rows of X (index build, ``ah_encode``).
@@ -131,8 +172,10 @@ def encode(X: torch.Tensor, codebook: torch.Tensor, T: float, passes: int = 10, 
         raise AhError(1, "codebook: need [d / dims_per_block, 16, dims_per_block]")
     if out is None:
         out = torch.empty((n, B // 2), dtype=torch.uint8, device=X.device)
+    _need(out, "out", torch.uint8, (n, B // 2), X.device)
     if passes_used is None:
         passes_used = torch.empty((n,), dtype=torch.int32, device=X.device)
+    _need(passes_used, "passes_used", torch.int32, (n,), X.device)
     with torch.cuda.device(X.device):
         _check(lib, lib.ah_encode(_ptr(X), n, d, dpb, _ptr(codebook), float(T), int(passes), _ptr(out),
                                   _ptr(passes_used), _stream(stream)))
@@ -171,6 +214,8 @@ def kmeans_update(X: torch.Tensor, assign: torch.Tensor, C_old: torch.Tensor, st
             or assign.device != X.device or not assign.is_contiguous():
         raise AhError(1, "assign: need contiguous int32 [n] on X's device")
     n, d = X.shape
+    if C_old.shape[1] != d:
+        raise AhError(1, "C_old: need [nl, d] with X's d")
     nl = C_old.shape[0]
     C_new = torch.empty_like(C_old)
     counts = torch.empty((nl,), dtype=torch.int64, device=X.device)
@@ -192,6 +237,10 @@ def merge_shards(cand_ids: torch.Tensor, cand_approx: torch.Tensor, cand_exact: 
     if cand_ids.dtype != torch.int32 or cand_ids.dim() != 3 or not cand_ids.is_contiguous() \
             or cand_ids.device.type != "cuda":
         raise AhError(1, "cand_ids: need contiguous int32 [G, nq, R] on a CUDA device")
+    if cand_approx is None:
+        raise AhError(1, "cand_approx: required")
+    if k < 1:
+        raise AhError(1, "need k >= 1")
     for name, t in (("cand_approx", cand_approx), ("cand_exact", cand_exact)):
         if t is not None and (t.dtype != torch.float32 or t.shape != cand_ids.shape or not t.is_contiguous()
                               or t.device != cand_ids.device):
@@ -242,6 +291,7 @@ class Index:
         rv = arrays.reorder_vecs
         if rv is not None and (not rv.is_contiguous() or rv.device != dev or rv.dtype not in (torch.float32, torch.bfloat16)):
             raise AhError(1, "reorder_vecs: need contiguous float32/bfloat16 on the index device")
+        _check_index_arrays(arrays)
         self.device = dev
         self.n = arrays.slot_ids.shape[0]
         self.d = c.shape[1]
@@ -297,6 +347,8 @@ class Index:
         if q.device != self.device or q.dtype != torch.float32 or not q.is_contiguous() or q.dim() != 2 \
                 or q.shape[1] != self.d:
             raise AhError(1, f"queries: need contiguous float32 [nq, {self.d}] on {self.device}")
+        if k < 1 or num_leaves_to_search < 1 or reorder_num < 0:
+            raise AhError(1, "need k >= 1, num_leaves_to_search >= 1, reorder_num >= 0")
         nq = q.shape[0]
         ids = torch.empty((nq, k), dtype=torch.int32, device=self.device)
         scores = torch.empty((nq, k), dtype=torch.float32, device=self.device)
@@ -329,13 +381,19 @@ class Index:
         host (ids, scores).  The copies in and out happen inside the call."""
         if isinstance(queries, np.ndarray):
             queries = torch.from_numpy(np.ascontiguousarray(queries, dtype=np.float32))
-        if queries.device.type != "cpu" or queries.dtype != torch.float32 or not queries.is_contiguous():
-            raise AhError(1, "queries: need a contiguous float32 host tensor")
+        if queries.device.type != "cpu" or queries.dtype != torch.float32 or not queries.is_contiguous() \
+                or queries.dim() != 2 or queries.shape[1] != self.d:
+            raise AhError(1, f"queries: need a contiguous float32 host tensor [nq, {self.d}]")
+        if k < 1:
+            raise AhError(1, "need k >= 1")
         nq = queries.shape[0]
+        cpu = torch.device("cpu")
         if out_ids is None:
             out_ids = torch.empty((nq, k), dtype=torch.int32, pin_memory=queries.is_pinned())
+        _need(out_ids, "out_ids", torch.int32, (nq, k), cpu)
         if out_scores is None:
             out_scores = torch.empty((nq, k), dtype=torch.float32, pin_memory=queries.is_pinned())
+        _need(out_scores, "out_scores", torch.float32, (nq, k), cpu)
         with torch.cuda.device(self.device):
             _check(self._lib, self._lib.ah_search_host(self._h, _ptr(queries), nq, k, num_leaves_to_search,
                                                        reorder_num, lut_mode, _ptr(out_ids), _ptr(out_scores),
@@ -390,6 +448,12 @@ class Index:
         """Partition stage into caller-provided outputs, with no device
         allocation anywhere on the call path (see ah_search_leaves_noalloc in
         include/ah.h for the scratch limit and the sharing rules)."""
+        _need(queries, "queries", torch.float32, (None, self.d), self.device)
+        nq, L = queries.shape[0], num_leaves_to_search
+        if L < 1:
+            raise AhError(1, "need num_leaves_to_search >= 1")
+        _need(out_leaf_ids, "out_leaf_ids", torch.int32, (nq, L), self.device)
+        _need(out_leaf_scores, "out_leaf_scores", torch.float32, (nq, L), self.device)
         with torch.cuda.device(self.device):
             _check(self._lib, self._lib.ah_search_leaves_noalloc(
                 self._h, _ptr(queries), queries.shape[0], num_leaves_to_search, _ptr(out_leaf_ids),
