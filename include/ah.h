@@ -23,6 +23,11 @@
  *  - Status codes only: no exceptions cross the ABI, nothing calls exit/abort.
  *  - Device pointers are CUDA device memory on the current device; the library
  *    never frees memory it did not allocate.
+ *  - Every array must hold at least the elements that its documented shape
+ *    and the sizes passed with it give.  The library checks the sizes, but it
+ *    cannot see the allocation behind a pointer: a shorter buffer is read or
+ *    written out of bounds.  (The Python binding checks tensor extents before
+ *    it calls.)
  *  - Work is enqueued on the given stream (a cudaStream_t passed as void*; NULL
  *    means the legacy default stream) and is asynchronous unless stated
  *    otherwise: outputs are valid once that stream has been synchronised.
