@@ -59,7 +59,7 @@ extern "C" {
 typedef enum {
     AH_OK = 0,
     AH_ERR_INVALID_ARG = 1,  /* a null pointer, an out-of-range size or knob   */
-    AH_ERR_UNSUPPORTED = 2,  /* valid request beyond this build's limits       */
+    AH_ERR_UNSUPPORTED = 2,  /* valid request beyond the library's AH_MAX_*    */
     AH_ERR_OOM = 3,          /* device allocation failed                       */
     AH_ERR_CUDA = 4,         /* a CUDA runtime call failed                     */
     AH_ERR_DEVICE = 5,       /* a kernel reported an error (see ah_sync_status) */
