@@ -77,6 +77,11 @@ enum { AH_LUT_F32 = 0, AH_LUT_U8 = 1 };
 #define AH_MAX_LEAVES_SEARCHED 4096
 #define AH_MAX_D 8192
 #define AH_MAX_BLOCKS 1024       /* d / dims_per_block                         */
+/* A search with fp32 tables (AH_LUT_F32) keeps eight queries' tables in one
+ * scan CTA's shared memory when B = d / dims_per_block is above 400: 512 * B
+ * bytes, which the 227 KB per-CTA limit of a B200 bounds at B <= 453.  Above
+ * that the scan launch is refused and ah_search returns AH_ERR_CUDA; uint8
+ * tables (AH_LUT_U8) serve every B up to AH_MAX_BLOCKS. */
 
 /*
  * Index arrays, all in device memory and BORROWED: they must stay allocated
