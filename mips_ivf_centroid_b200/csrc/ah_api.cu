@@ -29,6 +29,10 @@ ah_status fail(ah_status s, const std::string& msg) {
 
 ah_status cuda_fail(cudaError_t e, const char* what) {
     g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    // The status carries the error; clear the runtime's per-thread last error
+    // so that a non-sticky failure (a refused launch attribute, an allocation)
+    // is not reported again by the caller's or the next call's error check.
+    (void)cudaGetLastError();
     return e == cudaErrorMemoryAllocation ? AH_ERR_OOM : AH_ERR_CUDA;
 }
 
