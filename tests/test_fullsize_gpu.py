@@ -63,7 +63,9 @@ def test_bigann_full(Index):
     # integer data: centroid and exact scores are integers below 2^24, exact in fp32
     w, Q, ix, arr = _build("bigann")
     index = Index(ix)
-    sel = np.arange(0, w.nq, 250)                  # 40 of the 10,000 queries
+    # 40 of the 10,000 queries, and the last one: 10,000 = 78 x 128 + 16, so it
+    # sits in the partial row of 128-query centroid-score tiles
+    sel = np.r_[np.arange(0, w.nq, 250), w.nq - 1]
     r = compare_search(index, arr, Q, w.k, w.num_leaves_to_search, w.reorder_num, 0, qsel=sel,
                        max_leaf_mismatch=0.0)
     same = (r["ids"] == r["oracle"]["ids"]).all(axis=1)
