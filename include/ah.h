@@ -4,13 +4,15 @@
  * The search path is the one the ScaNN blog post describes in "Three stages of
  * a search" (ScaNN: Anisotropic Vector Quantization for Maximum Inner Product
  * Search):
- *   partitioning  -> the query scores every centroid and keeps the best
- *                    num_leaves_to_search leaves;
+ *   partitioning  -> q . c for every centroid c; the num_leaves_to_search
+ *                    highest-scoring leaves are the ones searched;
  *   asymmetric hashing (AH) -> a per-query lookup table of q . center for each
- *                    block's 16 centers; a point's approximate score is the sum
- *                    of its table entries, read through its 4-bit codes;
- *   reordering    -> the best few hundred candidates are rescored with exact
- *                    dot products, and the best k are returned.
+ *                    block's 16 centers; each point's 4-bit codes pick one
+ *                    entry per block, and those entries add up to its
+ *                    approximate score;
+ *   reordering    -> exact dot products replace the approximate scores of
+ *                    the top candidates (a few hundred), and the best k by
+ *                    exact score are returned.
  * The search-time knobs follow the post's "Using the library" section
  * (search_batched with leaves_to_search and pre_reorder_num_neighbors, and
  * final_num_neighbors).  Besides the search the library provides the steps

@@ -67,7 +67,8 @@ def test_leaf_ties_go_to_lower_id():
 
 
 def test_approximate_score_is_dot_with_reconstruction():
-    # "a point's approximate score is the sum of its table entries" = q . x~
+    # adding up the table entries a point's codes select gives q . x~ for its
+    # reconstruction x~ ("Three stages of a search")
     w, X, Q, ix, arr = _mini(aniso=True)
     orc = OracleIndex(arr)
     out = orc.search(Q, w.k, w.num_leaves_to_search, w.reorder_num)
