@@ -106,7 +106,7 @@ enum { AH_LUT_F32 = 0, AH_LUT_U8 = 1 };
  *                   reorder_num = 0
  *   residual        0: codes quantise each point; 1: codes quantise the
  *                   point minus its leaf's centroid (one codebook for all
- *                   leaves), so a point's approximate score is the query's
+ *                   leaves), so the approximate score of a point is the query's
  *                   centroid score of that leaf plus its table sum (added
  *                   after the sum, in fp32).  Residual indexes support fp32
  *                   tables only (AH_LUT_U8 is AH_ERR_UNSUPPORTED).

@@ -16,16 +16,16 @@ from oracle import avq
 def test_eta_closed_forms():
     # unit norm: eta = (d-1) T^2 / (1 - T^2)
     # d = 100, T = 1/5:  99 * (1/25) / (24/25) = 99/24 = 4.125
-    assert avq.eta_for(100, 0.2) == pytest.approx(float(Fraction(99, 24)), rel=1e-15)
+    assert avq.eta_ratio(100, 0.2) == pytest.approx(float(Fraction(99, 24)), rel=1e-15)
     # d = 1536, T = 1/20: 1535 * (1/400) / (399/400) = 1535/399
-    assert avq.eta_for(1536, 0.05) == pytest.approx(float(Fraction(1535, 399)), rel=1e-15)
+    assert avq.eta_ratio(1536, 0.05) == pytest.approx(float(Fraction(1535, 399)), rel=1e-15)
     # the generator's workloads carry the same values
     assert datagen.WORKLOADS["glove"].eta == pytest.approx(99 / 24, rel=1e-15)
     assert datagen.WORKLOADS["openai"].eta == pytest.approx(1535 / 399, rel=1e-15)
     # non-unit norm: T/||x|| enters squared
-    assert avq.eta_for(11, 1.0, norm=2.0) == pytest.approx(10 * 0.25 / 0.75, rel=1e-15)
+    assert avq.eta_ratio(11, 1.0, norm=2.0) == pytest.approx(10 * 0.25 / 0.75, rel=1e-15)
     with pytest.raises(ValueError):
-        avq.eta_for(10, 1.0, norm=1.0)
+        avq.eta_ratio(10, 1.0, norm=1.0)
 
 
 def test_loss_equals_weighted_parallel_plus_perpendicular():
@@ -69,15 +69,15 @@ def test_center_update_minimises_member_loss():
     assert np.linalg.norm(c - m.mean(0)) > 1e-6
 
 
-def test_train_avq_at_eta_one_is_lloyd():
+def test_anisotropic_kmeans_at_eta_one_is_lloyd():
     # eta = 1 when T^2 = 1/d for unit data: one iteration equals one k-means step.
     rng = np.random.default_rng(3)
     X = rng.standard_normal((120, 4))
     X /= np.linalg.norm(X, axis=1, keepdims=True)
     T = 1 / np.sqrt(4)
-    assert avq.eta_for(4, T) == pytest.approx(1.0)
-    C, a = avq.train_avq(X, 5, T, iters=1, seed=7)
-    C0 = X[np.random.default_rng(7).choice(120, 5, replace=False)]
+    assert avq.eta_ratio(4, T) == pytest.approx(1.0)
+    C, a = avq.anisotropic_kmeans(X, 5, T, iters=1, seed=7)
+    C0 = X[np.random.default_rng(7).permutation(120)[:5]]     # the documented initial centers
     d2 = ((X[:, None, :] - C0[None]) ** 2).sum(-1)
     a_ref = d2.argmin(1)
     np.testing.assert_array_equal(a, a_ref)

@@ -6,7 +6,7 @@ Checked against things other than the function itself:
 * One live block (the other block's 16 centers identical, so its choice
   changes nothing): the descent must reach the exhaustive argmin of the
   anisotropic loss over that block's 16 centers, with the loss computed by
-  ``avq.anisotropic_loss`` and eta by ``avq.eta_for`` (pinned in
+  ``avq.anisotropic_loss`` and eta by ``avq.eta_ratio`` (pinned in
   test_avq_pins.py) from each point's own norm.
 * Converged codes are a coordinate-wise minimum: no single-block change
   lowers the independently computed loss.
@@ -63,7 +63,7 @@ def test_single_live_block_reaches_exhaustive_argmin():
     X, norms = X[keep], norms[keep]
     codes, used = oracle.encode(X, cb, T=T, passes=10)
     got = _unpack(codes, 2)
-    eta = avq.eta_for(d, T, norms)
+    eta = avq.eta_ratio(d, T, norms)
     losses = np.empty((X.shape[0], 16))
     for j in range(16):
         xt = _recon(cb, np.stack([np.full(X.shape[0], j), got[:, 1]], axis=1))
@@ -85,7 +85,7 @@ def test_converged_codes_are_coordinatewise_minima(dpb):
     codes, used = oracle.encode(X, cb, T=T, passes=100)
     assert (used < 100).all()          # every point converged
     got = _unpack(codes, B)
-    eta = avq.eta_for(d, T, np.linalg.norm(X.astype(np.float64), axis=1))
+    eta = avq.eta_ratio(d, T, np.linalg.norm(X.astype(np.float64), axis=1))
     base = avq.anisotropic_loss(X, _recon(cb, got), eta)
     for b in range(B):
         for j in range(16):
