@@ -81,9 +81,10 @@ enum { AH_LUT_F32 = 0, AH_LUT_U8 = 1 };
 #define AH_MAX_BLOCKS 1024       /* d / dims_per_block                         */
 /* A search with fp32 tables (AH_LUT_F32) keeps eight queries' tables in one
  * scan CTA's shared memory when B = d / dims_per_block is above 400: 512 * B
- * bytes, which the 227 KB per-CTA limit of a B200 bounds at B <= 453.  Above
- * that the scan launch is refused and ah_search returns AH_ERR_CUDA; uint8
- * tables (AH_LUT_U8) serve every B up to AH_MAX_BLOCKS. */
+ * bytes, which the 227 KB per-CTA limit of a B200 bounds at B <= 452 (with
+ * 1 KB kept for the kernel's own arrays).  Above that a search with fp32
+ * tables returns AH_ERR_UNSUPPORTED before any work is enqueued; uint8 tables
+ * (AH_LUT_U8) serve every B up to AH_MAX_BLOCKS. */
 
 /*
  * Index arrays, all in device memory and BORROWED: they must stay allocated
@@ -160,9 +161,11 @@ AH_API ah_status ah_build_index_views(const ah_index_views *views, void *cuda_st
  *   out_ids      int32 [nq][k], device
  *   out_scores   float [nq][k], device: exact fp32 dot products when
  *                reorder_num > 0, otherwise approximate scores
- * Errors: AH_ERR_INVALID_ARG, AH_ERR_UNSUPPORTED, AH_ERR_OOM (workspace
- * growth), AH_ERR_CUDA (launch failure).  Device-side errors of this call are
- * reported by a later ah_sync_status().
+ * Errors: AH_ERR_INVALID_ARG, AH_ERR_UNSUPPORTED (a size above an AH_MAX_*
+ * limit; uint8 tables with residual codes; fp32 tables beyond B = 452, see
+ * AH_MAX_BLOCKS), AH_ERR_OOM (workspace growth), AH_ERR_CUDA (launch
+ * failure).  Device-side errors of this call are reported by a later
+ * ah_sync_status().
  */
 AH_API ah_status ah_search(ah_index *ix, const float *queries, int32_t nq, int32_t k,
                     int32_t num_leaves_to_search, int32_t reorder_num, int32_t lut_mode,

@@ -201,6 +201,9 @@ ah_status validate_search(ah_index* ix, const void* queries, int32_t nq, int32_t
     if (lut_mode != AH_LUT_F32 && lut_mode != AH_LUT_U8) return fail(AH_ERR_INVALID_ARG, "unknown lut_mode");
     if (lut_mode == AH_LUT_U8 && ix->views.residual)
         return fail(AH_ERR_UNSUPPORTED, "uint8 tables need codes of the points, not residuals");
+    if (ah::scan_table_bytes(ix->dix, lut_mode) + 1024 > ah::kMaxSmemPerCta)
+        return fail(AH_ERR_UNSUPPORTED, "a query group's fp32 tables exceed the scan's shared memory at this many "
+                                        "blocks (d / dims_per_block above 452); use uint8 tables");
     const int64_t per_query_cand = static_cast<int64_t>(cap_for(std::max(reorder_num, k)));
     if (static_cast<int64_t>(nq) * per_query_cand > (int64_t(1) << 40)) return fail(AH_ERR_UNSUPPORTED, "batch too large");
     return AH_OK;

@@ -1394,6 +1394,12 @@ int scan_group(const DeviceIndex& ix, int lut_mode) {
     return g;
 }
 
+size_t scan_table_bytes(const DeviceIndex& ix, int lut_mode) {
+    int nt, g;
+    scan_shape(ix, lut_mode, &nt, &g);
+    return static_cast<size_t>(ix.B) * g * kCenters * (lut_mode == 0 ? 4 : 1);
+}
+
 template <int MODE, int NT, int GMAX, bool RES>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {

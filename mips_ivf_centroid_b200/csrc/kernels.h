@@ -117,6 +117,10 @@ cudaError_t launch_redo_scan(const DeviceIndex& ix, const SearchArgs& a, const S
                              int num_sms, cudaStream_t s);
 
 int scan_group(const DeviceIndex& ix, int lut_mode);
+// Shared memory the scan needs for one query group's tables (its launch adds
+// at most the leaf item offsets when they fit, and 144 B of static arrays).
+size_t scan_table_bytes(const DeviceIndex& ix, int lut_mode);
+constexpr size_t kMaxSmemPerCta = 227 * 1024;   // sm_100 opt-in shared memory per CTA
 size_t finish_smem_bytes(int R, int d);
 
 // anisotropic code assignment (encode.cu)
