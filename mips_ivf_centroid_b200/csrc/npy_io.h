@@ -136,6 +136,14 @@ inline std::string read_header(const char* path, Header* out) {
         }
         out->shape.push_back(v);
     }
+    // element count and bytes within 2^40 each, so the length check below
+    // cannot overflow
+    int64_t elems = 1;
+    for (int64_t v : out->shape) {
+        if (v != 0 && elems > (int64_t(1) << 40) / v) return "shape too large";
+        elems *= v;
+    }
+    if (elems > (int64_t(1) << 40) / item_size(out->descr)) return "shape too large";
     out->data_offset = hstart + hlen;
     const int64_t need = out->data_offset + count(out->shape) * item_size(out->descr);
     if (out->file_bytes < need) return "file shorter than its shape";

@@ -82,7 +82,7 @@ def test_inspect_residual_line(tmp_path, arrays):
 
 
 @pytest.mark.parametrize("case", ["missing", "dtype", "offsets", "codes", "truncated", "fortran", "meta",
-                                  "bf16_as_f32", "codebook"])
+                                  "bf16_as_f32", "codebook", "huge_shape"])
 def test_inspect_rejects_malformed(tmp_path, arrays, case):
     from mips_ivf_centroid_b200 import inspect
     w, arr = arrays
@@ -109,9 +109,18 @@ def test_inspect_rejects_malformed(tmp_path, arrays, case):
         p.write_bytes(data[:-100])
     elif case == "meta":
         (tmp_path / "ah_index.txt").write_text("something else\n")
+    elif case == "huge_shape":
+        # 2^33 x 2^33 elements: the element count wraps to 0 in int64, so only
+        # a bound on the product keeps the length check meaningful
+        with open(tmp_path / "reorder_vecs.npy", "wb") as f:
+            np.lib.format.write_array_header_1_0(f, {"descr": "<f4", "fortran_order": False,
+                                                     "shape": (2 ** 33, 2 ** 33)})
+            f.write(b"\0" * 64)
     st, msg = _status(lambda: inspect(str(tmp_path)))
     assert st == 1, msg
+    if case == "huge_shape":
+        assert "shape too large" in msg, msg
     want = {"missing": "codes.npy", "dtype": "slot_ids.npy", "offsets": "leaf_offsets.npy", "codes": "codes.npy",
             "truncated": "reorder_vecs.npy", "fortran": "centroids.npy", "meta": "ah_index.txt",
-            "bf16_as_f32": "reorder_vecs.npy", "codebook": "codebook.npy"}[case]
+            "bf16_as_f32": "reorder_vecs.npy", "codebook": "codebook.npy", "huge_shape": "reorder_vecs.npy"}[case]
     assert want in msg, msg
