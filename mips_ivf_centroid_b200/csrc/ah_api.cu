@@ -882,7 +882,7 @@ ah_status ah_load(const char* dir, void* cuda_stream, ah_index** out) {
         cudaError_t e = cudaMalloc(&dev[i], static_cast<size_t>(std::max<int64_t>(bytes, 1)));
         if (e != cudaSuccess) {
             release();
-            return e == cudaErrorMemoryAllocation ? fail(AH_ERR_OOM, "index arrays") : cuda_fail(e, "index arrays");
+            return cuda_fail(e, "index arrays");      // AH_ERR_OOM for an allocation failure
         }
         total += static_cast<size_t>(bytes);
         const std::string p = path_in(dir, kIndexFiles[i]);
