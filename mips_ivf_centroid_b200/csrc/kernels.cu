@@ -1366,10 +1366,12 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
 }
 
 // Scan CTA shape: threads per CTA and queries per group.  Narrow tables
-// (a full group's tables within 64 KB): 256 threads, groups of 8 (fp32) or
-// 16 (uint8) queries, several CTAs per SM.  Wide tables: two CTAs of 512
-// threads per SM with half-size groups, so one CTA's table staging and
-// item-end barrier overlap the other's scanning.
+// (a full group's tables within 64 KB): 256 threads, groups of 8 queries
+// (fp32 and uint8), several CTAs per SM.  Wide tables (half a group within
+// 100 KB): two CTAs of 512 threads per SM with half-size groups, so one
+// CTA's table staging and item-end barrier overlap the other's scanning.
+// Wider fp32 tables (B 401-452): one CTA of 1,024 threads, groups of 8; the
+// search refuses fp32 tables beyond that.
 #ifndef AH_WIDE_SPLIT
 #define AH_WIDE_SPLIT 1
 #endif
