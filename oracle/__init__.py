@@ -79,6 +79,10 @@ def _load():
         lib.orc_search.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                    P, P, P, P, P, P, P, P, P]
+        lib.orc_search_leaves.restype = ctypes.c_int
+        lib.orc_search_leaves.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P,
+                                          ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                          P, P, P, P, P, P, P]
         lib.orc_centroid_scores.argtypes = [P, P, P]
         lib.orc_point_scores.argtypes = [P, P, ctypes.c_int64, P, P, P]
         lib.orc_u8_table.argtypes = [P, P, P, P, P]
@@ -154,6 +158,32 @@ class OracleIndex:
                             _ptr(out["ids"]), _ptr(out["scores"]), _ptr(g("leaves")),
                             _ptr(g("leaf_scores")), _ptr(g("cand_ids")), _ptr(g("cand_scores")),
                             _ptr(g("cand_sums")), _ptr(g("ncand")), _ptr(g("scanned")))
+        if rc != 0:
+            raise ValueError("oracle: invalid search arguments")
+        return out
+
+    def search_leaves(self, Q: np.ndarray, leaves: np.ndarray, k: int, reorder_num: int, lut_mode: int = 0,
+                      nthreads: int = 0) -> dict:
+        """Steps 2-5 of the search over caller-given leaves [nq, L] (int32,
+        distinct ids per row) instead of each query's own best L; the same
+        arithmetic as ``search``.  Returns ids/scores [nq,k], cand_ids/
+        cand_scores/cand_sums [nq,R], ncand and scanned [nq]."""
+        lib = _load()
+        Q = np.ascontiguousarray(Q, dtype=np.float32)
+        leaves = np.ascontiguousarray(leaves, dtype=np.int32)
+        nq = Q.shape[0]
+        if leaves.ndim != 2 or leaves.shape[0] != nq:
+            raise ValueError("oracle: leaves must be [nq, L]")
+        L = leaves.shape[1]
+        R = max(reorder_num, k)
+        out = {"ids": np.empty((nq, k), np.int32), "scores": np.empty((nq, k), np.float64),
+               "cand_ids": np.empty((nq, R), np.int32), "cand_scores": np.empty((nq, R), np.float64),
+               "cand_sums": np.empty((nq, R), np.uint32), "ncand": np.empty(nq, np.int32),
+               "scanned": np.empty(nq, np.int64)}
+        rc = lib.orc_search_leaves(self.ref, _ptr(Q), nq, k, L, _ptr(leaves), reorder_num, lut_mode, nthreads,
+                                   _ptr(out["ids"]), _ptr(out["scores"]), _ptr(out["cand_ids"]),
+                                   _ptr(out["cand_scores"]), _ptr(out["cand_sums"]), _ptr(out["ncand"]),
+                                   _ptr(out["scanned"]))
         if rc != 0:
             raise ValueError("oracle: invalid search arguments")
         return out

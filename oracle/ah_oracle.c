@@ -193,6 +193,115 @@ static double exact_score(const orc_index *ix, const float *q, int64_t slot) {
 }
 
 /*
+ * Steps 2-5 for one query over a given list of L leaves (the order of the list
+ * does not matter: every point of the listed leaves is scored, then ranked by
+ * (score, id)).  s: the query's fp64 centroid scores (read only for residual
+ * codes).  Outputs as for orc_search, for this query's row (NULL to skip).
+ */
+static void search_in_leaves(const orc_index *ix, const float *q, const double *s, const int32_t *leaf_list,
+                             int32_t L, int32_t k, int32_t R, int32_t reorder_num, int32_t lut_mode,
+                             int32_t *out_ids, double *out_scores, int32_t *out_cand_ids,
+                             double *out_cand_scores, uint32_t *out_cand_sums, int32_t *out_ncand,
+                             int64_t *out_scanned) {
+    const int B = blocks_of(ix);
+
+    /* 2. lookup table */
+    double *lut = NULL;
+    uint8_t *lut8 = NULL;
+    float delta = 0.0f, bias = 0.0f;
+    if (lut_mode == 0) {
+        lut = (double *)malloc(sizeof(double) * (size_t)B * ORC_CENTERS);
+        lut_f64(ix, q, lut);
+    } else {
+        lut8 = (uint8_t *)malloc((size_t)B * ORC_CENTERS);
+        lut_u8(ix, q, lut8, &delta, &bias);
+    }
+
+    /* 3. approximate score of every point in the kept leaves */
+    int64_t total = 0;
+    for (int i = 0; i < L; ++i) {
+        int c = leaf_list[i];
+        total += ix->leaf_offsets[c + 1] - ix->leaf_offsets[c];
+    }
+    orc_item *cand = NULL;
+    orc_uitem *ucand = NULL;
+    if (lut_mode == 0) cand = (orc_item *)malloc(sizeof(orc_item) * (total > 0 ? total : 1));
+    else ucand = (orc_uitem *)malloc(sizeof(orc_uitem) * (total > 0 ? total : 1));
+    int64_t m = 0;
+    for (int i = 0; i < L; ++i) {
+        int c = leaf_list[i];
+        for (int64_t p = ix->leaf_offsets[c]; p < ix->leaf_offsets[c + 1]; ++p, ++m) {
+            if (lut_mode == 0) {
+                /* residual codes: q . x~ = q . centroid + table sum */
+                cand[m].score = ix->residual ? ah_score_f64(ix, lut, p) + s[c] : ah_score_f64(ix, lut, p);
+                cand[m].id = ix->slot_ids[p];
+                cand[m].slot = (int32_t)p;
+            } else {
+                ucand[m].sum = ah_sum_u8(ix, lut8, p);
+                ucand[m].id = ix->slot_ids[p];
+                ucand[m].slot = (int32_t)p;
+            }
+        }
+    }
+    if (out_scanned) *out_scanned = total;
+
+    /* 4. best R by approximate score */
+    if (lut_mode == 0) qsort(cand, total, sizeof(orc_item), by_score_then_id);
+    else qsort(ucand, total, sizeof(orc_uitem), by_sum_then_id);
+    int32_t nc = total < R ? (int32_t)total : R;
+    if (out_ncand) *out_ncand = nc;
+    for (int32_t i = 0; i < R; ++i) {
+        if (i < nc) {
+            if (out_cand_ids) out_cand_ids[i] = lut_mode == 0 ? cand[i].id : ucand[i].id;
+            if (out_cand_scores)
+                out_cand_scores[i] = lut_mode == 0 ? cand[i].score : (double)fmaf(delta, (float)ucand[i].sum, bias);
+            if (out_cand_sums) out_cand_sums[i] = lut_mode == 0 ? 0u : ucand[i].sum;
+        } else {
+            if (out_cand_ids) out_cand_ids[i] = -1;
+            if (out_cand_scores) out_cand_scores[i] = -INFINITY;
+            if (out_cand_sums) out_cand_sums[i] = 0u;
+        }
+    }
+
+    /* 5. reorder (exact rescoring) or pure approximate ranking */
+    orc_item *fin = (orc_item *)malloc(sizeof(orc_item) * (nc > 0 ? nc : 1));
+    for (int32_t i = 0; i < nc; ++i) {
+        int32_t slot = lut_mode == 0 ? cand[i].slot : ucand[i].slot;
+        fin[i].id = ix->slot_ids[slot];
+        fin[i].slot = slot;
+        if (reorder_num > 0) fin[i].score = exact_score(ix, q, slot);
+        else if (lut_mode == 0) fin[i].score = cand[i].score;
+        else fin[i].score = (double)fmaf(delta, (float)ucand[i].sum, bias);
+    }
+    if (reorder_num > 0) qsort(fin, nc, sizeof(orc_item), by_score_then_id);
+    for (int32_t i = 0; i < k; ++i) {
+        if (i < nc) {
+            out_ids[i] = fin[i].id;
+            out_scores[i] = fin[i].score;
+        } else {
+            out_ids[i] = -1;
+            out_scores[i] = -INFINITY;
+        }
+    }
+    free(fin);
+    free(cand);
+    free(ucand);
+    free(lut);
+    free(lut8);
+}
+
+static int bad_search_args(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32_t L,
+                           int32_t reorder_num, int32_t lut_mode, const int32_t *out_ids,
+                           const double *out_scores) {
+    return !ix || !Q || !out_ids || !out_scores || nq < 0 || k <= 0 || L < 1 || L > ix->num_leaves ||
+           reorder_num < 0 || (reorder_num > 0 && reorder_num < k) || (lut_mode != 0 && lut_mode != 1) ||
+           (lut_mode == 1 && ix->residual);
+}
+
+/* Optional per-query output row (NULL stays NULL). */
+#define ORC_ROW(ptr, qi, w) ((ptr) ? (ptr) + (int64_t)(qi) * (w) : NULL)
+
+/*
  * Full search.  Required outputs: out_ids/out_scores [nq][k].  Optional (NULL
  * to skip): out_leaves/out_leaf_scores [nq][L]; out_cand_ids, out_cand_scores,
  * out_cand_sums [nq][R]; out_ncand [nq] (candidates kept, <= R);
@@ -205,11 +314,7 @@ int orc_search(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32
                int32_t *out_leaves, double *out_leaf_scores,
                int32_t *out_cand_ids, double *out_cand_scores, uint32_t *out_cand_sums,
                int32_t *out_ncand, int64_t *out_scanned) {
-    if (!ix || !Q || !out_ids || !out_scores || nq < 0 || k <= 0 || L < 1 ||
-        L > ix->num_leaves || reorder_num < 0 || (reorder_num > 0 && reorder_num < k) ||
-        (lut_mode != 0 && lut_mode != 1) || (lut_mode == 1 && ix->residual))
-        return -1;
-    const int B = blocks_of(ix);
+    if (bad_search_args(ix, Q, nq, k, L, reorder_num, lut_mode, out_ids, out_scores)) return -1;
     const int32_t R = reorder_num > k ? reorder_num : k;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -221,6 +326,7 @@ int orc_search(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32
         /* 1. partition: best L leaves */
         double *s = (double *)malloc(sizeof(double) * ix->num_leaves);
         orc_item *leaves = (orc_item *)malloc(sizeof(orc_item) * ix->num_leaves);
+        int32_t *leaf_list = (int32_t *)malloc(sizeof(int32_t) * L);
         centroid_scores(ix, q, s);
         for (int c = 0; c < ix->num_leaves; ++c) {
             leaves[c].score = s[c];
@@ -228,99 +334,51 @@ int orc_search(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32
             leaves[c].slot = c;
         }
         qsort(leaves, ix->num_leaves, sizeof(orc_item), by_score_then_id);
+        for (int i = 0; i < L; ++i) leaf_list[i] = leaves[i].id;
         if (out_leaves)
             for (int i = 0; i < L; ++i) out_leaves[(int64_t)qi * L + i] = leaves[i].id;
         if (out_leaf_scores)
             for (int i = 0; i < L; ++i) out_leaf_scores[(int64_t)qi * L + i] = leaves[i].score;
 
-        /* 2. lookup table */
-        double *lut = NULL;
-        uint8_t *lut8 = NULL;
-        float delta = 0.0f, bias = 0.0f;
-        if (lut_mode == 0) {
-            lut = (double *)malloc(sizeof(double) * (size_t)B * ORC_CENTERS);
-            lut_f64(ix, q, lut);
-        } else {
-            lut8 = (uint8_t *)malloc((size_t)B * ORC_CENTERS);
-            lut_u8(ix, q, lut8, &delta, &bias);
-        }
-
-        /* 3. approximate score of every point in the kept leaves */
-        int64_t total = 0;
-        for (int i = 0; i < L; ++i) {
-            int c = leaves[i].slot;
-            total += ix->leaf_offsets[c + 1] - ix->leaf_offsets[c];
-        }
-        orc_item *cand = NULL;
-        orc_uitem *ucand = NULL;
-        if (lut_mode == 0) cand = (orc_item *)malloc(sizeof(orc_item) * (total > 0 ? total : 1));
-        else ucand = (orc_uitem *)malloc(sizeof(orc_uitem) * (total > 0 ? total : 1));
-        int64_t m = 0;
-        for (int i = 0; i < L; ++i) {
-            int c = leaves[i].slot;
-            for (int64_t p = ix->leaf_offsets[c]; p < ix->leaf_offsets[c + 1]; ++p, ++m) {
-                if (lut_mode == 0) {
-                    /* residual codes: q . x~ = q . centroid + table sum */
-                    cand[m].score = ix->residual ? ah_score_f64(ix, lut, p) + s[c] : ah_score_f64(ix, lut, p);
-                    cand[m].id = ix->slot_ids[p];
-                    cand[m].slot = (int32_t)p;
-                } else {
-                    ucand[m].sum = ah_sum_u8(ix, lut8, p);
-                    ucand[m].id = ix->slot_ids[p];
-                    ucand[m].slot = (int32_t)p;
-                }
-            }
-        }
-        if (out_scanned) out_scanned[qi] = total;
-
-        /* 4. best R by approximate score */
-        if (lut_mode == 0) qsort(cand, total, sizeof(orc_item), by_score_then_id);
-        else qsort(ucand, total, sizeof(orc_uitem), by_sum_then_id);
-        int32_t nc = total < R ? (int32_t)total : R;
-        if (out_ncand) out_ncand[qi] = nc;
-        for (int32_t i = 0; i < R; ++i) {
-            int64_t o = (int64_t)qi * R + i;
-            if (i < nc) {
-                if (out_cand_ids) out_cand_ids[o] = lut_mode == 0 ? cand[i].id : ucand[i].id;
-                if (out_cand_scores)
-                    out_cand_scores[o] = lut_mode == 0
-                        ? cand[i].score
-                        : (double)fmaf(delta, (float)ucand[i].sum, bias);
-                if (out_cand_sums) out_cand_sums[o] = lut_mode == 0 ? 0u : ucand[i].sum;
-            } else {
-                if (out_cand_ids) out_cand_ids[o] = -1;
-                if (out_cand_scores) out_cand_scores[o] = -INFINITY;
-                if (out_cand_sums) out_cand_sums[o] = 0u;
-            }
-        }
-
-        /* 5. reorder (exact rescoring) or pure approximate ranking */
-        orc_item *fin = (orc_item *)malloc(sizeof(orc_item) * (nc > 0 ? nc : 1));
-        for (int32_t i = 0; i < nc; ++i) {
-            int32_t slot = lut_mode == 0 ? cand[i].slot : ucand[i].slot;
-            fin[i].id = ix->slot_ids[slot];
-            fin[i].slot = slot;
-            if (reorder_num > 0) fin[i].score = exact_score(ix, q, slot);
-            else if (lut_mode == 0) fin[i].score = cand[i].score;
-            else fin[i].score = (double)fmaf(delta, (float)ucand[i].sum, bias);
-        }
-        if (reorder_num > 0) qsort(fin, nc, sizeof(orc_item), by_score_then_id);
-        for (int32_t i = 0; i < k; ++i) {
-            int64_t o = (int64_t)qi * k + i;
-            if (i < nc) {
-                out_ids[o] = fin[i].id;
-                out_scores[o] = fin[i].score;
-            } else {
-                out_ids[o] = -1;
-                out_scores[o] = -INFINITY;
-            }
-        }
-        free(fin);
-        free(cand);
-        free(ucand);
-        free(lut);
-        free(lut8);
+        /* 2-5 over those leaves */
+        search_in_leaves(ix, q, s, leaf_list, L, k, R, reorder_num, lut_mode, ORC_ROW(out_ids, qi, k),
+                         ORC_ROW(out_scores, qi, k), ORC_ROW(out_cand_ids, qi, R), ORC_ROW(out_cand_scores, qi, R),
+                         ORC_ROW(out_cand_sums, qi, R), ORC_ROW(out_ncand, qi, 1), ORC_ROW(out_scanned, qi, 1));
+        free(leaf_list);
         free(leaves);
+        free(s);
+    }
+    return 0;
+}
+
+/*
+ * Steps 2-5 only, over caller-given leaves: leaves [nq][L] (each row L
+ * distinct leaf ids in [0, num_leaves)) replace step 1's choice; everything
+ * after it is the arithmetic of orc_search.  Used to check the downstream
+ * stages of a query whose searched leaf set differs from the oracle's own by a
+ * near-tie at the L-th leaf.  Outputs as for orc_search (no leaf outputs).
+ * Returns 0, or -1 on bad arguments (including a leaf id out of range).
+ */
+int orc_search_leaves(const orc_index *ix, const float *Q, int32_t nq, int32_t k, int32_t L,
+                      const int32_t *leaves, int32_t reorder_num, int32_t lut_mode, int32_t nthreads,
+                      int32_t *out_ids, double *out_scores, int32_t *out_cand_ids, double *out_cand_scores,
+                      uint32_t *out_cand_sums, int32_t *out_ncand, int64_t *out_scanned) {
+    if (bad_search_args(ix, Q, nq, k, L, reorder_num, lut_mode, out_ids, out_scores) || !leaves) return -1;
+    for (int64_t i = 0; i < (int64_t)nq * L; ++i)
+        if (leaves[i] < 0 || leaves[i] >= ix->num_leaves) return -1;
+    const int32_t R = reorder_num > k ? reorder_num : k;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        const float *q = Q + (int64_t)qi * ix->d;
+        double *s = (double *)malloc(sizeof(double) * ix->num_leaves);
+        centroid_scores(ix, q, s);
+        search_in_leaves(ix, q, s, leaves + (int64_t)qi * L, L, k, R, reorder_num, lut_mode,
+                         ORC_ROW(out_ids, qi, k), ORC_ROW(out_scores, qi, k), ORC_ROW(out_cand_ids, qi, R),
+                         ORC_ROW(out_cand_scores, qi, R), ORC_ROW(out_cand_sums, qi, R), ORC_ROW(out_ncand, qi, 1),
+                         ORC_ROW(out_scanned, qi, 1));
         free(s);
     }
     return 0;

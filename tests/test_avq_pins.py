@@ -119,3 +119,57 @@ def test_generator_l2_codes_are_nearest_centers():
         d2 = ((Xs[:, None, b * dpb:(b + 1) * dpb] - cb[b][None]) ** 2).sum(-1)
         chosen = d2[np.arange(len(Xs)), codes[:, b]]
         assert (chosen <= d2.min(1) + 1e-6).all()
+
+
+def test_point_eta_rule():
+    # eta_ratio at each row's norm; 1 where the weight is undefined
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((6, 100))
+    X /= np.linalg.norm(X, axis=1, keepdims=True)
+    np.testing.assert_allclose(avq.point_eta(X, 0.2), 99 / 24, rtol=1e-14)
+    X2 = X * np.array([1, 2, 3, 0.5, 0.1, 0.0])[:, None]       # norms 1, 2, 3, 0.5, 0.1, 0
+    e = avq.point_eta(X2, 0.2)
+    np.testing.assert_allclose(e[:4], [99 * s / (1 - s) for s in (0.04, 0.01, 0.04 / 9, 0.16)], rtol=1e-13)
+    assert e[4] == 1.0 and e[5] == 1.0                         # T above the norm; a zero row
+    np.testing.assert_array_equal(avq.point_eta(X2, 0.0), 1.0)
+    np.testing.assert_array_equal(avq.point_eta(X2, -1.0), 1.0)
+
+
+def test_center_updates_at_eta_one_are_member_means():
+    # T <= 0: every eta is 1 and each center is the plain mean of its members
+    # (numpy); a center without members keeps its old value; assignments
+    # outside [0, nl) belong to no center
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((300, 8))
+    assign = rng.integers(-1, 7, 300)           # -1 and center 6 (of 6) are outside; center 5 left empty
+    assign[assign == 5] = 4
+    C_old = rng.standard_normal((6, 8))
+    C, counts = avq.center_updates(X, assign, C_old, 0.0)
+    for c in range(6):
+        mem = X[assign == c]
+        assert counts[c] == mem.shape[0]
+        if mem.shape[0]:
+            np.testing.assert_allclose(C[c], mem.mean(0), rtol=1e-12, atol=1e-13)
+        else:
+            np.testing.assert_array_equal(C[c], C_old[c])
+
+
+def test_center_updates_minimise_each_members_loss():
+    # T > 0: each center minimises its members' summed anisotropic loss, with
+    # eta per member from its own norm
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal((200, 6)) * rng.uniform(0.5, 2.0, (200, 1))
+    assign = rng.integers(0, 3, 200)
+    C, _ = avq.center_updates(X, assign, np.zeros((3, 6)), 0.3)
+    for c in range(3):
+        mem = X[assign == c]
+        eta = avq.point_eta(mem, 0.3)
+        assert (eta != 1.0).all()
+
+        def total(cc):
+            return avq.anisotropic_loss(mem, np.repeat(cc[None, :], mem.shape[0], 0), eta).sum()
+
+        base = total(C[c])
+        for _ in range(30):
+            v = rng.standard_normal(6) * 1e-3
+            assert total(C[c] + v) > base and total(C[c] - v) > base

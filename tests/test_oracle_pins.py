@@ -313,3 +313,79 @@ def test_worked_example_operation_counts():
     out = orc.search(q, 10, L, 0)
     assert out["scanned"][0] == g["points_scanned"]
     assert out["scanned"][0] * B == g["lookups"]
+
+
+# -- steps 2-5 over caller-given leaves (orc_search_leaves) --------------------
+
+def test_search_leaves_with_own_leaves_equals_search():
+    # the downstream arithmetic is the search's own: given the leaves step 1
+    # picked, every output equals the full search's, in both table modes
+    w, X, Q, ix, arr = _mini(aniso=True)
+    orc = OracleIndex(arr)
+    for mode in (0, 1):
+        full = orc.search(Q, w.k, w.num_leaves_to_search, w.reorder_num, mode)
+        part = orc.search_leaves(Q, full["leaves"], w.k, w.reorder_num, mode)
+        for key in ("ids", "scores", "cand_ids", "cand_scores", "cand_sums", "ncand", "scanned"):
+            np.testing.assert_array_equal(part[key], full[key], err_msg=key)
+
+
+def test_search_leaves_matches_numpy_on_arbitrary_leaves():
+    # leaves that are not the query's best (random distinct lists, in any
+    # order): candidates are the best R of those leaves' points by q . x~
+    # (numpy reconstruction), finals the best k of them by exact dot product
+    w, X, Q, ix, arr = _mini(aniso=True)
+    orc = OracleIndex(arr)
+    rng = np.random.default_rng(7)
+    L = 5
+    leaves = np.stack([rng.permutation(w.num_leaves)[:L] for _ in range(Q.shape[0])]).astype(np.int32)
+    out = orc.search_leaves(Q, leaves, w.k, w.reorder_num)
+    xt = _reconstruct(arr)
+    xs = X[arr["slot_ids"]].astype(np.float64)
+    for qi in range(Q.shape[0]):
+        scanned = np.concatenate([np.arange(arr["leaf_offsets"][c], arr["leaf_offsets"][c + 1])
+                                  for c in leaves[qi]])
+        assert out["scanned"][qi] == scanned.shape[0]
+        q = Q[qi].astype(np.float64)
+        sc = xt[scanned] @ q
+        nc = min(w.reorder_num, scanned.shape[0])
+        best = scanned[_order(sc, arr["slot_ids"][scanned])][:nc]
+        assert out["ncand"][qi] == nc
+        np.testing.assert_array_equal(out["cand_ids"][qi][:nc], arr["slot_ids"][best])
+        np.testing.assert_allclose(out["cand_scores"][qi][:nc], xt[best] @ q, rtol=0, atol=1e-12)
+        ex = xs[best] @ q
+        fin = best[_order(ex, arr["slot_ids"][best])][: w.k]
+        np.testing.assert_array_equal(out["ids"][qi][: len(fin)], arr["slot_ids"][fin])
+
+
+def test_search_leaves_u8_sums_match_numpy():
+    # uint8 tables: integer sums of the table entries the codes select (numpy's
+    # own unpacking), best R by (sum desc, id asc) over the given leaves
+    w, X, Q, ix, arr = _mini()
+    orc = OracleIndex(arr)
+    rng = np.random.default_rng(11)
+    L = 3
+    leaves = np.stack([rng.permutation(w.num_leaves)[:L] for _ in range(Q.shape[0])]).astype(np.int32)
+    out = orc.search_leaves(Q, leaves, w.k, 0, 1)
+    codes = arr["codes"]
+    B = codes.shape[1] * 2
+    idx = np.empty((codes.shape[0], B), np.int64)
+    idx[:, 0::2] = codes & 0x0F
+    idx[:, 1::2] = codes >> 4
+    for qi in range(Q.shape[0]):
+        lut8, delta, bias = orc.u8_table(Q[qi])
+        scanned = np.concatenate([np.arange(arr["leaf_offsets"][c], arr["leaf_offsets"][c + 1])
+                                  for c in leaves[qi]])
+        sums = lut8.astype(np.int64)[np.arange(B)[None, :], idx[scanned]].sum(1)
+        nc = min(w.k, scanned.shape[0])
+        best = scanned[np.lexsort((arr["slot_ids"][scanned], -sums))][:nc]
+        np.testing.assert_array_equal(out["cand_ids"][qi][:nc], arr["slot_ids"][best])
+        np.testing.assert_array_equal(out["cand_sums"][qi][:nc],
+                                      lut8.astype(np.int64)[np.arange(B)[None, :], idx[best]].sum(1))
+
+
+def test_search_leaves_rejects_bad_leaf_ids():
+    w, X, Q, ix, arr = _mini()
+    orc = OracleIndex(arr)
+    bad = np.full((Q.shape[0], 2), w.num_leaves, np.int32)
+    with pytest.raises(ValueError):
+        orc.search_leaves(Q, bad, w.k, w.reorder_num)
