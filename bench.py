@@ -3,8 +3,10 @@
 One step = one batched search of the whole hot path (centroid scores -> top-L
 leaves -> lookup tables -> 4-bit code scan -> top-R -> exact reorder -> top-k)
 over one batch of synthetic queries, through the C ABI.  Default workload: the
-GloVe-shaped IVF-AH configuration (n = 1,000,000, d = 100, 1,000 leaves,
-32 searched, 1,000 queries, k = 10, reorder 100).
+largest fixed single-GPU configuration, OpenAI-embedding-shaped IVF-AH
+(n = 2,000,000, d = 1,536, dims_per_block = 4, 2,000 leaves, 40 searched,
+10,000 queries, k = 10, reorder 300 against a bfloat16 copy); ``--workload``
+selects another (tiny, glove, bigann, openai; ``--sweep`` for the sweep).
 
 Single GPU:  python bench.py [--steps K --warmup W]
 N GPUs:      python -m torch.distributed.run --nproc-per-node N bench.py --gpus N
@@ -48,7 +50,7 @@ def parse():
     p.add_argument("--steps", type=int, default=400)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="glove")
+    p.add_argument("--workload", default="openai")
     p.add_argument("--lut-mode", type=int, default=0, choices=[0, 1])
     p.add_argument("--nq", type=int, default=None)
     p.add_argument("--leaves", type=int, default=None, help="num_leaves_to_search")
@@ -127,22 +129,66 @@ def rank_workload(w, rank):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed
+    region, read-only.  NVML is polled in-process every ``period_s`` (1 ms by
+    default, so a timed region of a few milliseconds still gets samples);
+    without NVML it falls back to ``nvidia-smi -lms 100``."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                   "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device, period_s: float = 0.001):
+        self.device = device
+        self.period = period_s
         self.proc = None
         self.lines = []
+        self.samples = []            # (sm MHz, max MHz, reason bits)
+        self.source = None
+        self._stop = threading.Event()
+        self._t = None
+        self._nvml = None
+        self._h = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        idx = self.device.index if hasattr(self.device, "index") else int(self.device)
+        p = torch.cuda.get_device_properties(idx or 0)
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _poll(self):
+        nv, h = self._nvml, self._h
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def __enter__(self):
         try:
+            self._h = self._nvml_handle()
+            self.source = "nvml"
+            self._t = threading.Thread(target=self._poll, daemon=True)
+            self._t.start()
+            return self
+        except Exception:
+            self._nvml = None
+        try:
+            idx = self.device.index if hasattr(self.device, "index") else int(self.device)
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "100"],
+                                          "-i", str(idx or 0), "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
         except (FileNotFoundError, OSError):
@@ -154,6 +200,13 @@ class ClockSampler:
             self.lines.append(ln.strip())
 
     def __exit__(self, *a):
+        self._stop.set()
+        if self._nvml is not None and self._t is not None:
+            self._t.join(timeout=5)
+            try:
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc:
             self.proc.terminate()
             try:
@@ -163,6 +216,12 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
+        for s, m, bits in self.samples:
+            sm.append(s)
+            mx.append(m)
+            for nm, bit in self.REASON_BITS.items():
+                if bits & bit:
+                    reasons.add(nm)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
@@ -177,9 +236,9 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def workload_spec(args):
@@ -256,7 +315,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64" if args.lut_mode == 0 else "u8",
-            "data": "synthetic (seeded Gaussian mixture, GloVe-shaped)", "config": config_dict(w, args),
+            "data": f"synthetic (seeded Gaussian mixture, {w.name}-shaped)", "config": config_dict(w, args),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": oracle.max_threads(), "kind": "oracle", "cpu_model": cpu_model(),
                              "sample": f"{S} of {w.nq} queries per step, {len(times)} steps"},
@@ -317,9 +376,10 @@ def run_ours(args):
             ev0[s].record(stream)
             index.search(qg, k, L, R, mode)
             ev1[s].record(stream)
-            if s % 50 == 49 or s == args.steps - 1:
-                stage_ms.setdefault("scan_timed", []).append(sum(
-                    v for kname, v in index.stage_times().items() if kname in ("scan", "scan_rest")))
+            # the scan phases' events of every timed step (reading them waits
+            # for this step; the next step's flush and launches follow)
+            stage_ms.setdefault("scan_timed", []).append(sum(
+                v for kname, v in index.stage_times().items() if kname in ("scan", "scan_rest")))
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     # per-stage breakdown (every stage marked), outside the timed region
@@ -359,7 +419,7 @@ def run_ours(args):
 
     if rank == 0:
         med = {kname: statistics.median(v) for kname, v in stage_ms.items() if kname != "scan_timed"}
-        scan_ms = statistics.median(stage_ms["scan_timed"])      # scan kernel time inside the timed steps
+        scan_ms = statistics.fmean(stage_ms["scan_timed"])       # mean scan time over every timed step
         clocks = clk.summary()
         lookups = scanned * w.blocks
         bytes_per_lookup = 4 if mode == 0 else 1
@@ -379,7 +439,13 @@ def run_ours(args):
                                 if args.nq is None and args.leaves is None else None),
                     "kernel": "scan_kernel", "unit_bytes": f"{bytes_per_lookup} B per table lookup",
                     "lookups_per_launch": lookups,
-                    "peak_source": f"derived: {SM_COUNT} SMs x {SMEM_BYTES_PER_CLK} B/clk x {mhz:.0f} MHz"}
+                    "peak_source": f"derived: {SM_COUNT} SMs x {SMEM_BYTES_PER_CLK} B/clk x {mhz:.0f} MHz",
+                    "scan_ms_mean": scan_ms, "scan_steps": len(stage_ms["scan_timed"])}
+        if clocks.get("sm_mhz"):
+            # the same fraction against the peak at the SM clock sampled during the timed steps
+            at_clk = SM_COUNT * SMEM_BYTES_PER_CLK * clocks["sm_mhz"] * 1e6 / 1e9
+            roofline["frac_at_sampled_clock"] = achieved / at_clk
+            roofline["peak_at_sampled_clock"] = at_clk
         # the step against the sum of its stages' roofline times: centroid GEMM at
         # the SIMT fp32 FMA peak, the scan at the larger of its SMEM-lookup and
         # unique-code HBM times, the reorder gather at the HBM copy rate
@@ -396,7 +462,7 @@ def run_ours(args):
         line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32" if mode == 0 else "u8",
-                "data": "synthetic (seeded Gaussian mixture, GloVe-shaped; index trained on it)",
+                "data": f"synthetic (seeded Gaussian mixture, {w.name}-shaped; index trained on it)",
                 "config": config_dict(w, args),
                 "roofline": roofline, "step_roofline": step_roofline,
                 "scan": {"ms": scan_ms, "hbm_unique_code_gbs": unique_code_bytes / (scan_ms * 1e-3) / 1e9,
@@ -578,6 +644,20 @@ def run_kmeans(args):
             ta += e0.elapsed_time(e1)
             tu += e1.elapsed_time(e2)
     ta, tu = ta / args.steps, tu / args.steps
+    # the anisotropic center update on the same assignment (eta per point from
+    # the workload's threshold T, 0.2 where it names none)
+    from mips_ivf_centroid_b200 import avq_update
+    T_avq = w.threshold_T or 0.2
+    for _ in range(max(1, args.warmup)):
+        Cv, _, it = avq_update(Xg, a, Cg, T_avq)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        Cv, _, it = avq_update(Xg, a, Cg, T_avq)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    tv = e0.elapsed_time(e1) / args.steps
+    it_np = it.cpu().numpy()
     ops = 3.0 * w.n * w.num_leaves * w.d           # difference, square, sum per (point, centroid, coordinate)
     mhz = SM_MAX_MHZ_FALLBACK
     peak = SM_COUNT * 64 * mhz * 1e6
@@ -592,13 +672,17 @@ def run_kmeans(args):
             "data": "synthetic (seeded Gaussian mixture)",
             "config": {"workload": f"{w.name}-shaped: n={w.n:,} d={w.d} centroids={w.num_leaves}"},
             "assign_ms": ta, "update_ms": tu,
+            "avq_update": {"ms": tv, "T": T_avq, "cg_steps_mean": float(it_np.mean()), "cg_steps_max": int(it_np.max()),
+                           "points_per_s": w.n / (tv * 1e-3),
+                           "note": "closed-form anisotropic center update (conjugate gradients, fp64) on the same assignment"},
             "roofline": {"bound": "alu", "kernel": "kmeans_assign", "achieved": ops / (ta * 1e-3) / 1e12,
                          "peak": peak / 1e12, "unit": "Tops/s (fp64)", "frac": ops / (ta * 1e-3) / peak,
                          "traffic": None,
                          "peak_source": f"derived: {SM_COUNT} SMs x 64 fp64 lanes x {mhz:.0f} MHz (nominal rate)"},
             "cpu_baseline": {"value": ns / ot, "unit": "points/s (assignment)", "cores": oracle.max_threads(),
                              "kind": "oracle", "cpu_model": cpu_model(), "sample": f"first {ns} points"},
-            "oracle_match_on_sample": same, "clocks": clk.summary(), "gpu_launches": 2 * (args.steps + args.warmup)}
+            "oracle_match_on_sample": same, "clocks": clk.summary(),
+            "gpu_launches": 2 * (args.steps + args.warmup) + 4 * (args.steps + max(1, args.warmup))}
     print(json.dumps(line), flush=True)
 
 
