@@ -61,12 +61,23 @@ def same_set(a, b):
 
 
 def compare_search(index, arr, Q, k, L, reorder_num, lut_mode, qsel=None, max_leaf_mismatch=0.02,
-                   max_cand_mismatch=0.05, orc=None):
+                   max_cand_mismatch=0.05, orc=None, label=""):
     """Search all of Q on the GPU (one batch, as the benchmark launches it),
     then check the rows ``qsel`` stage by stage against the oracle.
 
-    Returns a dict with the mismatch counts and the GPU/oracle outputs of the
-    checked rows."""
+    Every checked query is checked through every stage.  Leaves: ranked match
+    with the oracle's own best L.  Where a near-tie at the L-th leaf makes the
+    GPU's leaf set differ (a swap the ranked match allows), the later stages
+    of that query are compared with the oracle run over the GPU's leaves
+    (``OracleIndex.search_leaves``: the same arithmetic from the table on), so
+    no query goes unchecked.  Candidates: ranked match (fp32 tables) or
+    bit-exact ids, integer sums and scores (uint8 tables).  Final results:
+    ranked match with the oracle's; where a near-tie at the R-th candidate
+    makes the candidate sets differ, the GPU's final ids must be the best k of
+    its own candidates by the oracle's scores.
+
+    Returns a dict with the counts (checked queries, leaf-set swaps,
+    candidate-set swaps) and the GPU/oracle outputs of the checked rows."""
     import torch
     from oracle import OracleIndex
 
@@ -84,48 +95,71 @@ def compare_search(index, arr, Q, k, L, reorder_num, lut_mode, qsel=None, max_le
     n = arr["slot_ids"].shape[0]
     inv = np.empty(n, np.int64)
     inv[arr["slot_ids"]] = np.arange(n)
-    leaf_mis = cand_mis = 0
-    for i in range(Qs.shape[0]):
-        q = Qs[i]
-        cs = orc.centroid_scores(q)
+    nq = Qs.shape[0]
+
+    # 1. leaves, every query
+    for i in range(nq):
+        def leaf_scores_of(g, i=i):
+            # the oracle's fp64 scores of the GPU's leaves: from its own list when
+            # it holds them all, else every centroid scored afresh
+            pos = {int(c): j for j, c in enumerate(o["leaves"][i])}
+            if all(int(c) in pos for c in g):
+                return o["leaf_scores"][i][[pos[int(c)] for c in g]]
+            return orc.centroid_scores(Qs[i])[g]
         ranked_match(tr["leaf_ids"][i], tr["leaf_scores"][i], o["leaves"][i], o["leaf_scores"][i],
-                     lambda g: cs[g], f"q{qsel[i]} leaves")
-        if not same_set(tr["leaf_ids"][i], o["leaves"][i]):
-            leaf_mis += 1
-            continue
-        assert tr["scanned"][i] == o["scanned"][i], f"q{qsel[i]} scanned"
-        assert tr["ncand"][i] == o["ncand"][i], f"q{qsel[i]} ncand"
+                     leaf_scores_of, f"{label} q{qsel[i]} leaves")
+    swapped = np.array([i for i in range(nq) if not same_set(tr["leaf_ids"][i], o["leaves"][i])], np.int64)
+    # the reference for the later stages: the oracle's own search, or for a
+    # swapped leaf set the oracle over the GPU's leaves
+    ref = {kk: o[kk].copy() for kk in ("ids", "scores", "cand_ids", "cand_scores", "cand_sums", "ncand", "scanned")}
+    if swapped.shape[0]:
+        o2 = orc.search_leaves(Qs[swapped], tr["leaf_ids"][swapped], k, reorder_num, lut_mode)
+        for kk in ref:
+            ref[kk][swapped] = o2[kk]
+
+    # 2.-3. candidates and final results, every query
+    cand_mis = 0
+    for i in range(nq):
+        q = Qs[i]
+        what = f"{label} q{qsel[i]}"
+        assert tr["scanned"][i] == ref["scanned"][i], f"{what} scanned {tr['scanned'][i]} vs {ref['scanned'][i]}"
+        assert tr["ncand"][i] == ref["ncand"][i], f"{what} ncand"
         gc = tr["cand_ids"][i]
         if lut_mode == 1:
-            np.testing.assert_array_equal(gc, o["cand_ids"][i], err_msg=f"q{qsel[i]} u8 candidates")
-            np.testing.assert_array_equal(tr["cand_sums"][i].astype(np.uint32), o["cand_sums"][i])
-            np.testing.assert_array_equal(tr["cand_scores"][i], o["cand_scores"][i].astype(np.float32))
+            np.testing.assert_array_equal(gc, ref["cand_ids"][i], err_msg=f"{what} u8 candidates")
+            np.testing.assert_array_equal(tr["cand_sums"][i].astype(np.uint32), ref["cand_sums"][i],
+                                          err_msg=f"{what} u8 sums")
+            np.testing.assert_array_equal(tr["cand_scores"][i], ref["cand_scores"][i].astype(np.float32),
+                                          err_msg=f"{what} u8 scores")
         else:
-            ranked_match(gc, tr["cand_scores"][i], o["cand_ids"][i], o["cand_scores"][i],
-                         lambda g: orc.point_scores(q, inv[g])[0], f"q{qsel[i]} candidates")
+            ranked_match(gc, tr["cand_scores"][i], ref["cand_ids"][i], ref["cand_scores"][i],
+                         lambda g: orc.point_scores(q, inv[g])[0], f"{what} candidates")
         if reorder_num > 0:
             exact_of = lambda g: orc.point_scores(q, inv[g])[1]
         elif lut_mode == 0:
             exact_of = lambda g: orc.point_scores(q, inv[g])[0]
         else:
             exact_of = None
-        if not same_set(gc, o["cand_ids"][i]):
+        if not same_set(gc, ref["cand_ids"][i]):
+            # only a near-tie at the R-th candidate (fp32 tables) gets here
+            assert exact_of is not None, f"{what}: u8 candidate sets differ"
             cand_mis += 1
             nc = int((gc >= 0).sum())
-            if exact_of is None:
-                continue
             ex = exact_of(gc[:nc])
             order = np.lexsort((gc[:nc], -ex))[:k]
             ranked_match(ids[i], scores[i], np.pad(gc[:nc][order], (0, k - len(order)), constant_values=-1),
                          np.pad(ex[order], (0, k - len(order)), constant_values=-np.inf), exact_of,
-                         f"q{qsel[i]} final*")
+                         f"{what} final (own candidates)")
             continue
-        if exact_of is None:
-            np.testing.assert_array_equal(ids[i], o["ids"][i])
-            np.testing.assert_array_equal(scores[i], o["scores"][i].astype(np.float32))
+        if exact_of is None:     # uint8 approximate ranking: bit-exact
+            np.testing.assert_array_equal(ids[i], ref["ids"][i], err_msg=f"{what} u8 final ids")
+            np.testing.assert_array_equal(scores[i], ref["scores"][i].astype(np.float32),
+                                          err_msg=f"{what} u8 final scores")
         else:
-            ranked_match(ids[i], scores[i], o["ids"][i], o["scores"][i], exact_of, f"q{qsel[i]} final")
-    nq = Qs.shape[0]
-    assert leaf_mis <= max(1, max_leaf_mismatch * nq), f"{leaf_mis} queries with a different leaf set"
+            ranked_match(ids[i], scores[i], ref["ids"][i], ref["scores"][i], exact_of, f"{what} final")
+    print(f"parity {label or ''}: {nq} queries checked through every stage, "
+          f"{swapped.shape[0]} leaf-set swaps, {cand_mis} candidate-set swaps")
+    assert swapped.shape[0] <= max(1, max_leaf_mismatch * nq), f"{swapped.shape[0]} queries with a different leaf set"
     assert cand_mis <= max(1, max_cand_mismatch * nq), f"{cand_mis} queries with a different candidate set"
-    return dict(leaf_mismatch=leaf_mis, cand_mismatch=cand_mis, ids=ids, scores=scores, oracle=o, trace=tr)
+    return dict(checked=nq, leaf_mismatch=int(swapped.shape[0]), cand_mismatch=cand_mis, ids=ids, scores=scores,
+                oracle=o, ref=ref, trace=tr)
