@@ -24,7 +24,10 @@
  * Conventions for every entry point:
  *  - Status codes only: no exceptions cross the ABI, nothing calls exit/abort.
  *  - Device pointers are CUDA device memory on the current device; the library
- *    never frees memory it did not allocate.
+ *    never frees memory it did not allocate.  An index belongs to the device
+ *    that was current when it was built: ah_search, ah_search_traced,
+ *    ah_search_host, ah_reserve and ah_search_leaves_noalloc need that device
+ *    current (AH_ERR_INVALID_ARG otherwise, before anything is enqueued).
  *  - Every array must hold at least the elements that its documented shape
  *    and the sizes passed with it give.  The library checks the sizes, but it
  *    cannot see the allocation behind a pointer: a shorter buffer is read or
@@ -65,7 +68,7 @@ typedef enum {
     AH_ERR_OOM = 3,          /* device allocation failed                       */
     AH_ERR_CUDA = 4,         /* a CUDA runtime call failed                     */
     AH_ERR_DEVICE = 5,       /* a kernel reported an error (see ah_sync_status) */
-    AH_ERR_TIMEOUT = 6       /* reserved: a bounded device wait gave up        */
+    AH_ERR_TIMEOUT = 6       /* a bounded device wait gave up (ah_sync_status) */
 } ah_status;
 
 /* reorder_dtype values */
@@ -227,25 +230,38 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
  *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves, to
  *                            bound its R-th best approximate score before the
  *                            scan (default 1024; the bound uses
- *                            max(value, 4 R) points, at most 4096)
+ *                            max(value, 4 R) points, at most 4096; batches of
+ *                            fewer than 1,024 queries use more, up to 4096,
+ *                            when the bound would otherwise keep many points)
  *   AH_OPT_THRESHOLD_LEAVES  how many of the best leaves that sample is spread
  *                            over, evenly; the rest of the sample follows
  *                            rank order (default 1: a prefix in rank order)
  *   AH_OPT_PROGRESSIVE_LEAVES  scan each query's best L1 leaves first, raise its
  *                            bound to the R-th best point they kept, then scan
  *                            up to 8x as many leaves at a time the same way:
- *                            0 = automatic (several phases when the sample's
- *                            bound is expected to keep many points and
- *                            nq >= 64), -1 = one pass, n = L1
+ *                            0 = automatic (batches of 1,024 or more queries:
+ *                            several phases when the sample's bound is
+ *                            expected to keep many points; smaller batches:
+ *                            one pass with a larger sample), -1 = one pass,
+ *                            n = L1
  *   AH_OPT_SCAN_CHUNK_TILES  32-point code tiles per scan work item (0 =
  *                            automatic, the default)
+ *   AH_OPT_UINT8_TENSOR_CORES  how the scan sums uint8 tables: 0 = table
+ *                            lookups; 2 = on the int8 tensor cores (each
+ *                            point's codes expanded one-hot, multiplied by the
+ *                            queries' tables, summed exactly in int32); 1 =
+ *                            automatic, the default (tensor cores when a
+ *                            searched leaf holds about 16 or more queries of
+ *                            the batch on average).  The integer sums are the
+ *                            same either way.
  * Errors: AH_ERR_INVALID_ARG for an unknown option or a value out of range.
  */
 enum {
     AH_OPT_THRESHOLD_SAMPLE = 1,
     AH_OPT_SCAN_CHUNK_TILES = 2,
     AH_OPT_THRESHOLD_LEAVES = 3,
-    AH_OPT_PROGRESSIVE_LEAVES = 4
+    AH_OPT_PROGRESSIVE_LEAVES = 4,
+    AH_OPT_UINT8_TENSOR_CORES = 5
 };
 AH_API ah_status ah_set_option(ah_index *ix, int32_t option, int64_t value);
 
@@ -294,19 +310,23 @@ AH_API ah_status ah_index_memory(ah_index *ix, int64_t *bytes);
  *   out_leaf_scores  float [nq][num_leaves_to_search], device (fp32 q . c)
  * The scratch must hold nq * num_leaves scores plus small counters; larger
  * batches are rejected with AH_ERR_UNSUPPORTED before anything is enqueued
- * (split the batch).  The index's device must be current.  The first call on
- * a device looks up the scratch array's device address (a runtime query, no
- * allocation); make that first call before any stream capture.  All calls
- * share the one scratch area: calls whose work overlaps on the GPU (different
- * streams, or different indexes on one device) race and must be serialised by
- * the caller.  Results equal the leaves ah_search_traced reports.
+ * (split the batch).  The index's device must be current.  The scratch's
+ * device address is looked up when the index is built (ah_build_index_views,
+ * ah_load): the first such lookup on a device loads the library's device
+ * module that holds the array, which is when the array's memory is placed, so
+ * this call itself neither allocates nor loads anything.  The address belongs
+ * to the index: after the device's primary context is reset
+ * (cudaDeviceReset) indexes built before the reset, and this address with
+ * them, are invalid.  All calls share the one scratch area: calls whose work
+ * overlaps on the GPU (different streams, or different indexes on one device)
+ * race and must be serialised by the caller.  Results equal the leaves
+ * ah_search_traced reports.
  */
 #define AH_NOALLOC_SCRATCH_BYTES (8u << 20)
 AH_API ah_status ah_search_leaves_noalloc(ah_index *ix, const float *queries, int32_t nq,
                                           int32_t num_leaves_to_search, int32_t *out_leaf_ids,
                                           float *out_leaf_scores, void *cuda_stream);
 
-/* Release everything the index owns.  Does not touch the borrowed views. */
 /*
  * Index directories (ScaNN blog, "Using the library": a built searcher is
  * written to a directory and loaded back later).  ah_save writes the index's
@@ -401,6 +421,38 @@ AH_API ah_status ah_kmeans_update(const float *X, int64_t n, int32_t d, const in
                                   const float *C_old, float *C_new, int64_t *counts, void *cuda_stream);
 
 /*
+ * Anisotropic center update, the closed-form step of anisotropic k-means
+ * (ScaNN blog, "Training an anisotropic codebook yourself", Theorem 4.2 form;
+ * loss from "The loss in one paragraph" with h_perp = 1).  For every center c
+ * with members i (assign[i] == c), in ascending point order:
+ *   eta_i = (d - 1) t / (1 - t), t = (T / ||x_i||)^2 (eta_i = 1 when T <= 0,
+ *   ||x_i|| = 0 or t >= 1), u_i = x_i / ||x_i||;
+ *   C_new[c] solves (m I + sum_i (eta_i - 1) u_i u_i^T) c = sum_i eta_i x_i,
+ * the minimiser of sum_i (eta_i - 1) ((x_i - c) . u_i)^2 + ||x_i - c||^2 (the
+ * plain mean when every eta_i = 1).  A center without members keeps C_old[c].
+ * The system matrix is never formed: conjugate gradients in fp64 from c = 0,
+ * each step applying it as m p + sum_i (eta_i - 1) (u_i . p) u_i, stop when
+ * the residual norm is at most tol times ||sum_i eta_i x_i|| or after
+ * max_iters steps (the matrix is symmetric positive definite whenever every
+ * eta_i > 0, with condition number at most max(eta) / min(eta, 1), so a few
+ * tens of steps reach tol = 1e-14).  Every reduction runs in a fixed order, so
+ * the result does not depend on scheduling; it is rounded to float at the end.
+ *   X [n][d] float, assign [n] int32 (entries outside [0, nl) belong to no
+ *   center), C_old [nl][d] float, C_new [nl][d] float out (must not overlap
+ *   C_old), counts [nl] int64 out or NULL (members), iters [nl] int32 out or
+ *   NULL (steps taken); all device memory.
+ * Asynchronous on cuda_stream; a temporary workspace of about 28 n + 12 nl
+ * bytes is taken from the device's stream-ordered memory pool on cuda_stream
+ * and returned to it on the same stream (no device synchronisation).  Errors:
+ * AH_ERR_INVALID_ARG (NULL array, n < 0, d < 1, nl < 1, max_iters outside
+ * [0, 100000], tol outside [0, 1)), AH_ERR_UNSUPPORTED (d above 6400, n of
+ * 2^31 or more), AH_ERR_OOM, AH_ERR_CUDA.
+ */
+AH_API ah_status ah_avq_update(const float *X, int64_t n, int32_t d, const int32_t *assign, int32_t nl,
+                               const float *C_old, double T, int32_t max_iters, double tol, float *C_new,
+                               int64_t *counts, int32_t *iters, void *cuda_stream);
+
+/*
  * Exact merge for a leaf-partitioned search.  G shards hold the same
  * centroids and codebook and disjoint sets of leaves' points (the other
  * leaves empty), so every shard picks the same L leaves and scans its own
@@ -424,6 +476,7 @@ AH_API ah_status ah_merge_shards(int32_t G, int32_t nq, int32_t R, int32_t k, co
                                  const float *cand_approx, const float *cand_exact, int32_t *out_ids,
                                  float *out_scores, void *cuda_stream);
 
+/* Release everything the index owns.  Does not touch the borrowed views. */
 AH_API void ah_destroy(ah_index *ix);
 
 /* Static text for a status code. */

@@ -6,10 +6,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -57,6 +57,29 @@ struct Workspace {
 
 int cap_for(int R) { return std::max(8192, 16 * R); }
 
+
+
+}  // namespace
+
+// Scratch of ah_search_leaves_noalloc: the centroid score matrix and the
+// per-leaf counters of the partition stage, in a file-scope device array so
+// that the call never allocates.  On the host this name is only a stand-in for
+// the array, not its device address: host code obtains the address with
+// cudaGetSymbolAddress (on the current device) and passes that to kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[AH_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of the scratch array on the current device.  The first
+// lookup on a device loads this file's device module, which places the array
+// in device memory; it is done when an index is built, so the search-time
+// call itself neither allocates nor loads anything.
+ah_status lookup_noalloc_scratch(void** out) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "scratch address lookup");
+    *out = p;
+    return AH_OK;
+}
 }  // namespace
 
 struct ah_index {
@@ -67,6 +90,7 @@ struct ah_index {
     int32_t* offs32 = nullptr;
     int32_t* ptile = nullptr;
     uint32_t* codes_il = nullptr;
+    float* c_split = nullptr;        // [2][NL][d] centroids split for the tensor-core scores (or null)
     int* err = nullptr;
     size_t owned_bytes = 0;
     Workspace ws;
@@ -83,7 +107,9 @@ struct ah_index {
     int opt_threshold_leaves = 1;
     int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
+    int opt_u8_tensor = 1;           // uint8 scan on the tensor cores: 0 never, 1 automatic, 2 always
     void* loaded[6] = {};            // index arrays owned by an index from ah_load
+    void* noalloc_scratch = nullptr; // device address of the library's fixed scratch on this device
     // side stream for the stages that do not depend on the partition stage
     // (lookup tables; the query->leaf inversion once top-L is known)
     cudaStream_t side = nullptr;
@@ -127,6 +153,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     add(stage ? sizeof(float) * (size_t)cnq * ck : 0);          // 17 dscores
     add(sizeof(int32_t) * (size_t)cnq * cap);                   // 18 candidate slots
     add(sizeof(int32_t) * (size_t)cnq);                         // 19 finish order
+    add(ix->c_split ? 2 * sizeof(float) * (size_t)cnq * d : 0);  // 20 queries split for the tensor cores
     size_t total = 0;
     for (int i = 0; i < n; ++i) total += sz[i];
     if (w.base) {
@@ -162,6 +189,8 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     b.ckey = reinterpret_cast<uint64_t*>(part[9]);
     b.cslot = reinterpret_cast<int32_t*>(part[18]);
     b.order = reinterpret_cast<int32_t*>(part[19]);
+    b.q_hi = ix->c_split ? reinterpret_cast<float*>(part[20]) : nullptr;
+    b.q_lo = ix->c_split ? b.q_hi + (size_t)cnq * d : nullptr;
     int32_t* zr = reinterpret_cast<int32_t*>(part[10]);
     b.qcount = zr;
     b.qcursor = zr + NL;
@@ -184,9 +213,22 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     return AH_OK;
 }
 
+// The index's pointers and workspace belong to the device it was built on; a
+// call made with another device current would allocate and launch there.
+ah_status check_current_device(const ah_index* ix) {
+    int device = -1;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    if (device != ix->device)
+        return fail(AH_ERR_INVALID_ARG, "the index's device (" + std::to_string(ix->device) +
+                                            ") is not the current device (" + std::to_string(device) + ")");
+    return AH_OK;
+}
+
 ah_status validate_search(ah_index* ix, const void* queries, int32_t nq, int32_t k, int32_t L, int32_t reorder_num,
                           int32_t lut_mode, const void* out_ids, const void* out_scores) {
     if (!ix) return fail(AH_ERR_INVALID_ARG, "index is NULL");
+    if (ah_status st = check_current_device(ix); st != AH_OK) return st;
     if (nq < 0) return fail(AH_ERR_INVALID_ARG, "nq < 0");
     if (nq > 0 && (!queries || !out_ids || !out_scores)) return fail(AH_ERR_INVALID_ARG, "NULL queries or outputs");
     if (k <= 0) return fail(AH_ERR_INVALID_ARG, "k must be >= 1");
@@ -224,7 +266,20 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     a.reorder_num = reorder_num;
     a.R = R;
     a.lut_mode = lut_mode;
-    a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : (nq >= 64 ? 32 : 8);   // code tiles per scan item
+    // uint8 tables scan on the int8 tensor cores when a leaf's queries fill a
+    // good part of the 128-row MMA tile (about 16 or more per searched leaf)
+    a.scan_tc = (lut_mode == AH_LUT_U8 && ix->opt_u8_tensor != 0 &&
+                 (ix->opt_u8_tensor == 2 || static_cast<double>(nq) * L >= 16.0 * ix->dix.nl)) ? 1 : 0;
+    // code tiles per scan item: up to 32, fewer (multiples of 8, one tile per
+    // warp of a 256-thread CTA) when the batch's tiles, estimated from the
+    // average leaf, would leave scan CTAs (about 6 per SM) without an item
+    {
+        const double est_tiles = static_cast<double>(nq) * L * std::max(1.0, static_cast<double>(ix->dix.n) / ix->dix.nl / 32.0);
+        const double ctas = static_cast<double>(ix->num_sms) * 6;
+        const int c = 8 * static_cast<int>(std::ceil(est_tiles / ctas / 8.0));
+        a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : std::min(32, std::max(8, c));
+        if (a.scan_tc) a.chunk = ah::scan_tc_chunk_tiles();
+    }
     a.threshold_sample = ix->opt_threshold_sample;
     a.threshold_leaves = ix->opt_threshold_leaves;
     a.out_ids = out_ids;
@@ -285,12 +340,25 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     // is raised to the R-th best point kept (and its buffer compacted).
     std::vector<int> bounds{0};
     {
-        const int M = ah::threshold_sample(a.R, ix->opt_threshold_sample);
         const double avg_leaf = static_cast<double>(dix.n) / dix.nl;
-        const double expect_one_pass = 0.25 * a.R * L * avg_leaf / M;   // points kept by the sample's bound
+        // points the sample's bound is expected to keep: about 0.25 R of
+        // every M scanned (the sample comes from the best leaves)
+        auto expect = [&](int M) { return 0.25 * a.R * L * avg_leaf / M; };
+        // batches under 1,024 queries: the sample grows (up to 4,096 points)
+        // until the expected kept set is an eighth of the buffer, and the scan
+        // runs in one pass; on the 50M-point sweep index this beat scan
+        // phases at every batch of 16-256 queries (phase boundaries cost more
+        // there than the larger sample)
+        const bool small = nq < 1024;
+        if (small && ix->opt_progressive_leaves == 0) {
+            const double need = 0.25 * a.R * L * avg_leaf / (b.cap / 8);
+            a.threshold_sample = std::max(ix->opt_threshold_sample,
+                                          static_cast<int>(std::min<double>(ah::kMaxThresholdSample, std::ceil(need))));
+        }
+        const int M = ah::threshold_sample(a.R, a.threshold_sample);
         int first = L;
         if (ix->opt_progressive_leaves > 0) first = std::min(L, ix->opt_progressive_leaves);
-        else if (ix->opt_progressive_leaves == 0 && nq >= 64 && expect_one_pass > b.cap / 8)
+        else if (ix->opt_progressive_leaves == 0 && !small && expect(M) > b.cap / 8)
             first = std::max(1, std::min(L, static_cast<int>(4.0 * M / avg_leaf)));
         for (int e2 = first; ; e2 = std::min(L, 8 * e2)) {
             bounds.push_back(e2);
@@ -409,6 +477,10 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
         delete ix;
         return cuda_fail(e, "device query");
     }
+    if (ah_status st = lookup_noalloc_scratch(&ix->noalloc_scratch); st != AH_OK) {
+        delete ix;
+        return st;
+    }
     const int B = v->d / v->dims_per_block;
     const int cb = B / 2;
     const int W = (cb + 3) / 4;
@@ -449,6 +521,22 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
         return cuda_fail(e, "index allocation");
     }
     ix->owned_bytes = il_bytes + 2 * offs_bytes + sizeof(int);
+    // centroids split into tf32 halves for the tensor-core scores (when their
+    // rows suit the tensor maps and there are enough of them)
+    const bool tc = ah::centroid_tc_usable(1 << 20, NL, v->d);
+    if (tc) {
+        const size_t cs_bytes = 2 * sizeof(float) * (size_t)NL * v->d;
+        if ((e = cudaMalloc(&ix->c_split, cs_bytes)) != cudaSuccess) {
+            ah_destroy(ix);
+            return cuda_fail(e, "index allocation");
+        }
+        ix->owned_bytes += cs_bytes;
+        if ((e = ah::launch_split_tf32(v->centroids, (int64_t)NL * v->d, ix->c_split, ix->c_split + (size_t)NL * v->d,
+                                       s)) != cudaSuccess) {
+            ah_destroy(ix);
+            return cuda_fail(e, "centroid split");
+        }
+    }
     if ((e = cudaMemcpy(ix->offs32, o32.data(), offs_bytes, cudaMemcpyHostToDevice)) != cudaSuccess ||
         (e = cudaMemcpy(ix->ptile, pt.data(), offs_bytes, cudaMemcpyHostToDevice)) != cudaSuccess ||
         (e = cudaMemsetAsync(ix->err, 0, sizeof(int), s)) != cudaSuccess ||
@@ -464,12 +552,15 @@ ah_status ah_build_index_views(const ah_index_views* v, void* cuda_stream, ah_in
     d.dpb = v->dims_per_block;
     d.B = B;
     d.W = W;
+    d.V = ah::code_vector_words(W);
     d.centroids = v->centroids;
     d.offs = ix->offs32;
     d.ptile = ix->ptile;
     d.slot_ids = v->slot_ids;
     d.codes_il = ix->codes_il;
     d.codebook = v->codebook;
+    d.c_hi = ix->c_split;
+    d.c_lo = ix->c_split ? ix->c_split + (size_t)NL * v->d : nullptr;
     d.reorder_vecs = v->reorder_vecs;
     d.reorder_bf16 = v->reorder_dtype == AH_BF16 ? 1 : 0;
     d.residual = v->residual;
@@ -534,6 +625,7 @@ ah_status ah_sync_status(ah_index* ix, void* cuda_stream) {
         case ah::kDevCandOverflow: return fail(AH_ERR_DEVICE, "candidate buffer overflow after the last rescan round");
         case ah::kDevBadLeaf: return fail(AH_ERR_DEVICE, "leaf id out of range");
         case ah::kDevSelectSize: return fail(AH_ERR_DEVICE, "selection size mismatch (duplicate keys)");
+        case ah::kDevTimeout: return fail(AH_ERR_TIMEOUT, "a bounded wait in the tensor-core centroid scores gave up");
         default: return fail(AH_ERR_DEVICE, "device error " + std::to_string(code));
     }
 }
@@ -552,6 +644,10 @@ ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
         case AH_OPT_PROGRESSIVE_LEAVES:
             if (value < -1 || value > AH_MAX_LEAVES_SEARCHED) return fail(AH_ERR_INVALID_ARG, "progressive leaves outside [-1, 4096]");
             ix->opt_progressive_leaves = static_cast<int>(value);
+            return AH_OK;
+        case AH_OPT_UINT8_TENSOR_CORES:
+            if (value < 0 || value > 2) return fail(AH_ERR_INVALID_ARG, "uint8 tensor-core scan option outside [0, 2]");
+            ix->opt_u8_tensor = static_cast<int>(value);
             return AH_OK;
         case AH_OPT_SCAN_CHUNK_TILES:
             if (value < 0 || value > 1024) return fail(AH_ERR_INVALID_ARG, "scan chunk outside [0, 1024] tiles");
@@ -629,6 +725,7 @@ void ah_destroy(ah_index* ix) {
     cudaDeviceSynchronize();
     if (ix->ws.base) cudaFree(ix->ws.base);
     if (ix->codes_il) cudaFree(ix->codes_il);
+    if (ix->c_split) cudaFree(ix->c_split);
     if (ix->offs32) cudaFree(ix->offs32);
     if (ix->ptile) cudaFree(ix->ptile);
     if (ix->err) cudaFree(ix->err);
@@ -641,34 +738,6 @@ void ah_destroy(ah_index* ix) {
         for (int i = 0; i < ah_index::kMaxMarks; ++i) cudaEventDestroy(ix->ev[i]);
     delete ix;
 }
-
-// Scratch of ah_search_leaves_noalloc: the centroid score matrix and the
-// per-leaf counters of the partition stage, in a file-scope device array so
-// that the call never allocates.  Host code must not take this symbol's
-// address directly (on the host it is only a stand-in); the device address is
-// looked up once per device below.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[AH_NOALLOC_SCRATCH_BYTES];
-
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_dev_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (first call per
-// device does the lookup).
-ah_status noalloc_scratch(int device, void** out) {
-    if (device < 0 || device >= kMaxDevices) return fail(AH_ERR_UNSUPPORTED, "device ordinal beyond the scratch table");
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_dev_ptr[device]) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "scratch address lookup");
-        g_noalloc_dev_ptr[device] = p;
-    }
-    *out = g_noalloc_dev_ptr[device];
-    return AH_OK;
-}
-}  // namespace
 
 ah_status ah_search_leaves_noalloc(ah_index* ix, const float* queries, int32_t nq, int32_t L,
                                    int32_t* out_leaf_ids, float* out_leaf_scores, void* cuda_stream) {
@@ -685,15 +754,10 @@ ah_status ah_search_leaves_noalloc(ah_index* ix, const float* queries, int32_t n
     if (score_bytes + count_bytes + scanned_bytes > AH_NOALLOC_SCRATCH_BYTES)
         return fail(AH_ERR_UNSUPPORTED, "nq * num_leaves scores exceed the library's fixed scratch "
                                         "(AH_NOALLOC_SCRATCH_BYTES); split the batch");
-    int device = -1;
-    cudaError_t e = cudaGetDevice(&device);
-    if (e != cudaSuccess) return cuda_fail(e, "device query");
-    if (device != ix->device) return fail(AH_ERR_INVALID_ARG, "the index's device is not current");
-    void* base = nullptr;
-    ah_status st = noalloc_scratch(device, &base);
-    if (st != AH_OK) return st;
+    if (ah_status st = check_current_device(ix); st != AH_OK) return st;
+    cudaError_t e;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    char* p = static_cast<char*>(base);
+    char* p = static_cast<char*>(ix->noalloc_scratch);
     ah::SearchBuffers b{};
     b.cscore = reinterpret_cast<float*>(p);
     b.qcount = reinterpret_cast<int32_t*>(p + score_bytes);
@@ -956,6 +1020,25 @@ ah_status ah_kmeans_assign(const float* X, int64_t n, int32_t d, const float* C,
     if (d > AH_MAX_D) return fail(AH_ERR_UNSUPPORTED, "d above AH_MAX_D");
     const cudaError_t e = ah::launch_kmeans_assign(X, n, d, C, nl, assign, dist, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? AH_OK : cuda_fail(e, "k-means assignment");
+}
+
+ah_status ah_avq_update(const float* X, int64_t n, int32_t d, const int32_t* assign, int32_t nl, const float* C_old,
+                        double T, int32_t max_iters, double tol, float* C_new, int64_t* counts, int32_t* iters,
+                        void* cuda_stream) {
+    if (n < 0 || d < 1 || nl < 1) return fail(AH_ERR_INVALID_ARG, "n < 0, d < 1 or nl < 1");
+    if ((n > 0 && (!X || !assign)) || !C_old || !C_new) return fail(AH_ERR_INVALID_ARG, "NULL array");
+    if (max_iters < 0 || max_iters > 100000) return fail(AH_ERR_INVALID_ARG, "max_iters outside [0, 100000]");
+    if (!(tol >= 0.0 && tol < 1.0)) return fail(AH_ERR_INVALID_ARG, "tol outside [0, 1)");
+    if (ah::avq_solve_smem_bytes(d) > 200 * 1024) return fail(AH_ERR_UNSUPPORTED, "d above 6400 for the update");
+    if (n >= (int64_t(1) << 31)) return fail(AH_ERR_UNSUPPORTED, "n of 2^31 or more");
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    void* ws = nullptr;
+    cudaError_t e = cudaMallocAsync(&ws, ah::avq_workspace_bytes(n, nl), s);
+    if (e != cudaSuccess) return cuda_fail(e, "center update workspace");
+    e = ah::launch_avq_update(X, n, d, assign, nl, C_old, T, C_new, counts, iters, max_iters, tol, ws, s);
+    const cudaError_t ef = cudaFreeAsync(ws, s);
+    if (e != cudaSuccess) return cuda_fail(e, "anisotropic center update");
+    return ef == cudaSuccess ? AH_OK : cuda_fail(ef, "center update workspace release");
 }
 
 ah_status ah_kmeans_update(const float* X, int64_t n, int32_t d, const int32_t* assign, int32_t nl, const float* C_old,

@@ -16,6 +16,7 @@ enum DeviceError : int {
     kDevCandOverflow = 1,   // candidate buffer still overflowing after the last redo round
     kDevBadLeaf = 2,        // a leaf id outside [0, NL) reached the scan
     kDevSelectSize = 3,     // a selection asked for more items than it holds
+    kDevTimeout = 4,        // a bounded wait (tensor-core pipeline barrier) gave up
 };
 
 __device__ __forceinline__ void raise_error(int* err, int code) {

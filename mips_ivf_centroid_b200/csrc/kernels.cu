@@ -29,6 +29,13 @@
 #include "kernels.h"
 #include "select.cuh"
 
+#ifndef AH_SINGLE_GROUP
+#define AH_SINGLE_GROUP 1
+#endif
+#ifndef AH_CENTROID_TC
+#define AH_CENTROID_TC 1
+#endif
+
 namespace ah {
 
 // cudaFuncSetAttribute costs host time on every call; each kernel's dynamic
@@ -87,19 +94,24 @@ static cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 bloc
 // index preparation
 // ---------------------------------------------------------------------------
 
-// codes [n][cb] bytes -> il[tile][w][lane] 32-bit words.  Tiles are padded
-// per leaf: leaf c owns tiles ptile[c] .. ptile[c+1]-1, and lane l of its tile
-// t holds slot offs[c] + 32 (t - ptile[c]) + l (zero codes past the leaf's
-// end).  Word w holds code bytes 4w..4w+3.
+// codes [n][cb] bytes -> il[tile][W/V][lane][V] 32-bit words.  Tiles are
+// padded per leaf: leaf c owns tiles ptile[c] .. ptile[c+1]-1, and lane l of
+// its tile t holds slot offs[c] + 32 (t - ptile[c]) + l (zero codes past the
+// leaf's end).  Word w holds code bytes 4w..4w+3; a lane's words come in
+// groups of V consecutive words (V = 4, 2 or 1, the largest dividing W), so it
+// reads a group with one 16- or 8-byte load and a warp's load of a group is
+// 128 V contiguous bytes.
 __global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, const int32_t* __restrict__ offs,
-                                        const int32_t* __restrict__ ptile, int nl, int cb, int W,
+                                        const int32_t* __restrict__ ptile, int nl, int cb, int W, int V,
                                         uint32_t* __restrict__ il, int64_t total_words) {
     int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e >= total_words) return;
-    const int lane = static_cast<int>(e & 31);
-    const int64_t tw = e >> 5;                 // tile*W + w
-    const int w = static_cast<int>(tw % W);
-    const int tile = static_cast<int>(tw / W);
+    const int per_tile = W * 32;
+    const int tile = static_cast<int>(e / per_tile);
+    const int r = static_cast<int>(e - static_cast<int64_t>(tile) * per_tile);
+    const int grp = r / (32 * V), rem = r - grp * 32 * V;
+    const int lane = rem / V;
+    const int w = grp * V + (rem - lane * V);
     int lo = 0, hi = nl - 1;                   // leaf owning the tile: last c with ptile[c] <= tile
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
@@ -118,12 +130,21 @@ __global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, const
     il[e] = v;
 }
 
+#ifndef AH_MAX_CODE_V
+#define AH_MAX_CODE_V 4
+#endif
+int code_vector_words(int W) {
+    const int v = (W % 4 == 0) ? 4 : (W % 2 == 0) ? 2 : 1;
+    return v < AH_MAX_CODE_V ? v : AH_MAX_CODE_V;
+}
+
 cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, int nl, const uint8_t* codes, int cb,
                                  int W, int64_t ntiles, uint32_t* codes_il, cudaStream_t s) {
     const int64_t total = ntiles * W * 32;
     if (total == 0) return cudaSuccess;
     const int64_t grid = (total + 255) / 256;
-    interleave_codes_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, offs32, ptile, nl, cb, W, codes_il, total);
+    interleave_codes_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(codes, offs32, ptile, nl, cb, W,
+                                                                          code_vector_words(W), codes_il, total);
     return cudaGetLastError();
 }
 
@@ -301,6 +322,12 @@ __global__ void __launch_bounds__(256, 2) centroid_scores128_kernel(const float*
 // 128x128 tiles for large batches, 64x64 for mid-size ones, 32x32 for very
 // small problems (more CTAs in flight).
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
+    if (AH_CENTROID_TC && ix.c_hi && b.q_hi && centroid_tc_usable(a.nq, ix.nl, ix.d)) {
+        // tensor cores: the queries split into tf32 halves, then the tiles
+        cudaError_t e = launch_split_tf32(a.queries, static_cast<int64_t>(a.nq) * ix.d, b.q_hi, b.q_lo, s);
+        if (e != cudaSuccess) return e;
+        return launch_centroid_scores_tc(b.q_hi, b.q_lo, ix.c_hi, ix.c_lo, b.cscore, a.nq, ix.nl, ix.d, b.err, s);
+    }
     const int64_t big = static_cast<int64_t>((ix.nl + 63) / 64) * ((a.nq + 63) / 64);
     const int64_t tiles128 = static_cast<int64_t>((ix.nl + 127) / 128) * ((a.nq + 127) / 128);
     if (tiles128 >= 256) {                   // enough 128-wide tiles to fill every SM twice
@@ -419,13 +446,13 @@ __device__ int block_topk_reg(GetKey get, GetVal pay, int n, int K, RegSelectScr
     return K;
 }
 
-// One CTA per query with the score row in registers (KPL per thread): for
-// 1024 < centroids <= KPL * 256.
-template <int KPL>
-__global__ void __launch_bounds__(kSelThreads) top_leaves_reg_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+// One CTA of NT threads per query with the score row in registers (KPL per
+// thread): for 1024 < centroids <= KPL * NT.
+template <int KPL, int NT>
+__global__ void __launch_bounds__(NT) top_leaves_reg_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ RegSelectScratch<kSelThreads> rs;
+    __shared__ RegSelectScratch<NT> rs;
     __shared__ int s_count;
     __shared__ long long s_scanned;
     const int q = blockIdx.x;
@@ -435,9 +462,9 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_reg_kernel(DeviceIndex
     auto get = [&](int i) { return make_key(float_key(row[i]), i); };
     auto pay = [&](int i) { return i; };
     if (threadIdx.x == 0) s_scanned = 0;
-    block_topk_reg<KPL, kSelThreads>(get, pay, nl, L, rs, &s_count, keys, static_cast<int32_t*>(nullptr), true);
+    block_topk_reg<KPL, NT>(get, pay, nl, L, rs, &s_count, keys, static_cast<int32_t*>(nullptr), true);
     long long local = 0;
-    for (int i = threadIdx.x; i < L; i += kSelThreads) {
+    for (int i = threadIdx.x; i < L; i += NT) {
         const uint64_t key = keys[i];
         const int leaf = key_id(key);
         b.leaves[static_cast<int64_t>(q) * L + i] = leaf;
@@ -511,6 +538,7 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_2stage_kernel(DeviceIn
 }
 
 constexpr int kTopWarps = 8;
+constexpr int kTopRegWide = 1024;      // threads of the widest register top-L form
 
 // One warp per query when the centroids fit 32 per lane: the scores stay in
 // registers and the selection needs no shared-memory passes.
@@ -555,15 +583,22 @@ cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchB
         if (le != cudaSuccess) return le;
         return cudaGetLastError();
     }
-    if (ix.nl <= 16 * kSelThreads) {
+    if (ix.nl <= 16 * kSelThreads || (ix.nl <= 16 * kTopRegWide && a.nq <= 512)) {
+        // the score row in registers: 256 threads up to 4096 centroids, 1024
+        // threads (16 keys each) up to 16384 for batches of at most 512
+        // queries (larger batches of such rows ran faster in the
+        // shared-memory radix form: its CTAs are lighter and more fit an SM)
         const size_t smem = static_cast<size_t>(next_pow2(a.L)) * sizeof(uint64_t);
-        const void* fn = (ix.nl <= 8 * kSelThreads) ? reinterpret_cast<const void*>(top_leaves_reg_kernel<8>)
-                                                    : reinterpret_cast<const void*>(top_leaves_reg_kernel<16>);
+        const int form = (ix.nl <= 8 * kSelThreads) ? 0 : (ix.nl <= 16 * kSelThreads) ? 1 : 2;
+        const void* fn = form == 0 ? reinterpret_cast<const void*>(top_leaves_reg_kernel<8, kSelThreads>)
+                       : form == 1 ? reinterpret_cast<const void*>(top_leaves_reg_kernel<16, kSelThreads>)
+                                   : reinterpret_cast<const void*>(top_leaves_reg_kernel<16, kTopRegWide>);
         cudaError_t e = ensure_smem(fn, smem, false);
         if (e != cudaSuccess) return e;
-        const cudaError_t le = (ix.nl <= 8 * kSelThreads)
-            ? launch_chained(top_leaves_reg_kernel<8>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b)
-            : launch_chained(top_leaves_reg_kernel<16>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b);
+        const cudaError_t le =
+            form == 0 ? launch_chained(top_leaves_reg_kernel<8, kSelThreads>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b)
+          : form == 1 ? launch_chained(top_leaves_reg_kernel<16, kSelThreads>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b)
+                      : launch_chained(top_leaves_reg_kernel<16, kTopRegWide>, dim3(a.nq), dim3(kTopRegWide), smem, s, ix, a, b);
         if (le != cudaSuccess) return le;
         return cudaGetLastError();
     }
@@ -666,7 +701,8 @@ cudaError_t launch_invert(const DeviceIndex& ix, const SearchArgs& a, const Sear
         if (e != cudaSuccess) return e;
         if (const cudaError_t le = launch_chained(invert_count_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     }
-    if (const cudaError_t le = launch_chained(invert_offsets_kernel, dim3(1), dim3(kScanBlock), 0, s, ix, b, scan_group(ix, a.lut_mode), a.chunk); le != cudaSuccess) return le;
+    const int group = a.scan_tc ? scan_tc_group() : scan_group(ix, a.lut_mode);
+    if (const cudaError_t le = launch_chained(invert_offsets_kernel, dim3(1), dim3(kScanBlock), 0, s, ix, b, group, a.chunk); le != cudaSuccess) return le;
     if (const cudaError_t le = launch_chained(invert_scatter_kernel, dim3(grid), dim3(256), 0, s, a, b, r0, r1); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
@@ -756,15 +792,40 @@ cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchB
 // uint8: table as [B][16] bytes; returns the integer sum.
 // `pos` is the slot's position in the leaf-padded code copy.
 // With residual codes the leaf's centroid score `off` is added after the sum.
+// Offset of word w of lane `lane` within a tile of the code copy
+// ([W/V][32][V] words, V a power of two up to 4).
+__device__ __forceinline__ int code_word(int w, int lane, int V) {
+    const int r = w & (V - 1);
+    return (w - r) * 32 + lane * V + r;
+}
+
+// Words w .. w+3 of a lane (w a multiple of 4): one 16-byte load (V = 4), two
+// 8-byte loads (V = 2) or four 4-byte loads.
+__device__ __forceinline__ void code_words4(const uint32_t* __restrict__ tile, int lane, int w, int V, uint32_t& c0,
+                                            uint32_t& c1, uint32_t& c2, uint32_t& c3) {
+    if (V == 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + w * 32 + lane * 4);
+        c0 = v.x; c1 = v.y; c2 = v.z; c3 = v.w;
+    } else if (V == 2) {
+        const uint2 a = *reinterpret_cast<const uint2*>(tile + w * 32 + lane * 2);
+        const uint2 b = *reinterpret_cast<const uint2*>(tile + (w + 2) * 32 + lane * 2);
+        c0 = a.x; c1 = a.y; c2 = b.x; c3 = b.y;
+    } else {
+        c0 = tile[w * 32 + lane]; c1 = tile[(w + 1) * 32 + lane];
+        c2 = tile[(w + 2) * 32 + lane]; c3 = tile[(w + 3) * 32 + lane];
+    }
+}
+
 template <int MODE>
-__device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int B,
+__device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int V, int B,
                                                const unsigned char* lut, int32_t pos, bool add_off, float off) {
-    const uint32_t* cw = codes_il + (static_cast<int64_t>(pos >> 5) * W) * 32 + (pos & 31);
+    const uint32_t* tile = codes_il + (static_cast<int64_t>(pos >> 5) * W) * 32;
+    const int lane = pos & 31;
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
         float acc = 0.0f;
         for (int w = 0; w < W; ++w) {
-            uint32_t c = cw[w * 32];
+            uint32_t c = tile[code_word(w, lane, V)];
             int nb = min(8, B - 8 * w);
             for (int i = 0; i < nb; ++i) acc = __fadd_rn(acc, lf[(8 * w + i) * kCenters + ((c >> (4 * i)) & 15u)]);
         }
@@ -772,7 +833,7 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
     } else {
         uint32_t acc = 0;
         for (int w = 0; w < W; ++w) {
-            uint32_t c = cw[w * 32];
+            uint32_t c = tile[code_word(w, lane, V)];
             int nb = min(8, B - 8 * w);
             for (int i = 0; i < nb; ++i) acc += lut[(8 * w + i) * kCenters + ((c >> (4 * i)) & 15u)];
         }
@@ -781,66 +842,84 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
 }
 
 // Four slots at once (independent chains for latency hiding); each slot's sum
-// still runs over blocks in order, identical to slot_value.
+// still runs over blocks in order, identical to slot_value.  A slot's code
+// words are read four at a time (one 16-byte load where the copy's vector
+// width is 4), so a warp's loads for consecutive slots stay contiguous.
 template <int MODE>
-__device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int B,
+__device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int V, int B,
                                              const unsigned char* lut, const int32_t* pos, const bool* valid,
                                              const float* off, uint32_t* out) {
     const uint32_t* cw[4];
+    int ln[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int32_t sl = valid[u] ? pos[u] : 0;
-        cw[u] = codes_il + (static_cast<int64_t>(sl >> 5) * W) * 32 + (sl & 31);
+        cw[u] = codes_il + (static_cast<int64_t>(sl >> 5) * W) * 32;
+        ln[u] = sl & 31;
     }
-    // the next word of each slot is loaded while the current one is looked up
-    uint32_t nxt[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) nxt[u] = cw[u][0];
+    const int Wf = B >> 3, tail = B & 7;
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int w = 0; w < W; ++w) {
-            uint32_t c[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                c[u] = nxt[u];
-                if (w + 1 < W) nxt[u] = cw[u][(w + 1) * 32];
-            }
-            const int nb = min(8, B - 8 * w);
+        auto word = [&](int u, uint32_t c, int w, int nb) {
             const float* base = lf + 8 * w * kCenters;
-            if (nb == 8) {
+            for (int i = 0; i < nb; ++i) acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c >> (4 * i)) & 15u)]);
+        };
+        int w = 0;
+        for (; w + 4 <= Wf; w += 4) {
+            uint32_t c[4][4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) code_words4(cw[u], ln[u], w, V, c[u][0], c[u][1], c[u][2], c[u][3]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float* base = lf + 8 * (w + k) * kCenters;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u] >> (4 * i)) & 15u)]);
-            } else {
-                for (int i = 0; i < nb; ++i)
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u] >> (4 * i)) & 15u)]);
+                    for (int u = 0; u < 4; ++u)
+                        acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u][k] >> (4 * i)) & 15u)]);
             }
         }
+        for (; w < Wf; ++w)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) word(u, cw[u][code_word(w, ln[u], V)], w, 8);
+        if (tail)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) word(u, cw[u][code_word(Wf, ln[u], V)], Wf, tail);
 #pragma unroll
         for (int u = 0; u < 4; ++u) out[u] = float_key(off ? __fadd_rn(acc[u], off[u]) : acc[u]);
     } else {
         uint32_t acc[4] = {0u, 0u, 0u, 0u};
-        for (int w = 0; w < W; ++w) {
-            uint32_t c[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                c[u] = nxt[u];
-                if (w + 1 < W) nxt[u] = cw[u][(w + 1) * 32];
-            }
-            const int nb = min(8, B - 8 * w);
+        auto word = [&](int u, uint32_t c, int w, int nb) {
             const unsigned char* base = lut + 8 * w * kCenters;
-            for (int i = 0; i < nb; ++i)
+            for (int i = 0; i < nb; ++i) acc[u] += base[i * kCenters + ((c >> (4 * i)) & 15u)];
+        };
+        int w = 0;
+        for (; w + 4 <= Wf; w += 4) {
+            uint32_t c[4][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) acc[u] += base[i * kCenters + ((c[u] >> (4 * i)) & 15u)];
+            for (int u = 0; u < 4; ++u) code_words4(cw[u], ln[u], w, V, c[u][0], c[u][1], c[u][2], c[u][3]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) word(u, c[u][k], w + k, 8);
         }
+        for (; w < Wf; ++w)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) word(u, cw[u][code_word(w, ln[u], V)], w, 8);
+        if (tail)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) word(u, cw[u][code_word(Wf, ln[u], V)], Wf, tail);
 #pragma unroll
         for (int u = 0; u < 4; ++u) out[u] = acc[u];
     }
 }
 
+// One query's table in shared memory for the query-major kernels, where each
+// lane scores its own slot: fp32 [b][16] floats, uint8 [b][16] bytes.  (A
+// conflict-free layout with every fp32 entry twice measured slower in the
+// threshold kernel: the doubled table cost more in occupancy than the bank
+// conflicts did.)
 template <int MODE>
 __device__ __forceinline__ void load_query_table(const DeviceIndex& ix, const SearchBuffers& b, int q, unsigned char* lut) {
     const int per_q = ix.B * kCenters;
@@ -854,6 +933,7 @@ __device__ __forceinline__ void load_query_table(const DeviceIndex& ix, const Se
     }
 }
 
+// Shared memory of one query's table in the query-major kernels.
 __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
     return B * kCenters * (mode == 0 ? 4 : 1);
 }
@@ -872,7 +952,7 @@ constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query a
 // best can only be lower), so every point of the final top R has a key >= it.
 // With fewer than R points in total the bound is 0 (keep everything).
 template <int MODE>
-__global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+__global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ SelectScratch scr;
@@ -987,7 +1067,7 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
             sid[u] = ok[u] ? ix.slot_ids[seg_slot[lo] + off] : 0;
             off4[u] = seg_off[lo];
         }
-        slot_values4<MODE>(ix.codes_il, ix.W, ix.B, lut, ps, ok, ix.residual ? off4 : nullptr, v);
+        slot_values4<MODE>(ix.codes_il, ix.W, ix.V, ix.B, lut, ps, ok, ix.residual ? off4 : nullptr, v);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = t0 + u * kSelThreads + threadIdx.x;
@@ -1005,6 +1085,18 @@ __global__ void __launch_bounds__(kSelThreads, 8) threshold_kernel(DeviceIndex i
                 kk[j] = (i < taken) ? vals[i] : 0ull;
             }
             tau = block_kth_reg<4, kSelThreads>(kk, taken, R, rs);
+        }
+        if (threadIdx.x == 0) b.tau[q] = tau;
+    } else if (taken <= 8 * kSelThreads) {
+        uint64_t tau = 0ull;
+        if (taken >= R) {
+            uint64_t kk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = threadIdx.x + kSelThreads * j;
+                kk[j] = (i < taken) ? vals[i] : 0ull;
+            }
+            tau = block_kth_reg<8, kSelThreads>(kk, taken, R, rs);
         }
         if (threadIdx.x == 0) b.tau[q] = tau;
     } else {
@@ -1106,22 +1198,50 @@ __device__ __forceinline__ void f32_tail(uint32_t c, int nb, const float2* __res
     }
 }
 
-// uint8 tables staged as [b][G/4][16] words (4 queries' bytes per word); two
-// 16-bit lanes per accumulator (queries 4d+0/4d+2 in ae, 4d+1/4d+3 in ao).
-template <int G>
-__device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, const uint32_t* __restrict__ base, uint32_t (&ae)[G / 4],
-                                           uint32_t (&ao)[G / 4]) {
-    constexpr int BS = (G / 4) * kCenters;   // words per block
+// uint8 tables, two staged layouts.
+// SPLIT: [b][G/4][16] word pairs: for a quad of queries the entry's four bytes
+// already spread into two words of 16-bit lanes (queries 4d+0/4d+2 in .x,
+// 4d+1/4d+3 in .y), so a nibble costs one 8-byte load and two adds per quad;
+// 16 entries x 8 B of a (block, quad) cover the 32 banks once (one wavefront
+// per half-warp).  Used when a group's tables stay within 64 KB (B <= 256).
+// Packed: [b][G/4][16] words (4 queries' bytes per word), spread into the
+// 16-bit lanes after the load (mask and byte permute): half the shared memory,
+// for wider tables.  Both accumulate queries 4d+0/4d+2 in ae and 4d+1/4d+3 in ao.
+template <bool SPLIT>
+struct U8Layout {
+    using Entry = uint32_t;
+    __device__ __forceinline__ static void add(const Entry* p, uint32_t& ae, uint32_t& ao) {
+        const uint32_t v = *p;
+        ae += v & 0x00FF00FFu;
+        ao += __byte_perm(v, 0u, 0x4341);
+    }
+    __device__ __forceinline__ static Entry make(const uint32_t (&v)[4]) {
+        return v[0] | (v[1] << 8) | (v[2] << 16) | (v[3] << 24);
+    }
+};
+template <>
+struct U8Layout<true> {
+    using Entry = uint2;
+    __device__ __forceinline__ static void add(const Entry* p, uint32_t& ae, uint32_t& ao) {
+        const uint2 v = *p;
+        ae += v.x;
+        ao += v.y;
+    }
+    __device__ __forceinline__ static Entry make(const uint32_t (&v)[4]) {
+        return make_uint2(v[0] | (v[2] << 16), v[1] | (v[3] << 16));
+    }
+};
+
+template <int G, bool SPLIT>
+__device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, const typename U8Layout<SPLIT>::Entry* __restrict__ base,
+                                           uint32_t (&ae)[G / 4], uint32_t (&ao)[G / 4]) {
+    constexpr int BS = (G / 4) * kCenters;   // entries per block
 #pragma unroll
     for (int nib = 0; nib < 8; ++nib) {
         if (nib < nb) {
-            const uint32_t* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
+            const typename U8Layout<SPLIT>::Entry* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
 #pragma unroll
-            for (int qd = 0; qd < G / 4; ++qd) {
-                const uint32_t v = p[qd * kCenters];
-                ae[qd] += v & 0x00FF00FFu;
-                ao[qd] += __byte_perm(v, 0u, 0x4341);
-            }
+            for (int qd = 0; qd < G / 4; ++qd) U8Layout<SPLIT>::add(p + qd * kCenters, ae[qd], ao[qd]);
         }
     }
 }
@@ -1139,6 +1259,13 @@ __device__ __forceinline__ void u8_flush(uint32_t (&sums)[G], uint32_t (&ae)[G /
     }
 }
 
+// Shared-memory bytes per (query, block, center) of the scan's staged tables:
+// fp32 4; uint8 2 (each quad's bytes spread into 16-bit lanes) or 1.
+__host__ __device__ __forceinline__ int scan_entry_bytes(int mode, bool split) { return mode == 0 ? 4 : (split ? 2 : 1); }
+// uint8 tables use the split layout when a group of 8 queries' tables stays
+// within 64 KB that way
+__host__ __device__ __forceinline__ bool u8_split(int B) { return B * kCenters * 2 * kGroupU8 <= 64 * 1024; }
+
 struct TileJob {
     int t0, t1;          // code tiles [t0, t1) of one leaf
     int slot_base;       // slot of lane 0 of tile t is slot_base + 32 t
@@ -1155,26 +1282,26 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
                                                const uint32_t* s_tl, const float* s_off) {
     constexpr int BS = (G / 2) * kCenters;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
+    const int W = ix.W, V = ix.V, Wf = ix.B >> 3, tail = ix.B & 7;
     const float2* lut2 = reinterpret_cast<const float2*>(smem);
     for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
         const int slot = job.slot_base + 32 * t + lane;
         const bool valid = slot < job.send;
-        const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
+        const uint32_t* tw = ix.codes_il + static_cast<int64_t>(t) * W * 32;
         float2 acc[G / 2];
 #pragma unroll
         for (int pr = 0; pr < G / 2; ++pr) acc[pr] = make_float2(0.0f, 0.0f);
         int w = 0;
         for (; w + 4 <= Wf; w += 4) {
-            const uint32_t c0 = cwp[(w + 0) * 32], c1 = cwp[(w + 1) * 32];
-            const uint32_t c2 = cwp[(w + 2) * 32], c3 = cwp[(w + 3) * 32];
+            uint32_t c0, c1, c2, c3;
+            code_words4(tw, lane, w, V, c0, c1, c2, c3);
             f32_word<G>(c0, lut2 + (8 * w + 0) * BS, acc);
             f32_word<G>(c1, lut2 + (8 * w + 8) * BS, acc);
             f32_word<G>(c2, lut2 + (8 * w + 16) * BS, acc);
             f32_word<G>(c3, lut2 + (8 * w + 24) * BS, acc);
         }
-        for (; w < Wf; ++w) f32_word<G>(cwp[w * 32], lut2 + 8 * w * BS, acc);
-        if (tail) f32_tail<G>(cwp[Wf * 32], tail, lut2 + 8 * Wf * BS, acc);
+        for (; w < Wf; ++w) f32_word<G>(tw[code_word(w, lane, V)], lut2 + 8 * w * BS, acc);
+        if (tail) f32_tail<G>(tw[code_word(Wf, lane, V)], tail, lut2 + 8 * Wf * BS, acc);
 #pragma unroll
         for (int qi = 0; qi < G; ++qi) {
             if (qi < job.gsize) {
@@ -1187,18 +1314,18 @@ __device__ __forceinline__ void scan_tiles_f32(const DeviceIndex& ix, const Sear
     }
 }
 
-template <int G, int NT>
+template <int G, int NT, bool SPLIT>
 __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                               const TileJob& job, const int* s_q, const uint32_t* s_th,
                                               const uint32_t* s_tl) {
     constexpr int BS = (G / 4) * kCenters;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = ix.W, Wf = ix.B >> 3, tail = ix.B & 7;
-    const uint32_t* lutw = reinterpret_cast<const uint32_t*>(smem);
+    const int W = ix.W, V = ix.V, Wf = ix.B >> 3, tail = ix.B & 7;
+    const auto* lutw = reinterpret_cast<const typename U8Layout<SPLIT>::Entry*>(smem);
     for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
         const int slot = job.slot_base + 32 * t + lane;
         const bool valid = slot < job.send;
-        const uint32_t* cwp = ix.codes_il + static_cast<int64_t>(t) * W * 32 + lane;
+        const uint32_t* tw = ix.codes_il + static_cast<int64_t>(t) * W * 32;
         uint32_t sums[G];
         uint32_t ae[G / 4], ao[G / 4];
 #pragma unroll
@@ -1210,18 +1337,18 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
             const int wend = min(Wf, w0 + 32);
             int w = w0;
             for (; w + 4 <= wend; w += 4) {
-                const uint32_t c0 = cwp[(w + 0) * 32], c1 = cwp[(w + 1) * 32];
-                const uint32_t c2 = cwp[(w + 2) * 32], c3 = cwp[(w + 3) * 32];
-                u8_nibbles<G>(c0, 8, lutw + (8 * w + 0) * BS, ae, ao);
-                u8_nibbles<G>(c1, 8, lutw + (8 * w + 8) * BS, ae, ao);
-                u8_nibbles<G>(c2, 8, lutw + (8 * w + 16) * BS, ae, ao);
-                u8_nibbles<G>(c3, 8, lutw + (8 * w + 24) * BS, ae, ao);
+                uint32_t c0, c1, c2, c3;
+                code_words4(tw, lane, w, V, c0, c1, c2, c3);
+                u8_nibbles<G, SPLIT>(c0, 8, lutw + (8 * w + 0) * BS, ae, ao);
+                u8_nibbles<G, SPLIT>(c1, 8, lutw + (8 * w + 8) * BS, ae, ao);
+                u8_nibbles<G, SPLIT>(c2, 8, lutw + (8 * w + 16) * BS, ae, ao);
+                u8_nibbles<G, SPLIT>(c3, 8, lutw + (8 * w + 24) * BS, ae, ao);
             }
-            for (; w < wend; ++w) u8_nibbles<G>(cwp[w * 32], 8, lutw + 8 * w * BS, ae, ao);
+            for (; w < wend; ++w) u8_nibbles<G, SPLIT>(tw[code_word(w, lane, V)], 8, lutw + 8 * w * BS, ae, ao);
             u8_flush<G>(sums, ae, ao);
         }
         if (tail) {
-            u8_nibbles<G>(cwp[Wf * 32], tail, lutw + 8 * Wf * BS, ae, ao);
+            u8_nibbles<G, SPLIT>(tw[code_word(Wf, lane, V)], tail, lutw + 8 * Wf * BS, ae, ao);
             u8_flush<G>(sums, ae, ao);
         }
 #pragma unroll
@@ -1232,24 +1359,95 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
     }
 }
 
+// A group of one query (common when queries seldom share a leaf: small
+// batches, or many leaves): its table staged once, entries twice as for the
+// query-major kernels (fp32 [b][16][2], uint8 [b][16]), so each lookup is
+// useful and a warp's 32 lookups take one wavefront, instead of padding the
+// group to a pair (fp32) or a quad (uint8).  Blocks are summed in order.
+template <int NT, bool RES>
+__device__ __forceinline__ void scan_tiles_f32_single(const DeviceIndex& ix, const SearchBuffers& b,
+                                                      const unsigned char* smem, const TileJob& job, const int* s_q,
+                                                      const uint32_t* s_th, const uint32_t* s_tl, const float* s_off) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = ix.W, V = ix.V, Wf = ix.B >> 3, tail = ix.B & 7;
+    const float* lut1 = reinterpret_cast<const float*>(smem) + ((lane >> 4) & 1);
+    auto word = [&](uint32_t c, int nb, const float* base, float& acc) {
+#pragma unroll
+        for (int nib = 0; nib < 8; ++nib)
+            if (nib < nb) acc = __fadd_rn(acc, base[2 * (nib * kCenters + ((c >> (4 * nib)) & 15u))]);
+    };
+    for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
+        const int slot = job.slot_base + 32 * t + lane;
+        const bool valid = slot < job.send;
+        const uint32_t* tw = ix.codes_il + static_cast<int64_t>(t) * W * 32;
+        float acc = 0.0f;
+        int w = 0;
+        for (; w + 4 <= Wf; w += 4) {
+            uint32_t c0, c1, c2, c3;
+            code_words4(tw, lane, w, V, c0, c1, c2, c3);
+            word(c0, 8, lut1 + 2 * (8 * w + 0) * kCenters, acc);
+            word(c1, 8, lut1 + 2 * (8 * w + 8) * kCenters, acc);
+            word(c2, 8, lut1 + 2 * (8 * w + 16) * kCenters, acc);
+            word(c3, 8, lut1 + 2 * (8 * w + 24) * kCenters, acc);
+        }
+        for (; w < Wf; ++w) word(tw[code_word(w, lane, V)], 8, lut1 + 2 * 8 * w * kCenters, acc);
+        if (tail) word(tw[code_word(Wf, lane, V)], tail, lut1 + 2 * 8 * Wf * kCenters, acc);
+        const float sc = RES ? __fadd_rn(acc, s_off[0]) : acc;
+        keep_if_reaches(valid, float_key(sc), slot, 0, s_q, s_th, s_tl, ix, b);
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void scan_tiles_u8_single(const DeviceIndex& ix, const SearchBuffers& b,
+                                                     const unsigned char* smem, const TileJob& job, const int* s_q,
+                                                     const uint32_t* s_th, const uint32_t* s_tl) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = ix.W, V = ix.V, Wf = ix.B >> 3, tail = ix.B & 7;
+    auto word = [&](uint32_t c, int nb, const unsigned char* base, uint32_t& acc) {
+#pragma unroll
+        for (int nib = 0; nib < 8; ++nib)
+            if (nib < nb) acc += base[nib * kCenters + ((c >> (4 * nib)) & 15u)];
+    };
+    for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
+        const int slot = job.slot_base + 32 * t + lane;
+        const bool valid = slot < job.send;
+        const uint32_t* tw = ix.codes_il + static_cast<int64_t>(t) * W * 32;
+        uint32_t acc = 0u;
+        int w = 0;
+        for (; w + 4 <= Wf; w += 4) {
+            uint32_t c0, c1, c2, c3;
+            code_words4(tw, lane, w, V, c0, c1, c2, c3);
+            word(c0, 8, smem + (8 * w + 0) * kCenters, acc);
+            word(c1, 8, smem + (8 * w + 8) * kCenters, acc);
+            word(c2, 8, smem + (8 * w + 16) * kCenters, acc);
+            word(c3, 8, smem + (8 * w + 24) * kCenters, acc);
+        }
+        for (; w < Wf; ++w) word(tw[code_word(w, lane, V)], 8, smem + 8 * w * kCenters, acc);
+        if (tail) word(tw[code_word(Wf, lane, V)], tail, smem + 8 * Wf * kCenters, acc);
+        keep_if_reaches(valid, acc, slot, 0, s_q, s_th, s_tl, ix, b);
+    }
+}
+
 // Persistent CTAs take work items (leaf, query group, chunk of code tiles) from
 // an atomic counter.  A leaf's m queries form groups of GMAX, then one group of
-// the remainder rounded up to GSTEP, so at most GSTEP-1 table slots of a leaf
-// are padding.  Per item the group's tables are staged in shared memory
-// (fp32 pair-interleaved, uint8 quad-interleaved) and the warps scan the
+// the remainder rounded up to GSTEP (a lone query stays a group of one), so
+// at most GSTEP-1 table slots of a leaf are padding.  Per item the group's
+// tables are staged in shared memory (fp32 pair-interleaved, uint8
+// quad-interleaved and spread into 16-bit lanes) and the warps scan the
 // chunk's tiles.  Only a leaf's last tile is partial (leaf-padded code copy).
 #ifndef AH_SCAN_MIN_BLOCKS
 #define AH_SCAN_MIN_BLOCKS 6
 #endif
-// uint8 scan: 6 CTAs per SM as for fp32 (groups of 8 queries keep 12
-// accumulator registers per lane, leaving room for loads in flight)
+// uint8 scan: 5 CTAs per SM (48 registers: groups of 8 queries keep 12
+// accumulator registers per lane plus 8-byte table loads; at 40 the compiler
+// spills)
 #ifndef AH_SCAN_MIN_BLOCKS_U8
-#define AH_SCAN_MIN_BLOCKS_U8 6
+#define AH_SCAN_MIN_BLOCKS_U8 5
 #endif
 
 // RES: residual codes (each query's centroid score of the leaf is added to its
 // sums); a separate instantiation so plain indexes pay nothing for it.
-template <int MODE, int NT, int GMAX, bool RES>
+template <int MODE, int NT, int GMAX, bool RES, bool SPLIT>
 __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOCKS : AH_SCAN_MIN_BLOCKS_U8)
                                                  : (NT == 512 ? 2 : 1)))
     scan_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
@@ -1262,17 +1460,24 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
     __shared__ float s_off[GMAX];            // residual codes: each query's score of this leaf
     const int B = ix.B;
     const int total_items = b.item_off[ix.nl];
-    const size_t lut_bytes = static_cast<size_t>(B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
+    const size_t lut_bytes = static_cast<size_t>(B) * GMAX * kCenters * scan_entry_bytes(MODE, SPLIT);
     int* s_item_off = reinterpret_cast<int*>(smem + lut_bytes);
     const bool off_in_smem = a.scan_item_off_smem != 0;
     if (off_in_smem)
         for (int i = threadIdx.x; i <= ix.nl; i += NT) s_item_off[i] = b.item_off[i];
     const int* item_off = off_in_smem ? s_item_off : b.item_off;
 
+    // 256-thread form (short items): the next item's index is claimed while
+    // the current one is scanned, so the atomic's latency is hidden (thread 0
+    // holds it in `next`).  The wide forms' items are long; they claim items
+    // as they go (the extra register would spill there).
+    constexpr bool kPrefetch = NT == 256;
+    int next = 0;
+    if (kPrefetch && threadIdx.x == 0) next = atomicAdd(&b.counters[a.scan_counter], 1);
     for (;;) {
         __syncthreads();   // previous item's tables are no longer read
         if (threadIdx.x == 0) {
-            int item = atomicAdd(&b.counters[a.scan_counter], 1);
+            const int item = kPrefetch ? next : atomicAdd(&b.counters[a.scan_counter], 1);
             s_item = item;
             if (item < total_items) {
                 int lo = 0, hi = ix.nl;
@@ -1286,6 +1491,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
         __syncthreads();
         const int item = s_item;
         if (item >= total_items) break;
+        if (kPrefetch && threadIdx.x == 0) next = atomicAdd(&b.counters[a.scan_counter], 1);
         const int leaf = s_leaf;
         const int pt0 = ix.ptile[leaf], ntile = ix.ptile[leaf + 1] - pt0;
         const int npc = (ntile + a.chunk - 1) / a.chunk;
@@ -1294,7 +1500,8 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
         const int qcnt = b.qcount[leaf];
         TileJob job;
         job.gsize = min(GMAX, qcnt - g * GMAX);
-        const int G = ((job.gsize + GSTEP - 1) / GSTEP) * GSTEP;   // table width of this group
+        // table width of this group (a lone query is not padded)
+        const int G = (AH_SINGLE_GROUP && job.gsize == 1) ? 1 : ((job.gsize + GSTEP - 1) / GSTEP) * GSTEP;
         job.t0 = pt0 + c * a.chunk;
         job.t1 = min(pt0 + ntile, job.t0 + a.chunk);
         job.slot_base = ix.offs[leaf] - 32 * pt0;
@@ -1310,7 +1517,17 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
         __syncthreads();
         // stage the group's tables
         const int per_q = B * kCenters;
-        if (MODE == 0) {
+        if (G == 1) {
+            const int q0 = s_q[0];
+            if (MODE == 0) {
+                float2* lf = reinterpret_cast<float2*>(smem);
+                const float* src = b.lut_f32 + static_cast<int64_t>(q0) * per_q;
+                for (int r = threadIdx.x; r < per_q; r += NT) lf[r] = make_float2(src[r], src[r]);
+            } else {
+                const uint8_t* src = b.lut_u8 + static_cast<int64_t>(q0) * per_q;
+                for (int r = threadIdx.x; r < per_q; r += NT) smem[r] = src[r];
+            }
+        } else if (MODE == 0) {
             // one 8-byte store per (block, center) of each query pair
             float2* lf = reinterpret_cast<float2*>(smem);
             const int half = G / 2;
@@ -1325,8 +1542,8 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
                 }
             }
         } else {
-            // one 4-byte store per (block, center) of each query quad
-            uint32_t* lw = reinterpret_cast<uint32_t*>(smem);
+            // one store per (block, center) of each query quad
+            auto* lw = reinterpret_cast<typename U8Layout<SPLIT>::Entry*>(smem);
             const int quads = G / 4;
             for (int qd = 0; qd < quads; ++qd) {
                 const uint8_t* src[4];
@@ -1338,16 +1555,18 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
                     src[u] = b.lut_u8 + static_cast<int64_t>(ok[u] ? qq : 0) * per_q;
                 }
                 for (int r = threadIdx.x; r < per_q; r += NT) {
-                    uint32_t v = 0u;
+                    uint32_t v[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (ok[u]) v |= static_cast<uint32_t>(src[u][r]) << (8 * u);
-                    lw[((r >> 4) * quads + qd) * kCenters + (r & 15)] = v;
+                    for (int u = 0; u < 4; ++u) v[u] = ok[u] ? static_cast<uint32_t>(src[u][r]) : 0u;
+                    lw[((r >> 4) * quads + qd) * kCenters + (r & 15)] = U8Layout<SPLIT>::make(v);
                 }
             }
         }
         __syncthreads();
-        if (MODE == 0) {
+        if (G == 1) {
+            if (MODE == 0) scan_tiles_f32_single<NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off);
+            else scan_tiles_u8_single<NT>(ix, b, smem, job, s_q, s_th, s_tl);
+        } else if (MODE == 0) {
             switch (G) {
                 case 8: scan_tiles_f32<8, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
                 case 6: scan_tiles_f32<6, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
@@ -1355,12 +1574,8 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
                 default: scan_tiles_f32<2, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
             }
         } else {
-            switch (G) {
-                case 16: scan_tiles_u8<16, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 12: scan_tiles_u8<12, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                case 8: scan_tiles_u8<8, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-                default: scan_tiles_u8<4, NT>(ix, b, smem, job, s_q, s_th, s_tl); break;
-            }
+            if (GMAX >= 8 && G == 8) scan_tiles_u8<(GMAX >= 8 ? 8 : 4), NT, SPLIT>(ix, b, smem, job, s_q, s_th, s_tl);
+            else scan_tiles_u8<4, NT, SPLIT>(ix, b, smem, job, s_q, s_th, s_tl);
         }
     }
 }
@@ -1370,14 +1585,14 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
 // (fp32 and uint8), several CTAs per SM.  Wide tables (half a group within
 // 100 KB): two CTAs of 512 threads per SM with half-size groups, so one
 // CTA's table staging and item-end barrier overlap the other's scanning.
-// Wider fp32 tables (B 401-452): one CTA of 1,024 threads, groups of 8; the
-// search refuses fp32 tables beyond that.
+// Wider tables: one CTA of 1,024 threads, fp32 groups of 8 (B 401-452; the
+// search refuses fp32 tables beyond that), uint8 groups of 4.
 #ifndef AH_WIDE_SPLIT
 #define AH_WIDE_SPLIT 1
 #endif
 void scan_shape(const DeviceIndex& ix, int lut_mode, int* nt, int* gmax) {
     const int g = lut_mode == 0 ? kGroupF32 : kGroupU8;
-    const size_t table = static_cast<size_t>(ix.B) * kCenters * (lut_mode == 0 ? 4 : 1) * g;
+    const size_t table = static_cast<size_t>(ix.B) * kCenters * scan_entry_bytes(lut_mode, u8_split(ix.B)) * g;
     if (table <= 64 * 1024) {
         *nt = 256;
         *gmax = g;
@@ -1385,8 +1600,10 @@ void scan_shape(const DeviceIndex& ix, int lut_mode, int* nt, int* gmax) {
         *nt = 512;
         *gmax = g / 2;
     } else {
+        // one CTA of 1,024 threads per SM: fp32 groups of 8 (B <= 452);
+        // uint8 groups of 4, which fit every B up to AH_MAX_BLOCKS
         *nt = 1024;
-        *gmax = g;
+        *gmax = lut_mode == 0 ? g : g / 2;
     }
 }
 
@@ -1399,28 +1616,29 @@ int scan_group(const DeviceIndex& ix, int lut_mode) {
 size_t scan_table_bytes(const DeviceIndex& ix, int lut_mode) {
     int nt, g;
     scan_shape(ix, lut_mode, &nt, &g);
-    return static_cast<size_t>(ix.B) * g * kCenters * (lut_mode == 0 ? 4 : 1);
+    return static_cast<size_t>(ix.B) * g * kCenters * scan_entry_bytes(lut_mode, u8_split(ix.B));
 }
 
-template <int MODE, int NT, int GMAX, bool RES>
+template <int MODE, int NT, int GMAX, bool RES, bool SPLIT = false>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
-    size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * (MODE == 0 ? 4 : 1);
+    size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * scan_entry_bytes(MODE, SPLIT);
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
     const size_t room = (NT == 512) ? 110 * 1024 : 200 * 1024;
     a.scan_item_off_smem = (smem + off_bytes <= room && off_bytes <= 64 * 1024) ? 1 : 0;
     if (a.scan_item_off_smem) smem += off_bytes;
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT, GMAX, RES>), smem, true);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(scan_kernel<MODE, NT, GMAX, RES, SPLIT>), smem, true);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT, GMAX, RES>, NT, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<MODE, NT, GMAX, RES, SPLIT>, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT, GMAX, RES>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
+    if (const cudaError_t le = launch_chained(scan_kernel<MODE, NT, GMAX, RES, SPLIT>, dim3(num_sms * per_sm), dim3(NT), smem, s, ix, a, b); le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s) {
+    if (a.scan_tc) return launch_scan_tc(ix, a, b, num_sms, s);
     int nt, g;
     scan_shape(ix, a.lut_mode, &nt, &g);
     if (a.lut_mode == 0) {
@@ -1434,9 +1652,10 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
         return launch_scan_t<0, 1024, kGroupF32, false>(ix, a, b, num_sms, s);
     }
     // uint8 tables are refused for residual codes before any launch
+    if (u8_split(ix.B)) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
     if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
     if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
-    return launch_scan_t<1, 1024, kGroupU8, false>(ix, a, b, num_sms, s);
+    return launch_scan_t<1, 1024, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -1550,7 +1769,7 @@ __global__ void __launch_bounds__(kSelThreads) redo_scan_kernel(DeviceIndex ix, 
         for (int base = s0; base < s1; base += kSelThreads) {
             const int slot = base + threadIdx.x;
             const bool in = slot < s1;
-            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.B, smem, slot + p0, ix.residual != 0, off)
+            const uint32_t v = in ? slot_value<MODE>(ix.codes_il, ix.W, ix.V, ix.B, smem, slot + p0, ix.residual != 0, off)
                                   : 0u;
             append_candidates(in && reaches(v, th, tl, ix.slot_ids, slot), v, slot, q, ix, b);
         }
@@ -1760,7 +1979,34 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
                 // the multiply-adds (same accumulation order), so a lane waits
                 // for memory once per batch rather than once per load.
                 const int n4 = d / 4;
-                if (ix.reorder_bf16) {
+                if (ix.reorder_bf16 && a.reorder_vec4 == 2) {
+                    // bfloat16 rows, d % 8 == 0: 16-byte loads of 8 values
+                    const uint4* v = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d);
+                    const int n8 = d / 8;
+                    for (int t0 = gl; t0 < n8; t0 += kReorderBatch * lpc) {
+                        uint4 h[kReorderBatch];
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            h[u] = (t < n8) ? v[t] : make_uint4(0u, 0u, 0u, 0u);
+                        }
+#pragma unroll
+                        for (int u = 0; u < kReorderBatch; ++u) {
+                            const int t = t0 + u * lpc;
+                            if (t < n8) {
+                                const float4 x0 = q4[2 * t], x1 = q4[2 * t + 1];
+                                acc = fmaf(x0.x, __uint_as_float(h[u].x << 16), acc);
+                                acc = fmaf(x0.y, __uint_as_float(h[u].x & 0xFFFF0000u), acc);
+                                acc = fmaf(x0.z, __uint_as_float(h[u].y << 16), acc);
+                                acc = fmaf(x0.w, __uint_as_float(h[u].y & 0xFFFF0000u), acc);
+                                acc = fmaf(x1.x, __uint_as_float(h[u].z << 16), acc);
+                                acc = fmaf(x1.y, __uint_as_float(h[u].z & 0xFFFF0000u), acc);
+                                acc = fmaf(x1.z, __uint_as_float(h[u].w << 16), acc);
+                                acc = fmaf(x1.w, __uint_as_float(h[u].w & 0xFFFF0000u), acc);
+                            }
+                        }
+                    }
+                } else if (ix.reorder_bf16) {
                     const uint2* v = reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(ix.reorder_vecs) + slot * d);
                     for (int t0 = gl; t0 < n4; t0 += kReorderBatch * lpc) {
                         uint2 h[kReorderBatch];
@@ -1887,7 +2133,8 @@ cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffe
                           cudaStream_t s) {
     const uintptr_t qa = reinterpret_cast<uintptr_t>(a.queries), va = reinterpret_cast<uintptr_t>(ix.reorder_vecs);
     a.reorder_vec4 = (ix.d % 4 == 0 && qa % 16 == 0 && va % 16 == 0) ? 1 : 0;
-    a.reorder_lanes = lanes_per_candidate(ix.d);
+    if (a.reorder_vec4 && ix.reorder_bf16 && ix.d % 8 == 0) a.reorder_vec4 = 2;   // 16-byte bf16 loads
+    a.reorder_lanes = lanes_per_candidate(a.reorder_vec4 == 2 ? ix.d / 2 : ix.d);
     const size_t smem = finish_smem_bytes(a.R, ix.d);
     const unsigned grid = (round == 0) ? static_cast<unsigned>(a.nq) : static_cast<unsigned>(std::min(a.nq, 2 * num_sms));
     cudaError_t e;

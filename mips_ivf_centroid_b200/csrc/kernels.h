@@ -30,12 +30,15 @@ __host__ __device__ __forceinline__ int threshold_sample(int R, int requested) {
 struct DeviceIndex {
     int64_t n;
     int d, nl, dpb, B, W;                 // W: 32-bit code words per point
+    int V;                                // words per lane per vector load of the code copy (4, 2 or 1)
     const float* centroids;               // [NL][d]
     const int32_t* offs;                  // [NL+1] int32 leaf offsets (owned copy)
     const int32_t* ptile;                 // [NL+1] first code tile of each leaf (leaf-padded copy)
     const int32_t* slot_ids;              // [n]
-    const uint32_t* codes_il;             // [ptile[NL]][W][32] leaf-padded tiles (owned)
+    const uint32_t* codes_il;             // [ptile[NL]][W/V][32][V] leaf-padded tiles (owned)
     const float* codebook;                // [B][16][dpb]
+    const float* c_hi;                    // [NL][d] centroids split for the tensor cores (owned; or null)
+    const float* c_lo;                    // [NL][d]
     const void* reorder_vecs;             // [n][d]
     int reorder_bf16;
     int residual;                         // codes quantise x - its leaf's centroid: scores add q . centroid
@@ -44,6 +47,8 @@ struct DeviceIndex {
 struct SearchBuffers {
     // per query
     float* cscore;          // [nq][NL]
+    float* q_hi;            // [nq][d] queries split for the tensor cores (or null: SIMT tiles)
+    float* q_lo;            // [nq][d]
     int32_t* leaves;        // [nq][L]
     float* leaf_scores;     // [nq][L]
     int64_t* scanned;       // [nq]
@@ -89,15 +94,19 @@ struct SearchArgs {
     int32_t* tr_rescans;
     int scan_item_off_smem;     // set by the scan launcher
     int topl_row_smem;          // set by the top-leaves launcher
-    int reorder_vec4;           // set by the finish launcher: 16-byte vector loads allowed
+    int reorder_vec4;           // set by the finish launcher: 16-byte vector loads of 4 floats (1) or
+                                // of 8 bfloat16 values (2) allowed
     int reorder_lanes;          // set by the finish launcher: lanes per rescored candidate
     int threshold_sample;       // slots sampled per query for the filter bound (requested)
     int threshold_leaves;       // best leaves the sample is spread over
     int scan_counter;           // index into counters[] of the scan's work counter
     int count_ranks;            // top-L kernel counts queries per leaf for ranks below this
+    int scan_tc;                // uint8 tables: scan on the int8 tensor cores (items of up to 128
+                                // queries x 256 points) instead of table lookups
 };
 
-// Build-time: the leaf-padded tiled code copy.
+// Build-time: the leaf-padded tiled code copy; V = code_vector_words(W).
+int code_vector_words(int W);
 cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, int nl, const uint8_t* codes, int cb,
                                  int W, int64_t ntiles, uint32_t* codes_il, cudaStream_t s);
 
@@ -134,6 +143,27 @@ cudaError_t launch_kmeans_assign(const float* X, int64_t n, int d, const float* 
 size_t kmeans_update_smem_bytes(int d);
 cudaError_t launch_kmeans_update(const float* X, int64_t n, int d, const int32_t* assign, int nl, const float* C_old,
                                  float* C_new, int64_t* counts, cudaStream_t s);
+
+// closed-form anisotropic center update (avq.cu)
+size_t avq_solve_smem_bytes(int d);
+size_t avq_workspace_bytes(int64_t n, int nl);
+cudaError_t launch_avq_update(const float* X, int64_t n, int d, const int32_t* assign, int nl, const float* C_old,
+                              double T, float* C_new, int64_t* counts, int32_t* iters, int max_iters, double tol,
+                              void* workspace, cudaStream_t s);
+
+// uint8-table scan on the int8 tensor cores (scan_tc.cu)
+int scan_tc_group();
+int scan_tc_chunk_tiles();
+size_t scan_tc_smem_bytes();
+cudaError_t launch_scan_tc(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms,
+                           cudaStream_t s);
+
+// centroid scores on the tensor cores (centroid_tc.cu)
+bool centroid_tc_usable(int nq, int nl, int d);
+size_t centroid_tc_smem_bytes();
+cudaError_t launch_split_tf32(const float* x, int64_t n, float* hi, float* lo, cudaStream_t s);
+cudaError_t launch_centroid_scores_tc(const float* q_hi, const float* q_lo, const float* c_hi, const float* c_lo,
+                                      float* S, int nq, int nl, int d, int* err, cudaStream_t s);
 
 // exact merge of per-shard candidates (merge.cu)
 cudaError_t launch_merge_shards(int G, int nq, int R, int k, const int32_t* ids, const float* approx,

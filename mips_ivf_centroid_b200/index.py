@@ -83,6 +83,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "ah_encode": (I32, [P, I64, I32, I32, P, ctypes.c_double, I32, P, P, P]),
         "ah_kmeans_assign": (I32, [P, I64, I32, P, I32, P, P, P]),
         "ah_kmeans_update": (I32, [P, I64, I32, P, I32, P, P, P, P]),
+        "ah_avq_update": (I32, [P, I64, I32, P, I32, P, ctypes.c_double, I32, ctypes.c_double, P, P, P, P]),
         "ah_save": (I32, [P, ctypes.c_char_p]),
         "ah_merge_shards": (I32, [I32, I32, I32, I32, P, P, P, P, P, P]),
         "ah_inspect": (I32, [ctypes.c_char_p, P]),
@@ -223,6 +224,30 @@ def kmeans_update(X: torch.Tensor, assign: torch.Tensor, C_old: torch.Tensor, st
         _check(lib, lib.ah_kmeans_update(_ptr(X), n, d, _ptr(assign), nl, _ptr(C_old), _ptr(C_new), _ptr(counts),
                                          _stream(stream)))
     return C_new, counts
+
+
+def avq_update(X: torch.Tensor, assign: torch.Tensor, C_old: torch.Tensor, T: float, max_iters: int = 200,
+               tol: float = 1e-14, stream=None):
+    """Anisotropic center update over each center's members (``ah_avq_update``):
+    (C_new [nl, d] float32, counts [nl] int64, iters [nl] int32), asynchronous
+    on the stream.  eta per point from the threshold T and the point's norm."""
+    lib = load_library()
+    _f32_2d(X, "X")
+    _f32_2d(C_old, "C_old", X.device)
+    if assign.dtype != torch.int32 or assign.dim() != 1 or assign.shape[0] != X.shape[0] \
+            or assign.device != X.device or not assign.is_contiguous():
+        raise AhError(1, "assign: need contiguous int32 [n] on X's device")
+    n, d = X.shape
+    if C_old.shape[1] != d:
+        raise AhError(1, "C_old: need [nl, d] with X's d")
+    nl = C_old.shape[0]
+    C_new = torch.empty_like(C_old)
+    counts = torch.empty((nl,), dtype=torch.int64, device=X.device)
+    iters = torch.empty((nl,), dtype=torch.int32, device=X.device)
+    with torch.cuda.device(X.device):
+        _check(lib, lib.ah_avq_update(_ptr(X), n, d, _ptr(assign), nl, _ptr(C_old), float(T), int(max_iters),
+                                      float(tol), _ptr(C_new), _ptr(counts), _ptr(iters), _stream(stream)))
+    return C_new, counts, iters
 
 
 def merge_shards(cand_ids: torch.Tensor, cand_approx: torch.Tensor, cand_exact: Optional[torch.Tensor], k: int,
@@ -412,6 +437,7 @@ class Index:
     OPT_SCAN_CHUNK_TILES = 2
     OPT_THRESHOLD_LEAVES = 3
     OPT_PROGRESSIVE_LEAVES = 4
+    OPT_UINT8_TENSOR_CORES = 5
 
     def set_option(self, option: int, value: int):
         """Tuning knob (ah_set_option): results are unchanged, only speed."""

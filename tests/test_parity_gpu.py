@@ -6,19 +6,18 @@ Each search is compared stage by stage on the same seeded inputs:
               tolerance; uint8 mode: ids, integer sums and fp32 scores
               bit-exact);
   final       ranked match with the oracle's exact (or approximate) scores.
-A query whose leaf set differs from the oracle's (only possible through a
-near-tie at the L-th leaf, which the ranked match checks) is checked for
-validity downstream instead of equality; likewise for a near-tie at the R-th
-candidate.  Such queries must stay rare.
+Every query is checked through every stage: one whose leaf set differs from
+the oracle's (a near-tie at the L-th leaf, which the ranked match allows) has
+its later stages compared with the oracle run over the GPU's leaves; one whose
+candidate set differs through a near-tie at the R-th candidate must return the
+best k of its own candidates.  Such swaps must stay rare.
 """
 import numpy as np
 import pytest
 import torch
 
 from mips_ivf_centroid_b200 import datagen
-from oracle import OracleIndex
-
-from parity import ranked_match, same_set
+from parity import compare_search
 
 pytestmark = pytest.mark.gpu
 
@@ -46,11 +45,18 @@ def _workload(name):
                                          n_means=100, training_sample_size=30_000),
         "leaves-5000": W["glove"].scaled(n=50_000, d=32, num_leaves=5000, num_leaves_to_search=16, nq=128,
                                          n_means=100, training_sample_size=50_000),
+        "leaves-20000": W["glove"].scaled(n=100_000, d=16, num_leaves=20_000, num_leaves_to_search=40, nq=96,
+                                          n_means=200, training_sample_size=100_000, code_loss="l2",
+                                          threshold_T=None),
         "gemm128-vec": W["glove"].scaled(n=40_000, d=64, num_leaves=2048, num_leaves_to_search=8, nq=2048,
                                          n_means=100, training_sample_size=40_000),
         "gemm128-scalar": W["glove"].scaled(n=40_000, d=34, dims_per_block=1, num_leaves=2048,
                                             num_leaves_to_search=8, nq=2048, n_means=100,
                                             training_sample_size=40_000),
+        "tc-ragged": W["glove"].scaled(n=60_000, d=36, num_leaves=3500, num_leaves_to_search=8, nq=300,
+                                       n_means=150, training_sample_size=60_000, code_loss="l2", threshold_T=None),
+        "tc-integer": W["bigann"].scaled(n=100_000, num_leaves=2000, num_leaves_to_search=16, nq=600,
+                                         n_means=400, training_sample_size=100_000),
         "glove-mini-residual": W["glove"].scaled(n=60_000, num_leaves=300, num_leaves_to_search=24, nq=300,
                                                  n_means=120, training_sample_size=60_000, residual=True),
         "tiny-leaves": W["glove"].scaled(n=3_000, d=16, num_leaves=2000, num_leaves_to_search=1500, nq=32,
@@ -78,62 +84,15 @@ def Index():
 
 def compare(Index, name, k, L, reorder_num, lut_mode, max_leaf_mismatch=0.02, max_cand_mismatch=0.05,
             qsel=None):
+    """Search the case's queries (or the rows ``qsel`` of them) as one batch and
+    check every query stage by stage against the oracle (parity.compare_search)."""
     w, X, Q, ix, arr = _workload(name)
     index = Index(ix)
     Qs = Q if qsel is None else Q[qsel]
-    qg = torch.from_numpy(Qs).cuda()
-    ids, scores, tr = index.search(qg, k, L, reorder_num, lut_mode, trace=True)
-    index.sync_status()
-    ids, scores = ids.cpu().numpy(), scores.cpu().numpy()
-    tr = {kk: v.cpu().numpy() for kk, v in tr.items()}
-    orc = OracleIndex(arr)
-    o = orc.search(Qs, k, L, reorder_num, lut_mode)
-    inv = np.empty(w.n, np.int64)
-    inv[arr["slot_ids"]] = np.arange(w.n)
-    nq = Qs.shape[0]
-    leaf_mis = cand_mis = 0
-    for i in range(nq):
-        q = Qs[i]
-        cs = orc.centroid_scores(q)
-        ranked_match(tr["leaf_ids"][i], tr["leaf_scores"][i], o["leaves"][i], o["leaf_scores"][i],
-                     lambda g: cs[g], f"q{i} leaves")
-        if not same_set(tr["leaf_ids"][i], o["leaves"][i]):
-            leaf_mis += 1
-            continue
-        assert tr["scanned"][i] == o["scanned"][i]
-        assert tr["ncand"][i] == o["ncand"][i]
-        gc = tr["cand_ids"][i]
-        if lut_mode == 1:
-            np.testing.assert_array_equal(gc, o["cand_ids"][i], err_msg=f"q{i} u8 candidates")
-            np.testing.assert_array_equal(tr["cand_sums"][i].astype(np.uint32), o["cand_sums"][i])
-            np.testing.assert_array_equal(tr["cand_scores"][i], o["cand_scores"][i].astype(np.float32))
-        else:
-            ranked_match(gc, tr["cand_scores"][i], o["cand_ids"][i], o["cand_scores"][i],
-                         lambda g: orc.point_scores(q, inv[g])[0], f"q{i} candidates")
-        if reorder_num > 0:
-            exact_of = lambda g: orc.point_scores(q, inv[g])[1]
-        elif lut_mode == 0:
-            exact_of = lambda g: orc.point_scores(q, inv[g])[0]
-        else:
-            exact_of = None
-        if not same_set(gc, o["cand_ids"][i]):
-            cand_mis += 1
-            # valid: the final ids are the best k of the GPU's candidates
-            nc = int((gc >= 0).sum())
-            ex = exact_of(gc[:nc])
-            order = np.lexsort((gc[:nc], -ex))[:k]
-            ranked_match(ids[i], scores[i], np.pad(gc[:nc][order], (0, k - len(order)), constant_values=-1),
-                         np.pad(ex[order], (0, k - len(order)), constant_values=-np.inf), exact_of, f"q{i} final*")
-            continue
-        if exact_of is None:     # uint8 approximate ranking: bit-exact
-            np.testing.assert_array_equal(ids[i], o["ids"][i])
-            np.testing.assert_array_equal(scores[i], o["scores"][i].astype(np.float32))
-        else:
-            ranked_match(ids[i], scores[i], o["ids"][i], o["scores"][i], exact_of, f"q{i} final")
-    assert leaf_mis <= max(1, max_leaf_mismatch * nq), f"{leaf_mis} queries with a different leaf set"
-    assert cand_mis <= max(1, max_cand_mismatch * nq), f"{cand_mis} queries with a different candidate set"
+    r = compare_search(index, arr, Qs, k, L, reorder_num, lut_mode, max_leaf_mismatch=max_leaf_mismatch,
+                       max_cand_mismatch=max_cand_mismatch, label=name)
     index.close()
-    return dict(leaf_mismatch=leaf_mis, cand_mismatch=cand_mis, ids=ids, scores=scores, oracle=o)
+    return r
 
 
 @pytest.mark.parametrize("lut_mode", [0, 1])
@@ -174,24 +133,36 @@ def test_sweep_mini(Index):
 
 
 @pytest.mark.parametrize("name,L", [("leaves-1500", 40), ("leaves-3000", 64), ("leaves-3000", 100),
-                                    ("leaves-5000", 16)])
+                                    ("leaves-5000", 16), ("leaves-5000", 300), ("leaves-20000", 40)])
 def test_many_centroids(Index, name, L):
     # more centroids than one warp holds in registers: two-stage warp selection
-    # (two register widths, L <= 64), the block's register form (L > 64), and
-    # beyond 4096 centroids the shared-memory radix
+    # (two register widths, L <= 64), the 256-thread register form (L > 64),
+    # the 1024-thread register form (4096 < centroids <= 16384), and beyond
+    # that the shared-memory radix
     compare(Index, name, 10, L, 100, 0)
 
 
 @pytest.mark.parametrize("name", ["gemm128-vec", "gemm128-scalar"])
 def test_large_batch_centroid_tiles(Index, name):
     # 2048 queries x 2048 centroids: the 128-wide centroid tiles (float4 operand
-    # loads when d % 4 == 0, scalar ones otherwise); the whole batch is searched,
-    # a sample of queries is checked stage by stage
-    from parity import compare_search
+    # loads when d % 4 == 0, scalar ones otherwise); the whole batch is searched
+    # and every query checked stage by stage
     w, X, Q, ix, arr = _workload(name)
-    index = Index(ix)
-    compare_search(index, arr, Q, 10, w.num_leaves_to_search, 100, 0, qsel=np.arange(0, w.nq, 16))
-    index.close()
+    compare(Index, name, 10, w.num_leaves_to_search, 100, 0)
+
+
+def test_tensor_core_scores_ragged_tiles(Index):
+    # 300 queries x 3,500 centroids x d = 36: the tensor-core centroid tiles
+    # (128 x 256, K slices of 16) with a partial last tile in every dimension
+    compare(Index, "tc-ragged", 10, 8, 100, 0)
+
+
+def test_tensor_core_scores_integer_data_exact(Index):
+    # integer coordinates 0..255 split with a zero low part, so the
+    # tensor-core products and sums are exact: leaf scores bit-identical to
+    # the oracle's fp64 scores
+    r = compare(Index, "tc-integer", 10, 16, 200, 0, max_leaf_mismatch=0.0)
+    np.testing.assert_array_equal(r["trace"]["leaf_scores"], r["oracle"]["leaf_scores"].astype(np.float32))
 
 
 @pytest.mark.parametrize("reorder_num", [100, 0])
@@ -377,3 +348,49 @@ def test_speed_knobs_do_not_change_results(Index, lut_mode):
         torch.testing.assert_close(got[1], ref[1], rtol=0, atol=0)
     index.sync_status()
     index.close()
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs two CUDA devices")
+def test_search_refuses_a_device_other_than_the_index_device(Index):
+    # the C entry points check the current device themselves (the binding's
+    # own device guard is bypassed here by calling the library directly)
+    import ctypes
+    from mips_ivf_centroid_b200.index import load_library
+    w, X, Q, ix, arr = _workload("glove-mini")
+    index = Index(ix)
+    lib = load_library()
+    qg = torch.from_numpy(Q[:8]).cuda(0)
+    ids = torch.empty((8, 10), dtype=torch.int32, device="cuda:0")
+    sc = torch.empty((8, 10), dtype=torch.float32, device="cuda:0")
+    with torch.cuda.device(1):
+        torch.cuda.synchronize(1)
+        free0, _ = torch.cuda.mem_get_info(1)
+        st = lib.ah_search(index._h, ctypes.c_void_p(qg.data_ptr()), 8, 10, 24, 100, 0,
+                           ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(sc.data_ptr()), None)
+        assert st == 1, lib.ah_last_error()
+        st = lib.ah_reserve(index._h, 8, 10, 24, 100, 0)
+        assert st == 1
+        torch.cuda.synchronize(1)
+        assert torch.cuda.mem_get_info(1)[0] == free0
+    index.close()
+
+
+@pytest.mark.parametrize("name,L", [("glove-mini", 24), ("openai-mini", 10), ("sweep-mini", 64), ("tiny-leaves", 1500)])
+def test_uint8_tensor_core_scan_equals_lookup_scan(Index, name, L):
+    # the int8 tensor-core scan sums the same integers as the table lookups:
+    # forced on and forced off give identical candidates, sums and results
+    w, X, Q, ix, arr = _workload(name)
+    index = Index(ix)
+    qg = torch.from_numpy(Q).cuda()
+    out = {}
+    for opt in (0, 2):
+        index.set_option(Index.OPT_UINT8_TENSOR_CORES, opt)
+        out[opt] = index.search(qg, 10, L, 100, 1, trace=True)
+        index.sync_status()
+    for x, y in zip(out[0][:2], out[2][:2]):
+        torch.testing.assert_close(x, y, rtol=0, atol=0)
+    for key in ("cand_ids", "cand_sums", "ncand", "scanned"):
+        torch.testing.assert_close(out[0][2][key], out[2][2][key], rtol=0, atol=0)
+    index.close()
+    compare(Index, name, 10, L, 100, 1)
