@@ -247,13 +247,11 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
  *   AH_OPT_SCAN_CHUNK_TILES  32-point code tiles per scan work item (0 =
  *                            automatic, the default)
  *   AH_OPT_UINT8_TENSOR_CORES  how the scan sums uint8 tables: 0 = table
- *                            lookups; 2 = on the int8 tensor cores (each
- *                            point's codes expanded one-hot, multiplied by the
- *                            queries' tables, summed exactly in int32); 1 =
- *                            automatic, the default (tensor cores when a
- *                            searched leaf holds about 16 or more queries of
- *                            the batch on average).  The integer sums are the
- *                            same either way.
+ *                            lookups in shared memory (the default); 1 = on
+ *                            the int8 tensor cores (each point's codes
+ *                            expanded one-hot and multiplied by the queries'
+ *                            tables, summed exactly in int32).  The integer
+ *                            sums, and so the results, are the same either way.
  * Errors: AH_ERR_INVALID_ARG for an unknown option or a value out of range.
  */
 enum {

@@ -107,7 +107,7 @@ struct ah_index {
     int opt_threshold_leaves = 1;
     int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
-    int opt_u8_tensor = 1;           // uint8 scan on the tensor cores: 0 never, 1 automatic, 2 always
+    int opt_u8_tensor = 0;           // uint8 scan: 0 table lookups (default), 1 int8 tensor cores
     void* loaded[6] = {};            // index arrays owned by an index from ah_load
     void* noalloc_scratch = nullptr; // device address of the library's fixed scratch on this device
     // side stream for the stages that do not depend on the partition stage
@@ -154,6 +154,8 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     add(sizeof(int32_t) * (size_t)cnq * cap);                   // 18 candidate slots
     add(sizeof(int32_t) * (size_t)cnq);                         // 19 finish order
     add(ix->c_split ? 2 * sizeof(float) * (size_t)cnq * d : 0);  // 20 queries split for the tensor cores
+    const bool split_topl = NL > 4096 && cL <= 256;
+    add(split_topl ? sizeof(uint64_t) * (size_t)std::min(cnq, 64) * 16 * cL : 0);   // 21 split top-L survivors
     size_t total = 0;
     for (int i = 0; i < n; ++i) total += sz[i];
     if (w.base) {
@@ -191,6 +193,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     b.order = reinterpret_cast<int32_t*>(part[19]);
     b.q_hi = ix->c_split ? reinterpret_cast<float*>(part[20]) : nullptr;
     b.q_lo = ix->c_split ? b.q_hi + (size_t)cnq * d : nullptr;
+    b.topl_tmp = split_topl ? reinterpret_cast<uint64_t*>(part[21]) : nullptr;
     int32_t* zr = reinterpret_cast<int32_t*>(part[10]);
     b.qcount = zr;
     b.qcursor = zr + NL;
@@ -266,10 +269,9 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     a.reorder_num = reorder_num;
     a.R = R;
     a.lut_mode = lut_mode;
-    // uint8 tables scan on the int8 tensor cores when a leaf's queries fill a
-    // good part of the 128-row MMA tile (about 16 or more per searched leaf)
-    a.scan_tc = (lut_mode == AH_LUT_U8 && ix->opt_u8_tensor != 0 &&
-                 (ix->opt_u8_tensor == 2 || static_cast<double>(nq) * L >= 16.0 * ix->dix.nl)) ? 1 : 0;
+    // uint8 tables: the int8 tensor-core scan only when asked for (on the
+    // benchmarked batches it ran 1.1-2.9x slower than the table lookups)
+    a.scan_tc = (lut_mode == AH_LUT_U8 && ix->opt_u8_tensor == 1) ? 1 : 0;
     // code tiles per scan item: up to 32, fewer (multiples of 8, one tile per
     // warp of a 256-thread CTA) when the batch's tiles, estimated from the
     // average leaf, would leave scan CTAs (about 6 per SM) without an item
@@ -646,7 +648,7 @@ ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
             ix->opt_progressive_leaves = static_cast<int>(value);
             return AH_OK;
         case AH_OPT_UINT8_TENSOR_CORES:
-            if (value < 0 || value > 2) return fail(AH_ERR_INVALID_ARG, "uint8 tensor-core scan option outside [0, 2]");
+            if (value < 0 || value > 1) return fail(AH_ERR_INVALID_ARG, "uint8 tensor-core scan option outside [0, 1]");
             ix->opt_u8_tensor = static_cast<int>(value);
             return AH_OK;
         case AH_OPT_SCAN_CHUNK_TILES:

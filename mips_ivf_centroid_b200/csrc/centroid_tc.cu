@@ -20,11 +20,12 @@
 // the accumulated error stays below about 64 ulps of sum |q_t c_t| (4e-6 on
 // unit vectors); d is limited to 4096 (171 MMAs, 1e-5).
 //
-// One CTA computes a 128 x 128 tile of S: TMA brings 16-wide K slices of
-// Q_hi, Q_lo and C_hi, C_lo (128 rows each) into shared memory (64-byte
-// swizzle, six stages, mbarrier completion), one thread issues tcgen05.mma
-// kind::tf32 (M = 128, N = 128, K = 8; three per half slice), and the four
-// warps read the accumulators back with tcgen05.ld and store the sums.
+// One CTA computes a 128 x 128 tile of S: one thread (warp 0) issues the TMA
+// loads of 16-wide K slices of Q_hi, Q_lo and C_hi, C_lo (128 rows each) into a
+// six-stage ring (64-byte swizzle, mbarrier completion), another (warp 1)
+// waits for each slice and issues tcgen05.mma kind::tf32 (M = N = 128, K = 8;
+// three per half slice), committing the stage free, and the four warps then
+// read the accumulators back with tcgen05.ld and store the sums.
 // Every mbarrier wait is bounded: on expiry the kernel records an error,
 // waits (bounded) for its own transfers, frees its tensor memory and returns.
 #include <cuda.h>
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) centroid_scores_tc_kernel(
     __shared__ __align__(8) uint64_t empty[kTcStages];
     __shared__ __align__(8) uint64_t done;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_fail;
+    __shared__ int s_fail, s_issued, s_consumed;
     // 1024-byte aligned stage buffers (the swizzle pattern repeats every 512 B)
     unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -171,9 +172,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) centroid_scores_tc_kernel(
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = s_tmem;
 
+    auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * kStageBytes; };
     if (tid == 0) {
-        auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * kStageBytes; };
-        auto load = [&](int kt, int s) {
+        // producer: a stage is refilled once the MMAs that read it are done
+        int kt = 0;
+        for (; kt < KT; ++kt) {
+            const int s = kt % kTcStages;
+            if (kt >= kTcStages && !mbar_wait(&empty[s], ((kt / kTcStages) + 1) & 1)) {
+                s_fail = 1;
+                break;
+            }
             unsigned char* p = stage_ptr(s);
             mbar_expect_tx(&full[s], kStageBytes);
             const int k0 = kt * kTcK;
@@ -181,22 +189,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) centroid_scores_tc_kernel(
             tma_load_2d(p + kATileBytes, &qlo, &full[s], k0, m0);
             tma_load_2d(p + 2 * kATileBytes, &chi, &full[s], k0, n0);
             tma_load_2d(p + 2 * kATileBytes + kBTileBytes, &clo, &full[s], k0, n0);
-        };
-        const int pre = KT < kTcStages ? KT : kTcStages;
-        for (int kt = 0; kt < pre; ++kt) load(kt, kt);
-        int issued = pre;                         // slices whose loads were issued
-        bool ok = true;
+        }
+        s_issued = kt;
+    } else if (tid == 32) {
+        // MMA issuer: hi . hi into accumulator kt % 3 (slices kt < 3 start
+        // it), the cross terms into accumulator 3 (slice 0 starts it)
         int kt = 0;
-        for (; kt < KT && ok; ++kt) {
+        for (; kt < KT; ++kt) {
             const int s = kt % kTcStages;
-            if (!mbar_wait(&full[s], (kt / kTcStages) & 1)) { ok = false; break; }
+            if (!mbar_wait(&full[s], (kt / kTcStages) & 1)) {
+                s_fail = 1;
+                break;
+            }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t a_hi = smem_u32(stage_ptr(s));
             const uint32_t a_lo = a_hi + kATileBytes;
             const uint32_t b_hi = a_hi + 2 * kATileBytes;
             const uint32_t b_lo = b_hi + kBTileBytes;
-            // hi . hi into accumulator kt % 3 (slices kt < 3 start it), the
-            // cross terms into accumulator 3 (slice 0 starts it)
             const uint32_t main = tmem + static_cast<uint32_t>((kt % 3) * kTcN);
             const uint32_t cross = tmem + static_cast<uint32_t>(3 * kTcN);
 #pragma unroll
@@ -207,21 +216,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) centroid_scores_tc_kernel(
                 mma_tf32(cross, sw64_desc(a_lo + off), sw64_desc(b_hi + off), 1u);
             }
             mma_commit(&empty[s]);
-            // refill the stage the previous slice used once its MMAs are done
-            if (kt > 0 && issued < KT) {
-                const int ps = (kt - 1) % kTcStages;
-                if (!mbar_wait(&empty[ps], ((kt - 1) / kTcStages) & 1)) { ok = false; ++kt; break; }
-                load(issued, ps);
-                ++issued;
-            }
-        }
-        if (!ok) {
-            s_fail = 1;
-            atomicCAS(err, 0, kDevTimeout);
-            // let this CTA's issued transfers land before its shared memory goes away
-            for (int j = kt; j < issued; ++j) mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1);
         }
         mma_commit(&done);                    // arrives once every MMA issued above has completed
+        s_consumed = kt;
+    }
+    // a failed wait can leave loads the MMA thread never consumed: let them
+    // land (bounded) before this CTA's shared memory goes away
+    __syncthreads();
+    if (tid == 0 && s_fail) {
+        atomicCAS(err, 0, kDevTimeout);
+        for (int j = s_consumed; j < s_issued; ++j) mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1);
     }
     __syncthreads();
     // epilogue: warp w reads accumulator lanes 32w .. 32w + 31 (its rows)

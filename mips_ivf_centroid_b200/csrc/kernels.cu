@@ -29,12 +29,6 @@
 #include "kernels.h"
 #include "select.cuh"
 
-#ifndef AH_SINGLE_GROUP
-#define AH_SINGLE_GROUP 1
-#endif
-#ifndef AH_CENTROID_TC
-#define AH_CENTROID_TC 1
-#endif
 
 namespace ah {
 
@@ -130,13 +124,7 @@ __global__ void interleave_codes_kernel(const uint8_t* __restrict__ codes, const
     il[e] = v;
 }
 
-#ifndef AH_MAX_CODE_V
-#define AH_MAX_CODE_V 4
-#endif
-int code_vector_words(int W) {
-    const int v = (W % 4 == 0) ? 4 : (W % 2 == 0) ? 2 : 1;
-    return v < AH_MAX_CODE_V ? v : AH_MAX_CODE_V;
-}
+int code_vector_words(int W) { return (W % 4 == 0) ? 4 : (W % 2 == 0) ? 2 : 1; }
 
 cudaError_t launch_prepare_index(const int32_t* offs32, const int32_t* ptile, int nl, const uint8_t* codes, int cb,
                                  int W, int64_t ntiles, uint32_t* codes_il, cudaStream_t s) {
@@ -322,7 +310,7 @@ __global__ void __launch_bounds__(256, 2) centroid_scores128_kernel(const float*
 // 128x128 tiles for large batches, 64x64 for mid-size ones, 32x32 for very
 // small problems (more CTAs in flight).
 cudaError_t launch_centroid_scores(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
-    if (AH_CENTROID_TC && ix.c_hi && b.q_hi && centroid_tc_usable(a.nq, ix.nl, ix.d)) {
+    if (ix.c_hi && b.q_hi && centroid_tc_usable(a.nq, ix.nl, ix.d)) {
         // tensor cores: the queries split into tf32 halves, then the tiles
         cudaError_t e = launch_split_tf32(a.queries, static_cast<int64_t>(a.nq) * ix.d, b.q_hi, b.q_lo, s);
         if (e != cudaSuccess) return e;
@@ -448,7 +436,9 @@ __device__ int block_topk_reg(GetKey get, GetVal pay, int n, int K, RegSelectScr
 
 // One CTA of NT threads per query with the score row in registers (KPL per
 // thread): for 1024 < centroids <= KPL * NT.
-template <int KPL, int NT>
+// MERGE: the keys are the survivors of top_leaves_seg_kernel's segments
+// instead of the score row (the leaf id is inside each key).
+template <int KPL, int NT, bool MERGE = false>
 __global__ void __launch_bounds__(NT) top_leaves_reg_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
     extern __shared__ __align__(16) unsigned char smem[];
@@ -459,10 +449,18 @@ __global__ void __launch_bounds__(NT) top_leaves_reg_kernel(DeviceIndex ix, Sear
     const int L = a.L, nl = ix.nl;
     uint64_t* keys = reinterpret_cast<uint64_t*>(smem);
     const float* row = b.cscore + static_cast<int64_t>(q) * nl;
-    auto get = [&](int i) { return make_key(float_key(row[i]), i); };
+    int n = nl;
+    const uint64_t* cand = nullptr;
+    if (MERGE) {
+        // segment s kept min(L, its size) keys, stored back to back
+        const int seg = a.topl_seg, S = (nl + seg - 1) / seg;
+        n = (S - 1) * min(L, seg) + min(L, nl - (S - 1) * seg);
+        cand = b.topl_tmp + static_cast<int64_t>(q) * a.topl_stride;
+    }
+    auto get = [&](int i) { return MERGE ? cand[i] : make_key(float_key(row[i]), i); };
     auto pay = [&](int i) { return i; };
     if (threadIdx.x == 0) s_scanned = 0;
-    block_topk_reg<KPL, NT>(get, pay, nl, L, rs, &s_count, keys, static_cast<int32_t*>(nullptr), true);
+    block_topk_reg<KPL, NT>(get, pay, n, L, rs, &s_count, keys, static_cast<int32_t*>(nullptr), true);
     long long local = 0;
     for (int i = threadIdx.x; i < L; i += NT) {
         const uint64_t key = keys[i];
@@ -539,6 +537,11 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_2stage_kernel(DeviceIn
 
 constexpr int kTopWarps = 8;
 constexpr int kTopRegWide = 1024;      // threads of the widest register top-L form
+// split top-L (small batches, more than 4096 centroids): up to this many
+// segments per query, batches up to kTopSplitMaxQ queries, L up to kTopSplitMaxL
+constexpr int kTopSplitSegs = 16;
+constexpr int kTopSplitMaxQ = 64;
+constexpr int kTopSplitMaxL = 256;
 
 // One warp per query when the centroids fit 32 per lane: the scores stay in
 // registers and the selection needs no shared-memory passes.
@@ -568,7 +571,51 @@ __global__ void __launch_bounds__(kTopWarps * 32) top_leaves_warp_kernel(DeviceI
     if (lane == 0) b.scanned[q] = local;
 }
 
+// Small batches over many centroids, first step: CTA (s, q) keeps the best
+// min(L, size) keys of segment s of query q's score row (1,024 scores per
+// segment at most, 4 per thread), unordered, at tmp[q][s * min(L, seg)].
+// Any key of the row's best L is among its segment's best L, so the
+// segments' survivors hold the row's best L; top_leaves_reg_kernel<...,
+// true> keeps those.
+__global__ void __launch_bounds__(kSelThreads) top_leaves_seg_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
+    __shared__ RegSelectScratch<kSelThreads> rs;
+    __shared__ int s_count;
+    __shared__ uint64_t keys[1024];
+    const int sidx = blockIdx.x, q = blockIdx.y;
+    const int seg = a.topl_seg, L = a.L;
+    const int lo = sidx * seg, n = min(seg, ix.nl - lo);
+    const float* row = b.cscore + static_cast<int64_t>(q) * ix.nl + lo;
+    auto get = [&](int i) { return make_key(float_key(row[i]), lo + i); };
+    auto pay = [&](int i) { return i; };
+    const int K = block_topk_reg<4, kSelThreads>(get, pay, n, min(L, n), rs, &s_count, keys,
+                                                 static_cast<int32_t*>(nullptr), false);
+    uint64_t* out = b.topl_tmp + static_cast<int64_t>(q) * a.topl_stride + static_cast<int64_t>(sidx) * min(L, seg);
+    for (int i = threadIdx.x; i < K; i += kSelThreads) out[i] = keys[i];
+}
+
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+    if (b.topl_tmp && ix.nl > 16 * kSelThreads && a.nq <= kTopSplitMaxQ && a.L <= kTopSplitMaxL) {
+        // split form: segments of at most 1,024 scores in parallel, then one
+        // CTA per query merges the survivors (at most 16 x 256 keys)
+        a.topl_seg = (ix.nl + kTopSplitSegs - 1) / kTopSplitSegs;
+        if (a.topl_seg > 1024) a.topl_seg = 1024;
+        const int S = (ix.nl + a.topl_seg - 1) / a.topl_seg;
+        a.topl_stride = S * a.L;
+        if (S <= kTopSplitSegs) {
+            if (const cudaError_t le = launch_chained(top_leaves_seg_kernel, dim3(S, a.nq), dim3(kSelThreads), 0, s, ix, a, b);
+                le != cudaSuccess)
+                return le;
+            const size_t smem = static_cast<size_t>(next_pow2(a.L)) * sizeof(uint64_t);
+            cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_reg_kernel<16, kSelThreads, true>), smem, false);
+            if (e != cudaSuccess) return e;
+            if (const cudaError_t le = launch_chained(top_leaves_reg_kernel<16, kSelThreads, true>, dim3(a.nq),
+                                                      dim3(kSelThreads), smem, s, ix, a, b);
+                le != cudaSuccess)
+                return le;
+            return cudaGetLastError();
+        }
+    }
     if (ix.nl <= 32 * 32 && a.L <= kWarpMaxK) {
         const size_t smem = static_cast<size_t>(kTopWarps) * next_pow2(a.L) * sizeof(uint64_t);
         cudaError_t e = ensure_smem(reinterpret_cast<const void*>(top_leaves_warp_kernel), smem, false);
@@ -611,56 +658,73 @@ cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchB
 
 constexpr int kScanBlock = 1024;
 
-__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* warp_sums, int* total) {
+// Exclusive prefix sums of a pair of values over a 1,024-thread block; the
+// block's totals in *total.
+__device__ __forceinline__ int2 block_exclusive_scan2_1024(int2 v, int2* warp_sums, int2* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+    int2 x = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
-        if (lane >= off) x += y;
+        const int yx = __shfl_up_sync(0xFFFFFFFFu, x.x, off), yy = __shfl_up_sync(0xFFFFFFFFu, x.y, off);
+        if (lane >= off) { x.x += yx; x.y += yy; }
     }
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_sums[lane];
-        int xs = w;
+        const int2 w = warp_sums[lane];
+        int2 xs = w;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            int y = __shfl_up_sync(0xFFFFFFFFu, xs, off);
-            if (lane >= off) xs += y;
+            const int yx = __shfl_up_sync(0xFFFFFFFFu, xs.x, off), yy = __shfl_up_sync(0xFFFFFFFFu, xs.y, off);
+            if (lane >= off) { xs.x += yx; xs.y += yy; }
         }
-        warp_sums[lane] = xs - w;   // exclusive prefix of warps
+        warp_sums[lane] = make_int2(xs.x - w.x, xs.y - w.y);   // exclusive prefix of warps
         if (lane == 31) *total = xs;
     }
     __syncthreads();
-    int r = warp_sums[warp] + x - v;
+    const int2 r = make_int2(warp_sums[warp].x + x.x - v.x, warp_sums[warp].y + x.y - v.y);
     __syncthreads();
     return r;
 }
 
 // Single CTA: qoff = exclusive scan of queries per leaf; item_off = exclusive
 // scan of work items per leaf (query groups x chunks of `chunk` code tiles).
+// Each thread takes 8 consecutive leaves, so 8,192 leaves cost one block scan.
 __global__ void __launch_bounds__(kScanBlock) invert_offsets_kernel(DeviceIndex ix, SearchBuffers b, int group, int chunk) {
     chain_entry();
-    __shared__ int warp_sums[32];
-    __shared__ int total_q, total_i;
+    constexpr int E = 8;
+    __shared__ int2 warp_sums[32];
+    __shared__ int2 total;
     int carry_q = 0, carry_i = 0;
-    for (int base = 0; base < ix.nl; base += kScanBlock) {
-        int c = base + threadIdx.x;
-        int qc = 0, it = 0;
-        if (c < ix.nl) {
-            qc = b.qcount[c];
-            int tiles = ix.ptile[c + 1] - ix.ptile[c];
-            it = (qc > 0 && tiles > 0) ? ((qc + group - 1) / group) * ((tiles + chunk - 1) / chunk) : 0;
+    for (int base = 0; base < ix.nl; base += kScanBlock * E) {
+        const int c0 = base + threadIdx.x * E;
+        int eq[E], ei[E];
+        int sq = 0, si = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int c = c0 + e;
+            int qc = 0, it = 0;
+            if (c < ix.nl) {
+                qc = b.qcount[c];
+                const int tiles = ix.ptile[c + 1] - ix.ptile[c];
+                it = (qc > 0 && tiles > 0) ? ((qc + group - 1) / group) * ((tiles + chunk - 1) / chunk) : 0;
+            }
+            eq[e] = sq;
+            ei[e] = si;
+            sq += qc;
+            si += it;
         }
-        int eq = block_exclusive_scan_1024(qc, warp_sums, &total_q);
-        int ei = block_exclusive_scan_1024(it, warp_sums, &total_i);
-        if (c < ix.nl) {
-            b.qoff[c] = carry_q + eq;
-            b.item_off[c] = carry_i + ei;
+        const int2 ex = block_exclusive_scan2_1024(make_int2(sq, si), warp_sums, &total);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int c = c0 + e;
+            if (c < ix.nl) {
+                b.qoff[c] = carry_q + ex.x + eq[e];
+                b.item_off[c] = carry_i + ex.y + ei[e];
+            }
         }
-        carry_q += total_q;
-        carry_i += total_i;
+        carry_q += total.x;
+        carry_i += total.y;
         __syncthreads();
     }
     if (threadIdx.x == 0) {
@@ -872,12 +936,22 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
             for (int u = 0; u < 4; ++u) code_words4(cw[u], ln[u], w, V, c[u][0], c[u][1], c[u][2], c[u][3]);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float* base = lf + 8 * (w + k) * kCenters;
+                // byte offsets of the word's 8 entries: nibbles 0, 2, 4, 6 in
+                // the bytes of ev, 1, 3, 5, 7 in those of od (times 4 bytes)
+                const char* base = reinterpret_cast<const char*>(lf + 8 * (w + k) * kCenters);
+                uint32_t ev[4], od[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    ev[u] = (c[u][k] & 0x0F0F0F0Fu) << 2;
+                    od[u] = ((c[u][k] >> 4) & 0x0F0F0F0Fu) << 2;
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        acc[u] = __fadd_rn(acc[u], base[i * kCenters + ((c[u][k] >> (4 * i)) & 15u)]);
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t off = __byte_perm((i & 1) ? od[u] : ev[u], 0u, 0x4440u | (i >> 1));
+                        acc[u] = __fadd_rn(acc[u], *reinterpret_cast<const float*>(base + i * 4 * kCenters + off));
+                    }
             }
         }
         for (; w < Wf; ++w)
@@ -1235,11 +1309,18 @@ struct U8Layout<true> {
 template <int G, bool SPLIT>
 __device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, const typename U8Layout<SPLIT>::Entry* __restrict__ base,
                                            uint32_t (&ae)[G / 4], uint32_t (&ao)[G / 4]) {
+    using Entry = typename U8Layout<SPLIT>::Entry;
     constexpr int BS = (G / 4) * kCenters;   // entries per block
+    constexpr int SH = sizeof(Entry) == 8 ? 3 : 2;
+    // byte offsets of the word's entries: nibbles 0, 2, 4, 6 in the bytes of
+    // ev, 1, 3, 5, 7 in those of od
+    const uint32_t ev = (c & 0x0F0F0F0Fu) << SH, od = ((c >> 4) & 0x0F0F0F0Fu) << SH;
+    const char* bb = reinterpret_cast<const char*>(base);
 #pragma unroll
     for (int nib = 0; nib < 8; ++nib) {
         if (nib < nb) {
-            const typename U8Layout<SPLIT>::Entry* p = base + nib * BS + ((c >> (4 * nib)) & 15u);
+            const uint32_t off = __byte_perm((nib & 1) ? od : ev, 0u, 0x4440u | (nib >> 1));
+            const Entry* p = reinterpret_cast<const Entry*>(bb + nib * BS * static_cast<int>(sizeof(Entry)) + off);
 #pragma unroll
             for (int qd = 0; qd < G / 4; ++qd) U8Layout<SPLIT>::add(p + qd * kCenters, ae[qd], ao[qd]);
         }
@@ -1501,7 +1582,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
         TileJob job;
         job.gsize = min(GMAX, qcnt - g * GMAX);
         // table width of this group (a lone query is not padded)
-        const int G = (AH_SINGLE_GROUP && job.gsize == 1) ? 1 : ((job.gsize + GSTEP - 1) / GSTEP) * GSTEP;
+        const int G = job.gsize == 1 ? 1 : ((job.gsize + GSTEP - 1) / GSTEP) * GSTEP;
         job.t0 = pt0 + c * a.chunk;
         job.t1 = min(pt0 + ntile, job.t0 + a.chunk);
         job.slot_base = ix.offs[leaf] - 32 * pt0;

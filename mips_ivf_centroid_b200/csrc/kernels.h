@@ -49,6 +49,7 @@ struct SearchBuffers {
     float* cscore;          // [nq][NL]
     float* q_hi;            // [nq][d] queries split for the tensor cores (or null: SIMT tiles)
     float* q_lo;            // [nq][d]
+    uint64_t* topl_tmp;     // [nq][16 L] split top-L survivors (batches of at most 64; or null)
     int32_t* leaves;        // [nq][L]
     float* leaf_scores;     // [nq][L]
     int64_t* scanned;       // [nq]
@@ -101,6 +102,8 @@ struct SearchArgs {
     int threshold_leaves;       // best leaves the sample is spread over
     int scan_counter;           // index into counters[] of the scan's work counter
     int count_ranks;            // top-L kernel counts queries per leaf for ranks below this
+    int topl_seg;               // split top-L: scores per segment (set by the top-L launcher)
+    int topl_stride;            // split top-L: keys per query in topl_tmp
     int scan_tc;                // uint8 tables: scan on the int8 tensor cores (items of up to 128
                                 // queries x 256 points) instead of table lookups
 };
