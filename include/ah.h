@@ -230,7 +230,7 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
  *   AH_OPT_THRESHOLD_SAMPLE  points scored per query, from its best leaves, to
  *                            bound its R-th best approximate score before the
  *                            scan (default 1024; the bound uses
- *                            max(value, 4 R) points, at most 4096; batches of
+ *                            max(value, 2 R) points, at most 4096; batches of
  *                            fewer than 1,024 queries use more, up to 4096,
  *                            when the bound would otherwise keep many points)
  *   AH_OPT_THRESHOLD_LEAVES  how many of the best leaves that sample is spread
@@ -252,6 +252,14 @@ AH_API ah_status ah_reserve(ah_index *ix, int32_t max_nq, int32_t k, int32_t num
  *                            expanded one-hot and multiplied by the queries'
  *                            tables, summed exactly in int32).  The integer
  *                            sums, and so the results, are the same either way.
+ *   AH_OPT_QUERY_MAJOR_SCAN  how the scan splits its work: 0 = automatic (the
+ *                            default): query-major when on average at most one
+ *                            query of the batch searches a leaf (nq x L <= NL)
+ *                            and each scan phase covers at most 1,024 leaf
+ *                            ranks, leaf-major (queries sharing a leaf share
+ *                            its code reads) otherwise; 1 = query-major
+ *                            whenever a phase covers at most 1,024 leaf
+ *                            ranks; -1 = always leaf-major
  * Errors: AH_ERR_INVALID_ARG for an unknown option or a value out of range.
  */
 enum {
@@ -259,7 +267,8 @@ enum {
     AH_OPT_SCAN_CHUNK_TILES = 2,
     AH_OPT_THRESHOLD_LEAVES = 3,
     AH_OPT_PROGRESSIVE_LEAVES = 4,
-    AH_OPT_UINT8_TENSOR_CORES = 5
+    AH_OPT_UINT8_TENSOR_CORES = 5,
+    AH_OPT_QUERY_MAJOR_SCAN = 6
 };
 AH_API ah_status ah_set_option(ah_index *ix, int32_t option, int64_t value);
 

@@ -108,6 +108,7 @@ struct ah_index {
     int opt_progressive_leaves = 0;
     int opt_chunk_tiles = 0;
     int opt_u8_tensor = 0;           // uint8 scan: 0 table lookups (default), 1 int8 tensor cores
+    int opt_query_scan = 0;          // query-major scan: 0 automatic, 1 whenever it applies, -1 never
     void* loaded[6] = {};            // index arrays owned by an index from ah_load
     void* noalloc_scratch = nullptr; // device address of the library's fixed scratch on this device
     // side stream for the stages that do not depend on the partition stage
@@ -272,14 +273,14 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     // uint8 tables: the int8 tensor-core scan only when asked for (on the
     // benchmarked batches it ran 1.1-2.9x slower than the table lookups)
     a.scan_tc = (lut_mode == AH_LUT_U8 && ix->opt_u8_tensor == 1) ? 1 : 0;
-    // code tiles per scan item: up to 32, fewer (multiples of 8, one tile per
+    // code tiles per scan item: up to 128, fewer (multiples of 8, one tile per
     // warp of a 256-thread CTA) when the batch's tiles, estimated from the
     // average leaf, would leave scan CTAs (about 6 per SM) without an item
     {
         const double est_tiles = static_cast<double>(nq) * L * std::max(1.0, static_cast<double>(ix->dix.n) / ix->dix.nl / 32.0);
         const double ctas = static_cast<double>(ix->num_sms) * 6;
         const int c = 8 * static_cast<int>(std::ceil(est_tiles / ctas / 8.0));
-        a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : std::min(32, std::max(8, c));
+        a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : std::min(128, std::max(8, c));
         if (a.scan_tc) a.chunk = ah::scan_tc_chunk_tiles();
     }
     a.threshold_sample = ix->opt_threshold_sample;
@@ -367,6 +368,18 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
             if (e2 >= L) break;
         }
     }
+    // Query-major scan when the batch's queries seldom share a leaf (on
+    // average at most one query per leaf over the searched ranks): the
+    // leaf-major groups would almost all be lone queries, each item staging
+    // its table again.  It needs no leaf inversion.
+    bool qmajor = false;
+    if (!a.scan_tc && ix->opt_query_scan >= 0) {
+        int widest = 0;
+        for (size_t p = 0; p + 1 < bounds.size(); ++p) widest = std::max(widest, bounds[p + 1] - bounds[p]);
+        const bool fits = widest <= ah::kQScanMaxLeaves &&
+                          ah::scan_query_smem_bytes(lut_mode, dix.B, widest) <= ah::kMaxSmemPerCta;
+        qmajor = fits && (ix->opt_query_scan == 1 || static_cast<double>(nq) * L <= static_cast<double>(dix.nl));
+    }
     mark(0);
     a.count_ranks = bounds[1];
     if ((e = ah::launch_top_leaves(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "top leaves");
@@ -376,8 +389,10 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
         if ((e = cudaEventRecord(ix->ev_tl, s)) != cudaSuccess || (e = cudaStreamWaitEvent(s2, ix->ev_tl, 0)) != cudaSuccess)
             return cuda_fail(e, "fork");
     }
-    if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], true, s2)) != cudaSuccess) return cuda_fail(e, "invert");
-    launches += 2;
+    if (!qmajor) {
+        if ((e = ah::launch_invert(dix, a, b, bounds[0], bounds[1], true, s2)) != cudaSuccess) return cuda_fail(e, "invert");
+        launches += 2;
+    }
     mark(2);
     if (fork) {
         if ((e = cudaEventRecord(ix->ev_inv, s2)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ix->ev_lut, 0)) != cudaSuccess)
@@ -394,14 +409,22 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     for (size_t p = 0; p + 1 < bounds.size(); ++p) {
         if (p > 0) {
             if ((e = ah::launch_tau_update(dix, a, b, s)) != cudaSuccess) return cuda_fail(e, "bound refinement");
-            if ((e = ah::launch_invert(dix, a, b, bounds[p], bounds[p + 1], false, s)) != cudaSuccess)
-                return cuda_fail(e, "invert");
-            launches += 4;
+            launches += 1;
+            if (!qmajor) {
+                if ((e = ah::launch_invert(dix, a, b, bounds[p], bounds[p + 1], false, s)) != cudaSuccess)
+                    return cuda_fail(e, "invert");
+                launches += 3;
+            }
             mark(6);
         }
-        a.scan_counter = 0;
-        if ((e = cudaMemsetAsync(b.counters, 0, sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "memset");
-        if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
+        if (qmajor) {
+            if ((e = ah::launch_scan_query(dix, a, b, bounds[p], bounds[p + 1], ix->num_sms, s)) != cudaSuccess)
+                return cuda_fail(e, "scan");
+        } else {
+            a.scan_counter = 0;
+            if ((e = cudaMemsetAsync(b.counters, 0, sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "memset");
+            if ((e = ah::launch_scan(dix, a, b, ix->num_sms, s)) != cudaSuccess) return cuda_fail(e, "scan");
+        }
         launches += 1;
         mark(p == 0 ? 5 : 7);
     }
@@ -654,6 +677,10 @@ ah_status ah_set_option(ah_index* ix, int32_t option, int64_t value) {
         case AH_OPT_SCAN_CHUNK_TILES:
             if (value < 0 || value > 1024) return fail(AH_ERR_INVALID_ARG, "scan chunk outside [0, 1024] tiles");
             ix->opt_chunk_tiles = static_cast<int>(value);
+            return AH_OK;
+        case AH_OPT_QUERY_MAJOR_SCAN:
+            if (value < -1 || value > 1) return fail(AH_ERR_INVALID_ARG, "query-major scan option outside [-1, 1]");
+            ix->opt_query_scan = static_cast<int>(value);
             return AH_OK;
         default:
             return fail(AH_ERR_INVALID_ARG, "unknown option");

@@ -880,6 +880,24 @@ __device__ __forceinline__ void code_words4(const uint32_t* __restrict__ tile, i
     }
 }
 
+// Shared loads by 32-bit shared-window address (the address arithmetic stays
+// 32-bit; a constant offset folds into the load).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 template <int MODE>
 __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ codes_il, int W, int V, int B,
                                                const unsigned char* lut, int32_t pos, bool add_off, float off) {
@@ -909,6 +927,9 @@ __device__ __forceinline__ uint32_t slot_value(const uint32_t* __restrict__ code
 // still runs over blocks in order, identical to slot_value.  A slot's code
 // words are read four at a time (one 16-byte load where the copy's vector
 // width is 4), so a warp's loads for consecutive slots stay contiguous.
+// fp32: `lut` starts 256-byte aligned in the shared window; a word's 8 blocks
+// span 512 bytes, so an entry's address is the word's address with its low
+// byte replaced by the nibble's byte offset (one byte permute per lookup).
 template <int MODE>
 __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_il, int W, int V, int B,
                                              const unsigned char* lut, const int32_t* pos, const bool* valid,
@@ -924,6 +945,7 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
     const int Wf = B >> 3, tail = B & 7;
     if (MODE == 0) {
         const float* lf = reinterpret_cast<const float*>(lut);
+        const uint32_t tb = static_cast<uint32_t>(__cvta_generic_to_shared(lut));
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         auto word = [&](int u, uint32_t c, int w, int nb) {
             const float* base = lf + 8 * w * kCenters;
@@ -938,7 +960,7 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
             for (int k = 0; k < 4; ++k) {
                 // byte offsets of the word's 8 entries: nibbles 0, 2, 4, 6 in
                 // the bytes of ev, 1, 3, 5, 7 in those of od (times 4 bytes)
-                const char* base = reinterpret_cast<const char*>(lf + 8 * (w + k) * kCenters);
+                const uint32_t xw = tb + static_cast<uint32_t>(w + k) * (8 * kCenters * 4);
                 uint32_t ev[4], od[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -949,8 +971,8 @@ __device__ __forceinline__ void slot_values4(const uint32_t* __restrict__ codes_
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const uint32_t off = __byte_perm((i & 1) ? od[u] : ev[u], 0u, 0x4440u | (i >> 1));
-                        acc[u] = __fadd_rn(acc[u], *reinterpret_cast<const float*>(base + i * 4 * kCenters + off));
+                        const uint32_t p = __byte_perm((i & 1) ? od[u] : ev[u], xw, 0x7650u | (i >> 1)) + i * 4 * kCenters;
+                        acc[u] = __fadd_rn(acc[u], __uint_as_float(lds_u32(p)));
                     }
             }
         }
@@ -1036,8 +1058,10 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
     __shared__ int s_nseg, s_taken;
     const int q = blockIdx.x;
     const int R = a.R;
-    unsigned char* lut = smem;
-    uint64_t* vals = reinterpret_cast<uint64_t*>(smem + ((table_bytes(MODE, ix.B) + 15) & ~15));
+    // the table starts 256-byte aligned in the shared window (slot_values4's
+    // byte-permute addressing); the launch adds 256 bytes for this
+    unsigned char* lut = smem + ((256u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 255u)) & 255u);
+    uint64_t* vals = reinterpret_cast<uint64_t*>(lut + ((table_bytes(MODE, ix.B) + 15) & ~15));
     uint64_t* top = nullptr;
     load_query_table<MODE>(ix, b, q, lut);
     __syncthreads();
@@ -1184,7 +1208,7 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
 
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
     cudaError_t e;
-    size_t smem = ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + static_cast<size_t>(threshold_sample(a.R, a.threshold_sample)) * sizeof(uint64_t);
+    size_t smem = 256 + ((table_bytes(a.lut_mode, ix.B) + 15) & ~15) + static_cast<size_t>(threshold_sample(a.R, a.threshold_sample)) * sizeof(uint64_t);
     if (a.lut_mode == 0) {
         e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
@@ -1306,23 +1330,38 @@ struct U8Layout<true> {
     }
 };
 
+// One code word (up to 8 blocks) for a group of G queries, uint8 tables.
+// xw: shared address of the word's first block's entries, a multiple of 256
+// (the staged tables start 256-byte aligned and a word's blocks span a
+// multiple of 256 bytes), so an entry's address is xw with its low byte
+// replaced by the nibble's byte offset (nibble x entry size < 256): one byte
+// permute per nibble, the block and quad offsets folding into the loads.
 template <int G, bool SPLIT>
-__device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, const typename U8Layout<SPLIT>::Entry* __restrict__ base,
-                                           uint32_t (&ae)[G / 4], uint32_t (&ao)[G / 4]) {
+__device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, uint32_t xw, uint32_t (&ae)[G / 4],
+                                           uint32_t (&ao)[G / 4]) {
     using Entry = typename U8Layout<SPLIT>::Entry;
-    constexpr int BS = (G / 4) * kCenters;   // entries per block
-    constexpr int SH = sizeof(Entry) == 8 ? 3 : 2;
+    constexpr int E = static_cast<int>(sizeof(Entry));
+    constexpr int BSB = (G / 4) * kCenters * E;   // bytes per block
+    constexpr int SH = E == 8 ? 3 : 2;
     // byte offsets of the word's entries: nibbles 0, 2, 4, 6 in the bytes of
     // ev, 1, 3, 5, 7 in those of od
     const uint32_t ev = (c & 0x0F0F0F0Fu) << SH, od = ((c >> 4) & 0x0F0F0F0Fu) << SH;
-    const char* bb = reinterpret_cast<const char*>(base);
 #pragma unroll
     for (int nib = 0; nib < 8; ++nib) {
         if (nib < nb) {
-            const uint32_t off = __byte_perm((nib & 1) ? od : ev, 0u, 0x4440u | (nib >> 1));
-            const Entry* p = reinterpret_cast<const Entry*>(bb + nib * BS * static_cast<int>(sizeof(Entry)) + off);
+            const uint32_t p = __byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * BSB;
 #pragma unroll
-            for (int qd = 0; qd < G / 4; ++qd) U8Layout<SPLIT>::add(p + qd * kCenters, ae[qd], ao[qd]);
+            for (int qd = 0; qd < G / 4; ++qd) {
+                if (SPLIT) {
+                    const uint2 v = lds_u64(p + qd * kCenters * E);
+                    ae[qd] += v.x;
+                    ao[qd] += v.y;
+                } else {
+                    const uint32_t v = lds_u32(p + qd * kCenters * E);
+                    ae[qd] += v & 0x00FF00FFu;
+                    ao[qd] += __byte_perm(v, 0u, 0x4341);
+                }
+            }
         }
     }
 }
@@ -1344,8 +1383,11 @@ __device__ __forceinline__ void u8_flush(uint32_t (&sums)[G], uint32_t (&ae)[G /
 // fp32 4; uint8 2 (each quad's bytes spread into 16-bit lanes) or 1.
 __host__ __device__ __forceinline__ int scan_entry_bytes(int mode, bool split) { return mode == 0 ? 4 : (split ? 2 : 1); }
 // uint8 tables use the split layout when a group of 8 queries' tables stays
-// within 64 KB that way
-__host__ __device__ __forceinline__ bool u8_split(int B) { return B * kCenters * 2 * kGroupU8 <= 64 * 1024; }
+// within AH_U8_SPLIT_BYTES that way
+#ifndef AH_U8_SPLIT_BYTES
+#define AH_U8_SPLIT_BYTES (64 * 1024)
+#endif
+__host__ __device__ __forceinline__ bool u8_split(int B) { return B * kCenters * 2 * kGroupU8 <= AH_U8_SPLIT_BYTES; }
 
 struct TileJob {
     int t0, t1;          // code tiles [t0, t1) of one leaf
@@ -1399,10 +1441,11 @@ template <int G, int NT, bool SPLIT>
 __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const SearchBuffers& b, const unsigned char* smem,
                                               const TileJob& job, const int* s_q, const uint32_t* s_th,
                                               const uint32_t* s_tl) {
-    constexpr int BS = (G / 4) * kCenters;
+    // bytes of one word's 8 blocks of entries (a multiple of 256)
+    constexpr uint32_t WB = 8u * (G / 4) * kCenters * static_cast<uint32_t>(sizeof(typename U8Layout<SPLIT>::Entry));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int W = ix.W, V = ix.V, Wf = ix.B >> 3, tail = ix.B & 7;
-    const auto* lutw = reinterpret_cast<const typename U8Layout<SPLIT>::Entry*>(smem);
+    const uint32_t tbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     for (int t = job.t0 + warp; t < job.t1; t += NT / 32) {
         const int slot = job.slot_base + 32 * t + lane;
         const bool valid = slot < job.send;
@@ -1420,16 +1463,17 @@ __device__ __forceinline__ void scan_tiles_u8(const DeviceIndex& ix, const Searc
             for (; w + 4 <= wend; w += 4) {
                 uint32_t c0, c1, c2, c3;
                 code_words4(tw, lane, w, V, c0, c1, c2, c3);
-                u8_nibbles<G, SPLIT>(c0, 8, lutw + (8 * w + 0) * BS, ae, ao);
-                u8_nibbles<G, SPLIT>(c1, 8, lutw + (8 * w + 8) * BS, ae, ao);
-                u8_nibbles<G, SPLIT>(c2, 8, lutw + (8 * w + 16) * BS, ae, ao);
-                u8_nibbles<G, SPLIT>(c3, 8, lutw + (8 * w + 24) * BS, ae, ao);
+                const uint32_t xw = tbase + w * WB;
+                u8_nibbles<G, SPLIT>(c0, 8, xw, ae, ao);
+                u8_nibbles<G, SPLIT>(c1, 8, xw + WB, ae, ao);
+                u8_nibbles<G, SPLIT>(c2, 8, xw + 2 * WB, ae, ao);
+                u8_nibbles<G, SPLIT>(c3, 8, xw + 3 * WB, ae, ao);
             }
-            for (; w < wend; ++w) u8_nibbles<G, SPLIT>(tw[code_word(w, lane, V)], 8, lutw + 8 * w * BS, ae, ao);
+            for (; w < wend; ++w) u8_nibbles<G, SPLIT>(tw[code_word(w, lane, V)], 8, tbase + w * WB, ae, ao);
             u8_flush<G>(sums, ae, ao);
         }
         if (tail) {
-            u8_nibbles<G, SPLIT>(tw[code_word(Wf, lane, V)], tail, lutw + 8 * Wf * BS, ae, ao);
+            u8_nibbles<G, SPLIT>(tw[code_word(Wf, lane, V)], tail, tbase + Wf * WB, ae, ao);
             u8_flush<G>(sums, ae, ao);
         }
 #pragma unroll
@@ -1542,7 +1586,12 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
     const int B = ix.B;
     const int total_items = b.item_off[ix.nl];
     const size_t lut_bytes = static_cast<size_t>(B) * GMAX * kCenters * scan_entry_bytes(MODE, SPLIT);
-    int* s_item_off = reinterpret_cast<int*>(smem + lut_bytes);
+    // uint8 tables start 256-byte aligned in the shared window (u8_nibbles
+    // builds entry addresses by replacing an address's low byte); the launch
+    // adds 256 bytes for this
+    unsigned char* tsm = smem;
+    if (MODE == 1) tsm += (256u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 255u)) & 255u;
+    int* s_item_off = reinterpret_cast<int*>(tsm + lut_bytes);
     const bool off_in_smem = a.scan_item_off_smem != 0;
     if (off_in_smem)
         for (int i = threadIdx.x; i <= ix.nl; i += NT) s_item_off[i] = b.item_off[i];
@@ -1606,7 +1655,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
                 for (int r = threadIdx.x; r < per_q; r += NT) lf[r] = make_float2(src[r], src[r]);
             } else {
                 const uint8_t* src = b.lut_u8 + static_cast<int64_t>(q0) * per_q;
-                for (int r = threadIdx.x; r < per_q; r += NT) smem[r] = src[r];
+                for (int r = threadIdx.x; r < per_q; r += NT) tsm[r] = src[r];
             }
         } else if (MODE == 0) {
             // one 8-byte store per (block, center) of each query pair
@@ -1624,7 +1673,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
             }
         } else {
             // one store per (block, center) of each query quad
-            auto* lw = reinterpret_cast<typename U8Layout<SPLIT>::Entry*>(smem);
+            auto* lw = reinterpret_cast<typename U8Layout<SPLIT>::Entry*>(tsm);
             const int quads = G / 4;
             for (int qd = 0; qd < quads; ++qd) {
                 const uint8_t* src[4];
@@ -1646,7 +1695,7 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
         __syncthreads();
         if (G == 1) {
             if (MODE == 0) scan_tiles_f32_single<NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off);
-            else scan_tiles_u8_single<NT>(ix, b, smem, job, s_q, s_th, s_tl);
+            else scan_tiles_u8_single<NT>(ix, b, tsm, job, s_q, s_th, s_tl);
         } else if (MODE == 0) {
             switch (G) {
                 case 8: scan_tiles_f32<8, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
@@ -1655,8 +1704,8 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
                 default: scan_tiles_f32<2, NT, RES>(ix, b, smem, job, s_q, s_th, s_tl, s_off); break;
             }
         } else {
-            if (GMAX >= 8 && G == 8) scan_tiles_u8<(GMAX >= 8 ? 8 : 4), NT, SPLIT>(ix, b, smem, job, s_q, s_th, s_tl);
-            else scan_tiles_u8<4, NT, SPLIT>(ix, b, smem, job, s_q, s_th, s_tl);
+            if (GMAX >= 8 && G == 8) scan_tiles_u8<(GMAX >= 8 ? 8 : 4), NT, SPLIT>(ix, b, tsm, job, s_q, s_th, s_tl);
+            else scan_tiles_u8<4, NT, SPLIT>(ix, b, tsm, job, s_q, s_th, s_tl);
         }
     }
 }
@@ -1697,13 +1746,13 @@ int scan_group(const DeviceIndex& ix, int lut_mode) {
 size_t scan_table_bytes(const DeviceIndex& ix, int lut_mode) {
     int nt, g;
     scan_shape(ix, lut_mode, &nt, &g);
-    return static_cast<size_t>(ix.B) * g * kCenters * scan_entry_bytes(lut_mode, u8_split(ix.B));
+    return static_cast<size_t>(ix.B) * g * kCenters * scan_entry_bytes(lut_mode, u8_split(ix.B)) + (lut_mode == 1 ? 256 : 0);
 }
 
 template <int MODE, int NT, int GMAX, bool RES, bool SPLIT = false>
 static cudaError_t launch_scan_t(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int num_sms,
                                  cudaStream_t s) {
-    size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * scan_entry_bytes(MODE, SPLIT);
+    size_t smem = static_cast<size_t>(ix.B) * GMAX * kCenters * scan_entry_bytes(MODE, SPLIT) + (MODE == 1 ? 256 : 0);
     const size_t off_bytes = static_cast<size_t>(ix.nl + 1) * sizeof(int);
     const size_t room = (NT == 512) ? 110 * 1024 : 200 * 1024;
     a.scan_item_off_smem = (smem + off_bytes <= room && off_bytes <= 64 * 1024) ? 1 : 0;
@@ -1737,6 +1786,219 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
     if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
     if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
     return launch_scan_t<1, 1024, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
+}
+
+// ---------------------------------------------------------------------------
+// the code scan (query-major, for batches whose queries seldom share a leaf)
+// ---------------------------------------------------------------------------
+
+// The leaf-major scan forms groups per leaf; when queries seldom share a leaf
+// nearly every group is a lone query whose table is staged again for every
+// item.  Here CTA (q, part) takes an even share of query q's code tiles over
+// its leaf ranks [r0, r1): the table is staged once, each leaf rank's tile
+// count, first tile, slot range and (residual codes) centroid score are held
+// in shared memory, and each warp scans two tiles at a time so that two
+// tiles' code loads are in flight together.  The sums run over blocks in
+// order, as in every other kernel that scores a slot.
+// The table starts 256-byte aligned in the shared window with a block's 16
+// entries 64 bytes apart (fp32) or 32 bytes apart (uint8: 16 bytes and 16 of
+// padding), so a code word's 8 blocks span a multiple of 256 bytes and each
+// lookup's address is one byte permute of the word's address.
+
+__host__ __device__ __forceinline__ size_t qscan_table_bytes(int mode, int B) {
+    return 256 + static_cast<size_t>(B) * (mode == 0 ? kCenters * 4 : 32);
+}
+
+size_t scan_query_smem_bytes(int mode, int B, int leaves) {
+    return qscan_table_bytes(mode, B) + sizeof(int32_t) * (5 * static_cast<size_t>(leaves) + 1);
+}
+
+template <int MODE, bool RES>
+__global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b,
+                                                                   int r0, int r1, int parts) {
+    chain_entry();
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_q[1];
+    __shared__ uint32_t s_th[1], s_tl[1];
+    constexpr int NW = kQScanThreads / 32;
+    const int q = blockIdx.x / parts, part = blockIdx.x - q * parts;
+    const int nL = r1 - r0;
+    const int B = ix.B, per_q = B * kCenters;
+    unsigned char* tsm = smem + ((256u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem)) & 255u)) & 255u);
+    const uint32_t tbase = static_cast<uint32_t>(__cvta_generic_to_shared(tsm));
+    int* s_pre = reinterpret_cast<int*>(smem + qscan_table_bytes(MODE, B));   // [nL + 1] tiles before rank i
+    int* s_pt = s_pre + nL + 1;                                               // first tile of the rank's leaf
+    int* s_os = s_pt + nL;                                                    // its first slot
+    int* s_oe = s_os + nL;                                                    // one past its last slot
+    float* s_lo = reinterpret_cast<float*>(s_oe + nL);                        // the query's score of the leaf
+    if (MODE == 0) {
+        float* lf = reinterpret_cast<float*>(tsm);
+        const float* src = b.lut_f32 + static_cast<int64_t>(q) * per_q;
+        for (int r = threadIdx.x; r < per_q; r += kQScanThreads) lf[r] = src[r];
+    } else {
+        const uint8_t* src = b.lut_u8 + static_cast<int64_t>(q) * per_q;
+        for (int r = threadIdx.x; r < per_q; r += kQScanThreads) tsm[(r >> 4) * 32 + (r & 15)] = src[r];
+    }
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int carry = 0;
+        for (int i0 = 0; i0 < nL; i0 += 32) {
+            const int i = i0 + lane;
+            int cnt = 0;
+            if (i < nL) {
+                const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + r0 + i];
+                const int pt = ix.ptile[leaf];
+                cnt = ix.ptile[leaf + 1] - pt;
+                s_pt[i] = pt;
+                s_os[i] = ix.offs[leaf];
+                s_oe[i] = ix.offs[leaf + 1];
+                if (RES) s_lo[i] = b.cscore[static_cast<int64_t>(q) * ix.nl + leaf];
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            if (i < nL) s_pre[i + 1] = carry + incl;
+            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            s_pre[0] = 0;
+            s_q[0] = q;
+            const uint64_t t = b.tau[q];
+            s_th[0] = static_cast<uint32_t>(t >> 32);
+            s_tl[0] = static_cast<uint32_t>(t);
+        }
+    }
+    __syncthreads();
+    const int total = s_pre[nL];
+    const int t_begin = static_cast<int>(static_cast<int64_t>(total) * part / parts);
+    const int t_end = static_cast<int>(static_cast<int64_t>(total) * (part + 1) / parts);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = ix.W, V = ix.V, Wf = B >> 3, tail = B & 7;
+    int ci = 0;                                    // leaf rank of the warp's tile (its tiles only increase)
+    for (int tt = t_begin + warp; tt < t_end; tt += 2 * NW) {
+        const int tu = tt + NW;
+        const bool two = tu < t_end;               // the same for the whole warp
+        while (s_pre[ci + 1] <= tt) ++ci;
+        int cj = ci;
+        if (two)
+            while (s_pre[cj + 1] <= tu) ++cj;
+        const int l0 = tt - s_pre[ci], l1 = (two ? tu : tt) - s_pre[cj];
+        const uint32_t* tw0 = ix.codes_il + static_cast<int64_t>(s_pt[ci] + l0) * W * 32;
+        const uint32_t* tw1 = ix.codes_il + static_cast<int64_t>(s_pt[cj] + l1) * W * 32;
+        const int slot0 = s_os[ci] + 32 * l0 + lane, slot1 = s_os[cj] + 32 * l1 + lane;
+        const bool v0 = slot0 < s_oe[ci], v1 = two && slot1 < s_oe[cj];
+        uint32_t k0, k1;
+        if (MODE == 0) {
+            constexpr uint32_t WB = 8 * kCenters * 4;      // bytes of a word's 8 blocks
+            auto word = [&](uint32_t c, int nb, uint32_t xw, float& acc) {
+                const uint32_t ev = (c & 0x0F0F0F0Fu) << 2, od = ((c >> 4) & 0x0F0F0F0Fu) << 2;
+#pragma unroll
+                for (int nib = 0; nib < 8; ++nib)
+                    if (nib < nb) {
+                        const uint32_t p = __byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * kCenters * 4;
+                        acc = __fadd_rn(acc, __uint_as_float(lds_u32(p)));
+                    }
+            };
+            float a0 = 0.0f, a1 = 0.0f;
+            int w = 0;
+            for (; w + 4 <= Wf; w += 4) {
+                uint32_t c0, c1, c2, c3, d0, d1, d2, d3;
+                code_words4(tw0, lane, w, V, c0, c1, c2, c3);
+                code_words4(tw1, lane, w, V, d0, d1, d2, d3);
+                const uint32_t xw = tbase + w * WB;
+                word(c0, 8, xw, a0);
+                word(d0, 8, xw, a1);
+                word(c1, 8, xw + WB, a0);
+                word(d1, 8, xw + WB, a1);
+                word(c2, 8, xw + 2 * WB, a0);
+                word(d2, 8, xw + 2 * WB, a1);
+                word(c3, 8, xw + 3 * WB, a0);
+                word(d3, 8, xw + 3 * WB, a1);
+            }
+            for (; w < Wf; ++w) {
+                const uint32_t c = tw0[code_word(w, lane, V)], d = tw1[code_word(w, lane, V)];
+                word(c, 8, tbase + w * WB, a0);
+                word(d, 8, tbase + w * WB, a1);
+            }
+            if (tail) {
+                const uint32_t c = tw0[code_word(Wf, lane, V)], d = tw1[code_word(Wf, lane, V)];
+                word(c, tail, tbase + Wf * WB, a0);
+                word(d, tail, tbase + Wf * WB, a1);
+            }
+            k0 = float_key(RES ? __fadd_rn(a0, s_lo[ci]) : a0);
+            k1 = float_key(RES ? __fadd_rn(a1, s_lo[cj]) : a1);
+        } else {
+            constexpr uint32_t WB = 8 * 32;                // bytes of a word's 8 blocks
+            auto word = [&](uint32_t c, int nb, uint32_t xw, uint32_t& acc) {
+                const uint32_t ev = c & 0x0F0F0F0Fu, od = (c >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                for (int nib = 0; nib < 8; ++nib)
+                    if (nib < nb) acc += lds_u8(__byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * 32);
+            };
+            uint32_t a0 = 0u, a1 = 0u;
+            int w = 0;
+            for (; w + 4 <= Wf; w += 4) {
+                uint32_t c0, c1, c2, c3, d0, d1, d2, d3;
+                code_words4(tw0, lane, w, V, c0, c1, c2, c3);
+                code_words4(tw1, lane, w, V, d0, d1, d2, d3);
+                const uint32_t xw = tbase + w * WB;
+                word(c0, 8, xw, a0);
+                word(d0, 8, xw, a1);
+                word(c1, 8, xw + WB, a0);
+                word(d1, 8, xw + WB, a1);
+                word(c2, 8, xw + 2 * WB, a0);
+                word(d2, 8, xw + 2 * WB, a1);
+                word(c3, 8, xw + 3 * WB, a0);
+                word(d3, 8, xw + 3 * WB, a1);
+            }
+            for (; w < Wf; ++w) {
+                const uint32_t c = tw0[code_word(w, lane, V)], d = tw1[code_word(w, lane, V)];
+                word(c, 8, tbase + w * WB, a0);
+                word(d, 8, tbase + w * WB, a1);
+            }
+            if (tail) {
+                const uint32_t c = tw0[code_word(Wf, lane, V)], d = tw1[code_word(Wf, lane, V)];
+                word(c, tail, tbase + Wf * WB, a0);
+                word(d, tail, tbase + Wf * WB, a1);
+            }
+            k0 = a0;
+            k1 = a1;
+        }
+        keep_if_reaches(v0, k0, slot0, 0, s_q, s_th, s_tl, ix, b);
+        if (two) keep_if_reaches(v1, k1, slot1, 0, s_q, s_th, s_tl, ix, b);
+        ci = cj;
+    }
+}
+
+cudaError_t launch_scan_query(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
+                              int num_sms, cudaStream_t s) {
+    const int nL = r1 - r0;
+    if (nL < 1 || nL > kQScanMaxLeaves) return cudaErrorInvalidValue;
+    const size_t smem = scan_query_smem_bytes(a.lut_mode, ix.B, nL);
+    // CTAs per query: enough to fill the SMs, no more than about two tiles per warp
+    // of the query's expected tiles (from the average leaf)
+    const double avg_tiles = std::max(1.0, static_cast<double>(ix.n) / ix.nl / 32.0);
+    const int max_parts = std::max(1, static_cast<int>(nL * avg_tiles / (2.0 * kQScanThreads / 32)));
+    auto go = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem, true);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQScanThreads, smem)) != cudaSuccess)
+            return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        const int want = (num_sms * per_sm + a.nq - 1) / a.nq;
+        const int parts = std::max(1, std::min(want, max_parts));
+        if (const cudaError_t le = launch_chained(kernel, dim3(static_cast<unsigned>(a.nq) * parts), dim3(kQScanThreads),
+                                                  smem, s, ix, a, b, r0, r1, parts);
+            le != cudaSuccess)
+            return le;
+        return cudaGetLastError();
+    };
+    if (a.lut_mode == 0) return ix.residual ? go(scan_query_kernel<0, true>) : go(scan_query_kernel<0, false>);
+    return go(scan_query_kernel<1, false>);
 }
 
 // ---------------------------------------------------------------------------
@@ -2043,8 +2305,16 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
         }
         return;
     }
-    // exact reorder: groups of `lpc` lanes, one candidate per group per round
-    for (int t = threadIdx.x; t < d; t += kFinishThreads) qv[t] = a.queries[static_cast<int64_t>(q) * d + t];
+    // exact reorder: groups of `lpc` lanes, one candidate per group per round.
+    // For 8-value bfloat16 loads the query is staged as two halves, values
+    // 8c..8c+3 at 4c and 8c+4..8c+7 at d/2 + 4c, so that the lanes' 16-byte
+    // reads of their chunks are consecutive (no bank conflicts).
+    const bool split_q = ix.reorder_bf16 && a.reorder_vec4 == 2;
+    for (int t = threadIdx.x; t < d; t += kFinishThreads) {
+        const int c = t >> 3, r = t & 7;
+        const int dst = !split_q ? t : (r < 4 ? 4 * c + r : (d >> 1) + 4 * c + (r - 4));
+        qv[dst] = a.queries[static_cast<int64_t>(q) * d + t];
+    }
     __syncthreads();
     const int lpc = a.reorder_lanes;                  // power of two in [2, 32]
     const int groups = kFinishThreads / lpc;
@@ -2075,7 +2345,7 @@ __device__ void finish_query(const DeviceIndex& ix, const SearchArgs& a, const S
                         for (int u = 0; u < kReorderBatch; ++u) {
                             const int t = t0 + u * lpc;
                             if (t < n8) {
-                                const float4 x0 = q4[2 * t], x1 = q4[2 * t + 1];
+                                const float4 x0 = q4[t], x1 = q4[n8 + t];
                                 acc = fmaf(x0.x, __uint_as_float(h[u].x << 16), acc);
                                 acc = fmaf(x0.y, __uint_as_float(h[u].x & 0xFFFF0000u), acc);
                                 acc = fmaf(x0.z, __uint_as_float(h[u].y << 16), acc);

@@ -13,7 +13,7 @@ constexpr int kGroupF32 = 8;
 constexpr int kGroupU8 = 8;
 constexpr int kScanThreads = 256;
 #ifndef AH_SAMPLE_MULT
-#define AH_SAMPLE_MULT 4
+#define AH_SAMPLE_MULT 2
 #endif
 constexpr int kSampleMult = AH_SAMPLE_MULT;       // the threshold sample holds at least this many times R slots
 constexpr int kMaxThresholdSample = 4096;   // slots scored per query for the threshold
@@ -121,6 +121,14 @@ cudaError_t launch_tau_update(const DeviceIndex& ix, const SearchArgs& a, const 
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s);
 cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int num_sms, cudaStream_t s);
+// Query-major scan of leaf ranks [r0, r1) of every query (r1 - r0 at most
+// kQScanMaxLeaves), for batches whose queries seldom share a leaf: no leaf
+// inversion needed.
+constexpr int kQScanThreads = 256;
+constexpr int kQScanMaxLeaves = 1024;
+size_t scan_query_smem_bytes(int mode, int B, int leaves);
+cudaError_t launch_scan_query(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, int r0, int r1,
+                              int num_sms, cudaStream_t s);
 // best R, exact reorder, best k.  round 0: all queries; rounds 1..2: the
 // redo list of the previous round
 cudaError_t launch_finish(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, int round, int num_sms,

@@ -438,6 +438,7 @@ class Index:
     OPT_THRESHOLD_LEAVES = 3
     OPT_PROGRESSIVE_LEAVES = 4
     OPT_UINT8_TENSOR_CORES = 5
+    OPT_QUERY_MAJOR_SCAN = 6
 
     def set_option(self, option: int, value: int):
         """Tuning knob (ah_set_option): results are unchanged, only speed."""

@@ -83,11 +83,14 @@ def Index():
 
 
 def compare(Index, name, k, L, reorder_num, lut_mode, max_leaf_mismatch=0.02, max_cand_mismatch=0.05,
-            qsel=None):
+            qsel=None, options=()):
     """Search the case's queries (or the rows ``qsel`` of them) as one batch and
-    check every query stage by stage against the oracle (parity.compare_search)."""
+    check every query stage by stage against the oracle (parity.compare_search).
+    ``options``: (option, value) pairs set on the index first."""
     w, X, Q, ix, arr = _workload(name)
     index = Index(ix)
+    for opt, val in options:
+        index.set_option(opt, val)
     Qs = Q if qsel is None else Q[qsel]
     r = compare_search(index, arr, Qs, k, L, reorder_num, lut_mode, max_leaf_mismatch=max_leaf_mismatch,
                        max_cand_mismatch=max_cand_mismatch, label=name)
@@ -380,6 +383,38 @@ def test_search_refuses_a_device_other_than_the_index_device(Index):
         assert st == 1
         torch.cuda.synchronize(1)
         assert torch.cuda.mem_get_info(1)[0] == free0
+    index.close()
+
+
+QUERY_MAJOR_CASES = [("glove-mini", 24, 0, slice(0, 8), 0), ("glove-mini", 24, 1, slice(0, 8), 0),
+                     ("glove-mini", 24, 0, None, 3), ("glove-mini-residual", 24, 0, slice(0, 8), 0),
+                     ("openai-mini", 10, 0, slice(0, 5), 0), ("openai-mini", 10, 1, None, 2),
+                     ("sweep-mini", 64, 0, slice(0, 3), 0), ("tiny", 1, 0, None, 0)]
+
+
+@pytest.mark.parametrize("name,L,lut_mode,qsel,first", QUERY_MAJOR_CASES)
+def test_query_major_scan(Index, name, L, lut_mode, qsel, first):
+    # the query-major scan (CTAs split each query's tiles; chosen on its own
+    # when queries seldom share a leaf) forced on: every query checked stage
+    # by stage against the oracle, and the same candidates, sums and results
+    # as the leaf-major scan forced on.  `first` > 0: scan phases over leaf
+    # ranks [0, first), [first, 8 first), ..., so later phases start past rank 0
+    prog = [(Index.OPT_PROGRESSIVE_LEAVES, first)] if first else []
+    compare(Index, name, 10, L, 100, lut_mode, qsel=qsel, options=[(Index.OPT_QUERY_MAJOR_SCAN, 1)] + prog)
+    w, X, Q, ix, arr = _workload(name)
+    index = Index(ix)
+    for opt, val in prog:
+        index.set_option(opt, val)
+    qg = torch.from_numpy(Q if qsel is None else Q[qsel]).cuda()
+    out = {}
+    for opt in (1, -1):
+        index.set_option(Index.OPT_QUERY_MAJOR_SCAN, opt)
+        out[opt] = index.search(qg, 10, L, 100, lut_mode, trace=True)
+        index.sync_status()
+    for x, y in zip(out[1][:2], out[-1][:2]):
+        torch.testing.assert_close(x, y, rtol=0, atol=0)
+    for key in ("cand_ids", "cand_sums", "ncand", "scanned"):
+        torch.testing.assert_close(out[1][2][key], out[-1][2][key], rtol=0, atol=0)
     index.close()
 
 
