@@ -144,7 +144,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     add(sizeof(float) * (size_t)cnq);                           // 7 bias
     add(sizeof(uint64_t) * (size_t)cnq);                        // 8 tau
     add(sizeof(uint64_t) * (size_t)cnq * cap);                  // 9 candidate keys
-    add(sizeof(int32_t) * (size_t)(2 * NL + cnq + 8));          // 10 zero region: qcount, qcursor, count, counters
+    add(sizeof(int32_t) * (size_t)(2 * NL + 2 * cnq + 8));      // 10 zero region: qcount, qcursor, count, counters, tdone
     add(sizeof(int32_t) * (size_t)2 * cnq);                     // 11 redo
     add(sizeof(int32_t) * (size_t)(NL + 1));                    // 12 qoff
     add(sizeof(int32_t) * (size_t)(NL + 1));                    // 13 item_off
@@ -200,6 +200,7 @@ ah_status carve(ah_index* ix, int nq, int L, int R, int lut_mode, int k, bool ho
     b.qcursor = zr + NL;
     b.count = zr + 2 * NL;
     b.counters = zr + 2 * NL + cnq;
+    b.tdone = zr + 2 * NL + cnq + 8;
     b.redo = reinterpret_cast<int32_t*>(part[11]);
     b.qoff = reinterpret_cast<int32_t*>(part[12]);
     b.item_off = reinterpret_cast<int32_t*>(part[13]);
@@ -273,17 +274,20 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
     // uint8 tables: the int8 tensor-core scan only when asked for (on the
     // benchmarked batches it ran 1.1-2.9x slower than the table lookups)
     a.scan_tc = (lut_mode == AH_LUT_U8 && ix->opt_u8_tensor == 1) ? 1 : 0;
-    // code tiles per scan item: up to 128, fewer (multiples of 8, one tile per
+    // code tiles per scan item: up to 128 (each item stages its group's
+    // tables, so long items stage less), fewer (multiples of 8, one tile per
     // warp of a 256-thread CTA) when the batch's tiles, estimated from the
-    // average leaf, would leave scan CTAs (about 6 per SM) without an item
+    // average leaf, would give scan CTAs (about 6 per SM) fewer than about 32
+    // items each, which leaves a ragged end on small batches
     {
         const double est_tiles = static_cast<double>(nq) * L * std::max(1.0, static_cast<double>(ix->dix.n) / ix->dix.nl / 32.0);
         const double ctas = static_cast<double>(ix->num_sms) * 6;
-        const int c = 8 * static_cast<int>(std::ceil(est_tiles / ctas / 8.0));
+        const int c = 8 * static_cast<int>(std::ceil(est_tiles / ctas / 32.0 / 8.0));
         a.chunk = ix->opt_chunk_tiles > 0 ? ix->opt_chunk_tiles : std::min(128, std::max(8, c));
         if (a.scan_tc) a.chunk = ah::scan_tc_chunk_tiles();
     }
     a.threshold_sample = ix->opt_threshold_sample;
+    a.threshold_parts = 1;
     a.threshold_leaves = ix->opt_threshold_leaves;
     a.out_ids = out_ids;
     a.out_scores = out_scores;
@@ -313,7 +317,7 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
             cudaEventRecord(ix->ev[ix->n_marks++], s);
         }
     };
-    e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)(2 * dix.nl + ix->ws.nq + 8), s);
+    e = cudaMemsetAsync(b.qcount, 0, sizeof(int32_t) * (size_t)(2 * dix.nl + 2 * ix->ws.nq + 8), s);
     if (e != cudaSuccess) return cuda_fail(e, "memset");
     // With per-stage profiling everything runs in order on s (clean stage
     // times); otherwise the tables and the inversion run on the side stream,
@@ -359,6 +363,11 @@ ah_status run_search(ah_index* ix, const float* queries, int32_t nq, int32_t k, 
                                           static_cast<int>(std::min<double>(ah::kMaxThresholdSample, std::ceil(need))));
         }
         const int M = ah::threshold_sample(a.R, a.threshold_sample);
+        // batches too small to give every SM a query: several CTAs per query
+        // score the sample (256 points or more each; the last to finish
+        // selects the bound)
+        if (nq < ix->num_sms)
+            a.threshold_parts = std::max(1, std::min((2 * ix->num_sms + nq - 1) / nq, M / 256));
         int first = L;
         if (ix->opt_progressive_leaves > 0) first = std::min(L, ix->opt_progressive_leaves);
         else if (ix->opt_progressive_leaves == 0 && !small && expect(M) > b.cap / 8)

@@ -1041,7 +1041,10 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 
 constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
 
-// One CTA per query.  Scores a sample of M = min(points, threshold_sample)
+// One CTA per query, or `threshold_parts` CTAs per query for batches too
+// small to fill the GPU: each scores an even share of the sample into the
+// query's candidate buffer (unused until the scan) and the last to finish
+// copies all the keys to its shared memory and selects.  Scores a sample of M = min(points, threshold_sample)
 // slots of the query's best leaves (an even share of the S best, topped up in
 // rank order); the R-th largest (score, id) key among them
 // is a lower bound on the R-th largest over all its leaves (a subset's R-th
@@ -1055,8 +1058,9 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
     __shared__ RegSelectScratch<kSelThreads> rs;
     __shared__ int seg_end[kThresholdSegs], seg_pos[kThresholdSegs], seg_slot[kThresholdSegs];
     __shared__ float seg_off[kThresholdSegs];       // residual codes: the leaf's centroid score
-    __shared__ int s_nseg, s_taken;
-    const int q = blockIdx.x;
+    __shared__ int s_nseg, s_taken, s_last;
+    const int parts = a.threshold_parts;
+    const int q = blockIdx.x / parts, part = blockIdx.x - q * parts;
     const int R = a.R;
     // the table starts 256-byte aligned in the shared window (slot_values4's
     // byte-permute addressing); the launch adds 256 bytes for this
@@ -1146,7 +1150,12 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
     }
     __syncthreads();
     const int nseg = s_nseg, taken = s_taken;
-    for (int t0 = 0; t0 < taken; t0 += 4 * kSelThreads) {
+    // this CTA's share of the sample; with several CTAs per query the keys
+    // go to the query's candidate buffer (unused until the scan)
+    const int i_begin = static_cast<int>(static_cast<int64_t>(taken) * part / parts);
+    const int i_end = static_cast<int>(static_cast<int64_t>(taken) * (part + 1) / parts);
+    uint64_t* gk = b.ckey + static_cast<int64_t>(q) * b.cap;
+    for (int t0 = i_begin; t0 < i_end; t0 += 4 * kSelThreads) {
         int32_t ps[4], sid[4];
         bool ok[4];
         uint32_t v[4];
@@ -1154,7 +1163,7 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = t0 + u * kSelThreads + threadIdx.x;
-            ok[u] = i < taken;
+            ok[u] = i < i_end;
             int lo = 0, hi = nseg - 1;                 // first segment whose end is above i
             while (lo < hi) {
                 const int mid = (lo + hi) >> 1;
@@ -1169,8 +1178,22 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = t0 + u * kSelThreads + threadIdx.x;
-            if (ok[u]) vals[i] = make_key(v[u], sid[u]);
+            if (ok[u]) {
+                const uint64_t key = make_key(v[u], sid[u]);
+                if (parts == 1) vals[i] = key;
+                else gk[i] = key;
+            }
         }
+    }
+    if (parts > 1) {
+        // the query's last CTA to finish selects from all parts' keys
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) s_last = atomicAdd(&b.tdone[q], 1) == parts - 1;
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        for (int i = threadIdx.x; i < taken; i += kSelThreads) vals[i] = __ldcg(gk + i);
     }
     __syncthreads();
     if (taken <= 4 * kSelThreads) {
@@ -1212,11 +1235,11 @@ cudaError_t launch_threshold(const DeviceIndex& ix, const SearchArgs& a, const S
     if (a.lut_mode == 0) {
         e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<0>), smem, true);
         if (e != cudaSuccess) return e;
-        if (const cudaError_t le = launch_chained(threshold_kernel<0>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
+        if (const cudaError_t le = launch_chained(threshold_kernel<0>, dim3(a.nq * a.threshold_parts), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
     } else {
         e = ensure_smem(reinterpret_cast<const void*>(threshold_kernel<1>), smem, true);
         if (e != cudaSuccess) return e;
-        if (const cudaError_t le = launch_chained(threshold_kernel<1>, dim3(a.nq), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
+        if (const cudaError_t le = launch_chained(threshold_kernel<1>, dim3(a.nq * a.threshold_parts), dim3(kSelThreads), smem, s, ix, a, b); le != cudaSuccess) return le;
     }
     return cudaGetLastError();
 }
@@ -1346,20 +1369,35 @@ __device__ __forceinline__ void u8_nibbles(uint32_t c, int nb, uint32_t xw, uint
     // byte offsets of the word's entries: nibbles 0, 2, 4, 6 in the bytes of
     // ev, 1, 3, 5, 7 in those of od
     const uint32_t ev = (c & 0x0F0F0F0Fu) << SH, od = ((c >> 4) & 0x0F0F0F0Fu) << SH;
+    if (SPLIT) {
 #pragma unroll
-    for (int nib = 0; nib < 8; ++nib) {
-        if (nib < nb) {
-            const uint32_t p = __byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * BSB;
+        for (int nib = 0; nib < 8; ++nib) {
+            if (nib < nb) {
+                const uint32_t p = __byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * BSB;
 #pragma unroll
-            for (int qd = 0; qd < G / 4; ++qd) {
-                if (SPLIT) {
+                for (int qd = 0; qd < G / 4; ++qd) {
                     const uint2 v = lds_u64(p + qd * kCenters * E);
                     ae[qd] += v.x;
                     ao[qd] += v.y;
-                } else {
-                    const uint32_t v = lds_u32(p + qd * kCenters * E);
-                    ae[qd] += v & 0x00FF00FFu;
-                    ao[qd] += __byte_perm(v, 0u, 0x4341);
+                }
+            }
+        }
+    } else {
+        // packed words: nibbles in pairs, so each 16-bit-lane accumulator
+        // takes both nibbles' halves in one three-input add (the integer
+        // pipe, at half the issue rate, bounds this loop)
+#pragma unroll
+        for (int n2 = 0; n2 < 8; n2 += 2) {
+            if (n2 < nb) {
+                const bool second = n2 + 1 < nb;
+                const uint32_t p0 = __byte_perm(ev, xw, 0x7650u | (n2 >> 1)) + n2 * BSB;
+                const uint32_t p1 = __byte_perm(od, xw, 0x7650u | (n2 >> 1)) + (n2 + 1) * BSB;
+#pragma unroll
+                for (int qd = 0; qd < G / 4; ++qd) {
+                    const uint32_t v0 = lds_u32(p0 + qd * kCenters * E);
+                    const uint32_t v1 = second ? lds_u32(p1 + qd * kCenters * E) : 0u;
+                    ae[qd] += (v0 & 0x00FF00FFu) + (v1 & 0x00FF00FFu);
+                    ao[qd] += __byte_perm(v0, 0u, 0x4341) + __byte_perm(v1, 0u, 0x4341);
                 }
             }
         }
@@ -1839,11 +1877,15 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
         const uint8_t* src = b.lut_u8 + static_cast<int64_t>(q) * per_q;
         for (int r = threadIdx.x; r < per_q; r += kQScanThreads) tsm[(r >> 4) * 32 + (r & 15)] = src[r];
     }
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
+    // tile counts per leaf rank, and their prefix sums: every thread takes
+    // ranks tid, tid + 256, ... (one round of loads for up to 256 ranks), then
+    // warp scans and one pass over the warp totals per round
+    __shared__ int s_wsum[kQScanThreads / 32];
+    {
+        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
         int carry = 0;
-        for (int i0 = 0; i0 < nL; i0 += 32) {
-            const int i = i0 + lane;
+        for (int i0 = 0; i0 < nL; i0 += kQScanThreads) {
+            const int i = i0 + threadIdx.x;
             int cnt = 0;
             if (i < nL) {
                 const int leaf = b.leaves[static_cast<int64_t>(q) * a.L + r0 + i];
@@ -1860,10 +1902,20 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
                 const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
                 if (lane >= off) incl += v;
             }
-            if (i < nL) s_pre[i + 1] = carry + incl;
-            carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            if (lane == 31) s_wsum[wid] = incl;
+            __syncthreads();
+            int before = carry, all = 0;
+#pragma unroll
+            for (int w2 = 0; w2 < kQScanThreads / 32; ++w2) {
+                const int ws = s_wsum[w2];
+                before += (w2 < wid) ? ws : 0;
+                all += ws;
+            }
+            if (i < nL) s_pre[i + 1] = before + incl;
+            carry += all;
+            __syncthreads();                   // s_wsum is rewritten next round
         }
-        if (lane == 0) {
+        if (threadIdx.x == 0) {
             s_pre[0] = 0;
             s_q[0] = q;
             const uint64_t t = b.tau[q];

@@ -61,6 +61,7 @@ struct SearchBuffers {
     uint64_t* ckey;         // [nq][cap] kept candidates: (score key, id) keys
     int32_t* cslot;         // [nq][cap] and their slots
     int32_t* count;         // [nq]          (zeroed per search)
+    int32_t* tdone;         // [nq]          (zeroed per search) threshold CTAs of the query done
     int32_t* redo;          // [2][nq]       queries to rescan after rounds 0 and 1
     int32_t* order;         // [nq]          finish order: queries with many kept candidates first
     int32_t* counters;      // [8]           (zeroed per search): 0 scan work (first phase), 1..2 redo
@@ -106,6 +107,7 @@ struct SearchArgs {
     int topl_stride;            // split top-L: keys per query in topl_tmp
     int scan_tc;                // uint8 tables: scan on the int8 tensor cores (items of up to 128
                                 // queries x 256 points) instead of table lookups
+    int threshold_parts;        // CTAs per query scoring the threshold sample (1: one CTA does all)
 };
 
 // Build-time: the leaf-padded tiled code copy; V = code_vector_words(W).
