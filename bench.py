@@ -38,10 +38,10 @@ L2_BYTES = 126 * 1024 * 1024
 SM_COUNT = 148
 SMEM_BYTES_PER_CLK = 128          # per SM: 32 banks x 4 B
 SM_MAX_MHZ_FALLBACK = 1965.0
-# DRAM bytes (read + write) that one ncu capture counted for one scan launch, per
-# (workload, table mode) at the workload's default batch; None where no capture
-# of the current scan kernel exists.
-SCAN_TRAFFIC_BYTES = {("glove", 0): 35.75e6}
+# DRAM bytes (read + write) that one ncu capture counted for the scan launches of
+# one step (all scan phases), per (workload, table mode) at the workload's default
+# batch; None where no capture of the current scan kernel exists.
+SCAN_TRAFFIC_BYTES = {("openai", 0): 8.43e9}   # the three phase launches of one step, one ncu pass
 
 
 def parse():

@@ -594,7 +594,159 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_seg_kernel(DeviceIndex
     for (int i = threadIdx.x; i < K; i += kSelThreads) out[i] = keys[i];
 }
 
+// One CTA of 1,024 threads per query with the score row in registers (up to
+// 16 keys per thread: 16,384 centroids), L <= 256: the L-th largest (score,
+// id) key by 8-bit digits from the highest bit where the row's keys differ
+// (a 256-bin shared histogram of the current bucket per digit, one warp
+// picking the digit), stopping once the keys above the bucket plus the
+// bucket itself are exactly L.  The L keys are gathered and each is placed by
+// its rank (the number of selected keys above it; keys are unique).
+constexpr int kTopRadixThreads = 1024;
+constexpr int kTopRadixKPL = 16;
+constexpr int kTopRadixMaxL = 256;
+
+__global__ void __launch_bounds__(kTopRadixThreads) top_leaves_radix_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
+    chain_entry();
+    __shared__ int hist[256];
+    __shared__ uint64_t s_and[kTopRadixThreads / 32], s_or[kTopRadixThreads / 32];
+    __shared__ uint64_t sel[kTopRadixMaxL];
+    __shared__ int s_digit, s_above, s_in, s_count;
+    __shared__ long long s_scanned;
+    const int q = blockIdx.x;
+    const int L = a.L, nl = ix.nl;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float* row = b.cscore + static_cast<int64_t>(q) * nl;
+    uint64_t k[kTopRadixKPL];
+    uint64_t kand = ~0ull, kor = 0ull;
+#pragma unroll
+    for (int j = 0; j < kTopRadixKPL; ++j) {
+        const int i = threadIdx.x + kTopRadixThreads * j;
+        k[j] = (i < nl) ? make_key(float_key(row[i]), i) : 0ull;
+        if (i < nl) kand &= k[j];
+        kor |= k[j];
+    }
+    kand = warp_and64(kand);
+    kor = warp_or64(kor);
+    if (lane == 0) {
+        s_and[warp] = kand;
+        s_or[warp] = kor;
+    }
+    if (threadIdx.x == 0) {
+        s_count = 0;
+        s_scanned = 0;
+    }
+    __syncthreads();
+    kand = ~0ull;
+    kor = 0ull;
+#pragma unroll
+    for (int w = 0; w < kTopRadixThreads / 32; ++w) {
+        kand &= s_and[w];
+        kor |= s_or[w];
+    }
+    // the selected keys are those with (key & mask) >= prefix (and real)
+    uint64_t prefix = 0ull, mask = 0ull;
+    const uint64_t diff = kand ^ kor;
+    if (L < nl && diff != 0ull) {
+        const int top = 63 - __clzll(diff);
+        mask = (top >= 63) ? 0ull : (~0ull << (top + 1));
+        prefix = kand & mask;
+        int lo = top + 1, need = L;
+        for (;;) {
+            const int wd = lo < 8 ? lo : 8;
+            const int sh = lo - wd;
+            const uint64_t dmask = (1ull << wd) - 1ull;
+            if (threadIdx.x < 256) hist[threadIdx.x] = 0;
+            __syncthreads();
+            // one atomic per distinct digit of a warp's keys (scores share
+            // their high bits, so a digit often covers much of a warp)
+#pragma unroll
+            for (int j = 0; j < kTopRadixKPL; ++j) {
+                const bool in = k[j] != 0ull && (k[j] & mask) == prefix;
+                const unsigned dg = static_cast<unsigned>((k[j] >> sh) & dmask);
+                const unsigned peers = __match_any_sync(0xFFFFFFFFu, in ? dg : (0x100u | lane));
+                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane l holds digits 255 - 8 l down to 248 - 8 l
+                int c[8], tot = 0;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    c[u] = hist[255 - 8 * lane - u];
+                    tot += c[u];
+                }
+                int incl = tot;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const unsigned m = __ballot_sync(0xFFFFFFFFu, incl >= need);
+                if (lane == __ffs(m) - 1) {
+                    int run = incl - tot;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (run + c[u] >= need) {
+                            s_digit = 255 - 8 * lane - u;
+                            s_above = run;
+                            s_in = c[u];
+                            break;
+                        }
+                        run += c[u];
+                    }
+                }
+            }
+            __syncthreads();
+            need -= s_above;
+            prefix |= static_cast<uint64_t>(s_digit) << sh;
+            mask |= dmask << sh;
+            lo = sh;
+            // keys are unique, so by the last bit the bucket is one key
+            if (s_in == need || lo == 0) break;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kTopRadixKPL; ++j) {
+        const bool take = k[j] != 0ull && (k[j] & mask) >= prefix;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
+        if (m) {
+            int base = 0;
+            if (lane == __ffs(m) - 1) base = atomicAdd(&s_count, __popc(m));
+            base = __shfl_sync(0xFFFFFFFFu, base, __ffs(m) - 1);
+            if (take) sel[base + __popc(m & ((1u << lane) - 1u))] = k[j];
+        }
+    }
+    __syncthreads();
+    const int n = s_count;                          // min(L, nl)
+    long long local = 0;
+    if (threadIdx.x < n) {
+        const uint64_t key = sel[threadIdx.x];
+        int r = 0;
+        for (int t = 0; t < n; ++t) r += (sel[t] > key) ? 1 : 0;
+        const int leaf = key_id(key);
+        b.leaves[static_cast<int64_t>(q) * L + r] = leaf;
+        b.leaf_scores[static_cast<int64_t>(q) * L + r] = key_float(key_score(key));
+        if (r < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);
+        local = ix.offs[leaf + 1] - ix.offs[leaf];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, off);
+    if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
+    __syncthreads();
+    if (threadIdx.x == 0) b.scanned[q] = s_scanned;
+}
+
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
+    // the radix form: rows above 4,096 centroids (up to 16,384) at any batch,
+    // and smaller rows with L > 32 for batches too small to fill the SMs with
+    // the warp and register forms' one-warp or one-CTA queries
+    if (ix.nl <= kTopRadixThreads * kTopRadixKPL && a.L <= kTopRadixMaxL &&
+        (ix.nl > 16 * kSelThreads || (a.nq <= 256 && a.L > 32 && ix.nl > 64))) {
+        if (const cudaError_t le = launch_chained(top_leaves_radix_kernel, dim3(a.nq), dim3(kTopRadixThreads), 0, s, ix, a, b);
+            le != cudaSuccess)
+            return le;
+        return cudaGetLastError();
+    }
     if (b.topl_tmp && ix.nl > 16 * kSelThreads && a.nq <= kTopSplitMaxQ && a.L <= kTopSplitMaxL) {
         // split form: segments of at most 1,024 scores in parallel, then one
         // CTA per query merges the survivors (at most 16 x 256 keys)
@@ -1820,7 +1972,10 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
         return launch_scan_t<0, 1024, kGroupF32, false>(ix, a, b, num_sms, s);
     }
     // uint8 tables are refused for residual codes before any launch
-    if (u8_split(ix.B)) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
+    if (u8_split(ix.B)) {
+        if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
+        return launch_scan_t<1, 512, kGroupU8 / 2, false, true>(ix, a, b, num_sms, s);
+    }
     if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
     if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
     return launch_scan_t<1, 1024, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
