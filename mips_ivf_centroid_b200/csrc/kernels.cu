@@ -21,6 +21,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 #include <mutex>
 #include <unordered_map>
 #include <utility>
@@ -594,159 +595,7 @@ __global__ void __launch_bounds__(kSelThreads) top_leaves_seg_kernel(DeviceIndex
     for (int i = threadIdx.x; i < K; i += kSelThreads) out[i] = keys[i];
 }
 
-// One CTA of 1,024 threads per query with the score row in registers (up to
-// 16 keys per thread: 16,384 centroids), L <= 256: the L-th largest (score,
-// id) key by 8-bit digits from the highest bit where the row's keys differ
-// (a 256-bin shared histogram of the current bucket per digit, one warp
-// picking the digit), stopping once the keys above the bucket plus the
-// bucket itself are exactly L.  The L keys are gathered and each is placed by
-// its rank (the number of selected keys above it; keys are unique).
-constexpr int kTopRadixThreads = 1024;
-constexpr int kTopRadixKPL = 16;
-constexpr int kTopRadixMaxL = 256;
-
-__global__ void __launch_bounds__(kTopRadixThreads) top_leaves_radix_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
-    chain_entry();
-    __shared__ int hist[256];
-    __shared__ uint64_t s_and[kTopRadixThreads / 32], s_or[kTopRadixThreads / 32];
-    __shared__ uint64_t sel[kTopRadixMaxL];
-    __shared__ int s_digit, s_above, s_in, s_count;
-    __shared__ long long s_scanned;
-    const int q = blockIdx.x;
-    const int L = a.L, nl = ix.nl;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const float* row = b.cscore + static_cast<int64_t>(q) * nl;
-    uint64_t k[kTopRadixKPL];
-    uint64_t kand = ~0ull, kor = 0ull;
-#pragma unroll
-    for (int j = 0; j < kTopRadixKPL; ++j) {
-        const int i = threadIdx.x + kTopRadixThreads * j;
-        k[j] = (i < nl) ? make_key(float_key(row[i]), i) : 0ull;
-        if (i < nl) kand &= k[j];
-        kor |= k[j];
-    }
-    kand = warp_and64(kand);
-    kor = warp_or64(kor);
-    if (lane == 0) {
-        s_and[warp] = kand;
-        s_or[warp] = kor;
-    }
-    if (threadIdx.x == 0) {
-        s_count = 0;
-        s_scanned = 0;
-    }
-    __syncthreads();
-    kand = ~0ull;
-    kor = 0ull;
-#pragma unroll
-    for (int w = 0; w < kTopRadixThreads / 32; ++w) {
-        kand &= s_and[w];
-        kor |= s_or[w];
-    }
-    // the selected keys are those with (key & mask) >= prefix (and real)
-    uint64_t prefix = 0ull, mask = 0ull;
-    const uint64_t diff = kand ^ kor;
-    if (L < nl && diff != 0ull) {
-        const int top = 63 - __clzll(diff);
-        mask = (top >= 63) ? 0ull : (~0ull << (top + 1));
-        prefix = kand & mask;
-        int lo = top + 1, need = L;
-        for (;;) {
-            const int wd = lo < 8 ? lo : 8;
-            const int sh = lo - wd;
-            const uint64_t dmask = (1ull << wd) - 1ull;
-            if (threadIdx.x < 256) hist[threadIdx.x] = 0;
-            __syncthreads();
-            // one atomic per distinct digit of a warp's keys (scores share
-            // their high bits, so a digit often covers much of a warp)
-#pragma unroll
-            for (int j = 0; j < kTopRadixKPL; ++j) {
-                const bool in = k[j] != 0ull && (k[j] & mask) == prefix;
-                const unsigned dg = static_cast<unsigned>((k[j] >> sh) & dmask);
-                const unsigned peers = __match_any_sync(0xFFFFFFFFu, in ? dg : (0x100u | lane));
-                if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[dg], __popc(peers));
-            }
-            __syncthreads();
-            if (warp == 0) {
-                // lane l holds digits 255 - 8 l down to 248 - 8 l
-                int c[8], tot = 0;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    c[u] = hist[255 - 8 * lane - u];
-                    tot += c[u];
-                }
-                int incl = tot;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-                    if (lane >= off) incl += v;
-                }
-                const unsigned m = __ballot_sync(0xFFFFFFFFu, incl >= need);
-                if (lane == __ffs(m) - 1) {
-                    int run = incl - tot;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (run + c[u] >= need) {
-                            s_digit = 255 - 8 * lane - u;
-                            s_above = run;
-                            s_in = c[u];
-                            break;
-                        }
-                        run += c[u];
-                    }
-                }
-            }
-            __syncthreads();
-            need -= s_above;
-            prefix |= static_cast<uint64_t>(s_digit) << sh;
-            mask |= dmask << sh;
-            lo = sh;
-            // keys are unique, so by the last bit the bucket is one key
-            if (s_in == need || lo == 0) break;
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < kTopRadixKPL; ++j) {
-        const bool take = k[j] != 0ull && (k[j] & mask) >= prefix;
-        const unsigned m = __ballot_sync(0xFFFFFFFFu, take);
-        if (m) {
-            int base = 0;
-            if (lane == __ffs(m) - 1) base = atomicAdd(&s_count, __popc(m));
-            base = __shfl_sync(0xFFFFFFFFu, base, __ffs(m) - 1);
-            if (take) sel[base + __popc(m & ((1u << lane) - 1u))] = k[j];
-        }
-    }
-    __syncthreads();
-    const int n = s_count;                          // min(L, nl)
-    long long local = 0;
-    if (threadIdx.x < n) {
-        const uint64_t key = sel[threadIdx.x];
-        int r = 0;
-        for (int t = 0; t < n; ++t) r += (sel[t] > key) ? 1 : 0;
-        const int leaf = key_id(key);
-        b.leaves[static_cast<int64_t>(q) * L + r] = leaf;
-        b.leaf_scores[static_cast<int64_t>(q) * L + r] = key_float(key_score(key));
-        if (r < a.count_ranks) atomicAdd(&b.qcount[leaf], 1);
-        local = ix.offs[leaf + 1] - ix.offs[leaf];
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(0xFFFFFFFFu, local, off);
-    if (lane == 0 && local) atomicAdd(reinterpret_cast<unsigned long long*>(&s_scanned), static_cast<unsigned long long>(local));
-    __syncthreads();
-    if (threadIdx.x == 0) b.scanned[q] = s_scanned;
-}
-
 cudaError_t launch_top_leaves(const DeviceIndex& ix, SearchArgs a, const SearchBuffers& b, cudaStream_t s) {
-    // the radix form: rows above 4,096 centroids (up to 16,384) at any batch,
-    // and smaller rows with L > 32 for batches too small to fill the SMs with
-    // the warp and register forms' one-warp or one-CTA queries
-    if (ix.nl <= kTopRadixThreads * kTopRadixKPL && a.L <= kTopRadixMaxL &&
-        (ix.nl > 16 * kSelThreads || (a.nq <= 256 && a.L > 32 && ix.nl > 64))) {
-        if (const cudaError_t le = launch_chained(top_leaves_radix_kernel, dim3(a.nq), dim3(kTopRadixThreads), 0, s, ix, a, b);
-            le != cudaSuccess)
-            return le;
-        return cudaGetLastError();
-    }
     if (b.topl_tmp && ix.nl > 16 * kSelThreads && a.nq <= kTopSplitMaxQ && a.L <= kTopSplitMaxL) {
         // split form: segments of at most 1,024 scores in parallel, then one
         // CTA per query merges the survivors (at most 16 x 256 keys)
@@ -934,16 +783,15 @@ __device__ __forceinline__ float lut_entry(const float* __restrict__ q, const fl
     return v;
 }
 
+// grid (queries, entries / 256): thread r of query blockIdx.x writes entry r
 __global__ void lut_f32_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b) {
     chain_entry();
-    int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int per_q = ix.B * kCenters;
-    if (e >= static_cast<int64_t>(a.nq) * per_q) return;
-    int q = static_cast<int>(e / per_q);
-    int r = static_cast<int>(e - static_cast<int64_t>(q) * per_q);
-    int blk = r >> 4;
-    b.lut_f32[e] = lut_entry(a.queries + static_cast<int64_t>(q) * ix.d + blk * ix.dpb,
-                             ix.codebook + static_cast<int64_t>(r) * ix.dpb, ix.dpb);
+    const int q = blockIdx.x;
+    const int r = blockIdx.y * blockDim.x + threadIdx.x;
+    if (r >= per_q) return;
+    b.lut_f32[static_cast<int64_t>(q) * per_q + r] =
+        lut_entry(a.queries + static_cast<int64_t>(q) * ix.d + (r >> 4) * ix.dpb, ix.codebook + r * ix.dpb, ix.dpb);
 }
 
 // One CTA per query: the uint8 table, delta and bias, all in fp32 with
@@ -989,8 +837,8 @@ __global__ void __launch_bounds__(256) lut_u8_kernel(DeviceIndex ix, SearchArgs 
 
 cudaError_t launch_lut(const DeviceIndex& ix, const SearchArgs& a, const SearchBuffers& b, cudaStream_t s) {
     if (a.lut_mode == 0) {
-        int64_t total = static_cast<int64_t>(a.nq) * ix.B * kCenters;
-        if (const cudaError_t le = launch_chained(lut_f32_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, s, ix, a, b); le != cudaSuccess) return le;
+        const unsigned per_q = static_cast<unsigned>(ix.B) * kCenters;
+        if (const cudaError_t le = launch_chained(lut_f32_kernel, dim3(static_cast<unsigned>(a.nq), (per_q + 255) / 256), dim3(256), 0, s, ix, a, b); le != cudaSuccess) return le;
     } else {
         size_t smem = (static_cast<size_t>(ix.B) * kCenters + ix.B) * sizeof(float);
         cudaError_t e = ensure_smem(reinterpret_cast<const void*>(lut_u8_kernel), smem, true);
@@ -1972,10 +1820,7 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
         return launch_scan_t<0, 1024, kGroupF32, false>(ix, a, b, num_sms, s);
     }
     // uint8 tables are refused for residual codes before any launch
-    if (u8_split(ix.B)) {
-        if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
-        return launch_scan_t<1, 512, kGroupU8 / 2, false, true>(ix, a, b, num_sms, s);
-    }
+    if (u8_split(ix.B)) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
     if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
     if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
     return launch_scan_t<1, 1024, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
@@ -2006,7 +1851,9 @@ size_t scan_query_smem_bytes(int mode, int B, int leaves) {
     return qscan_table_bytes(mode, B) + sizeof(int32_t) * (5 * static_cast<size_t>(leaves) + 1);
 }
 
-template <int MODE, bool RES>
+// VW: the code copy's words per vector load (ix.V), fixed per instantiation so
+// the per-word index arithmetic folds (each word feeds only 8 lookups here).
+template <int MODE, bool RES, int VW>
 __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex ix, SearchArgs a, SearchBuffers b,
                                                                    int r0, int r1, int parts) {
     chain_entry();
@@ -2083,21 +1930,26 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
     const int t_begin = static_cast<int>(static_cast<int64_t>(total) * part / parts);
     const int t_end = static_cast<int>(static_cast<int64_t>(total) * (part + 1) / parts);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = ix.W, V = ix.V, Wf = B >> 3, tail = B & 7;
-    int ci = 0;                                    // leaf rank of the warp's tile (its tiles only increase)
-    for (int tt = t_begin + warp; tt < t_end; tt += 2 * NW) {
-        const int tu = tt + NW;
-        const bool two = tu < t_end;               // the same for the whole warp
-        while (s_pre[ci + 1] <= tt) ++ci;
-        int cj = ci;
-        if (two)
-            while (s_pre[cj + 1] <= tu) ++cj;
-        const int l0 = tt - s_pre[ci], l1 = (two ? tu : tt) - s_pre[cj];
-        const uint32_t* tw0 = ix.codes_il + static_cast<int64_t>(s_pt[ci] + l0) * W * 32;
-        const uint32_t* tw1 = ix.codes_il + static_cast<int64_t>(s_pt[cj] + l1) * W * 32;
-        const int slot0 = s_os[ci] + 32 * l0 + lane, slot1 = s_os[cj] + 32 * l1 + lane;
-        const bool v0 = slot0 < s_oe[ci], v1 = two && slot1 < s_oe[cj];
-        uint32_t k0, k1;
+    constexpr int V = VW;
+    const int W = ix.W, Wf = B >> 3, tail = B & 7;
+    int ci = 0;                                    // leaf rank of the warp's latest tile (tiles only increase)
+    // U tiles at a time (U = 2 while two remain), their code loads issued together
+    auto run = [&](auto u_tag, int tt) {
+        constexpr int U = decltype(u_tag)::value;
+        int cr[U], slot[U];
+        bool valid[U];
+        const uint32_t* tw[U];
+        uint32_t key[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int t = tt + u * NW;
+            while (s_pre[ci + 1] <= t) ++ci;
+            cr[u] = ci;
+            const int l = t - s_pre[ci];
+            tw[u] = ix.codes_il + static_cast<int64_t>(s_pt[ci] + l) * W * 32;
+            slot[u] = s_os[ci] + 32 * l + lane;
+            valid[u] = slot[u] < s_oe[ci];
+        }
         if (MODE == 0) {
             constexpr uint32_t WB = 8 * kCenters * 4;      // bytes of a word's 8 blocks
             auto word = [&](uint32_t c, int nb, uint32_t xw, float& acc) {
@@ -2109,34 +1961,36 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
                         acc = __fadd_rn(acc, __uint_as_float(lds_u32(p)));
                     }
             };
-            float a0 = 0.0f, a1 = 0.0f;
+            float acc[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) acc[u] = 0.0f;
             int w = 0;
             for (; w + 4 <= Wf; w += 4) {
-                uint32_t c0, c1, c2, c3, d0, d1, d2, d3;
-                code_words4(tw0, lane, w, V, c0, c1, c2, c3);
-                code_words4(tw1, lane, w, V, d0, d1, d2, d3);
+                uint32_t cw[U][4];
+#pragma unroll
+                for (int u = 0; u < U; ++u) code_words4(tw[u], lane, w, V, cw[u][0], cw[u][1], cw[u][2], cw[u][3]);
                 const uint32_t xw = tbase + w * WB;
-                word(c0, 8, xw, a0);
-                word(d0, 8, xw, a1);
-                word(c1, 8, xw + WB, a0);
-                word(d1, 8, xw + WB, a1);
-                word(c2, 8, xw + 2 * WB, a0);
-                word(d2, 8, xw + 2 * WB, a1);
-                word(c3, 8, xw + 3 * WB, a0);
-                word(d3, 8, xw + 3 * WB, a1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) word(cw[u][k], 8, xw + k * WB, acc[u]);
             }
             for (; w < Wf; ++w) {
-                const uint32_t c = tw0[code_word(w, lane, V)], d = tw1[code_word(w, lane, V)];
-                word(c, 8, tbase + w * WB, a0);
-                word(d, 8, tbase + w * WB, a1);
+                uint32_t cw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(w, lane, V)];
+#pragma unroll
+                for (int u = 0; u < U; ++u) word(cw[u], 8, tbase + w * WB, acc[u]);
             }
             if (tail) {
-                const uint32_t c = tw0[code_word(Wf, lane, V)], d = tw1[code_word(Wf, lane, V)];
-                word(c, tail, tbase + Wf * WB, a0);
-                word(d, tail, tbase + Wf * WB, a1);
+                uint32_t cw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(Wf, lane, V)];
+#pragma unroll
+                for (int u = 0; u < U; ++u) word(cw[u], tail, tbase + Wf * WB, acc[u]);
             }
-            k0 = float_key(RES ? __fadd_rn(a0, s_lo[ci]) : a0);
-            k1 = float_key(RES ? __fadd_rn(a1, s_lo[cj]) : a1);
+#pragma unroll
+            for (int u = 0; u < U; ++u) key[u] = float_key(RES ? __fadd_rn(acc[u], s_lo[cr[u]]) : acc[u]);
         } else {
             constexpr uint32_t WB = 8 * 32;                // bytes of a word's 8 blocks
             auto word = [&](uint32_t c, int nb, uint32_t xw, uint32_t& acc) {
@@ -2145,38 +1999,43 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
                 for (int nib = 0; nib < 8; ++nib)
                     if (nib < nb) acc += lds_u8(__byte_perm((nib & 1) ? od : ev, xw, 0x7650u | (nib >> 1)) + nib * 32);
             };
-            uint32_t a0 = 0u, a1 = 0u;
+            uint32_t acc[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) acc[u] = 0u;
             int w = 0;
             for (; w + 4 <= Wf; w += 4) {
-                uint32_t c0, c1, c2, c3, d0, d1, d2, d3;
-                code_words4(tw0, lane, w, V, c0, c1, c2, c3);
-                code_words4(tw1, lane, w, V, d0, d1, d2, d3);
+                uint32_t cw[U][4];
+#pragma unroll
+                for (int u = 0; u < U; ++u) code_words4(tw[u], lane, w, V, cw[u][0], cw[u][1], cw[u][2], cw[u][3]);
                 const uint32_t xw = tbase + w * WB;
-                word(c0, 8, xw, a0);
-                word(d0, 8, xw, a1);
-                word(c1, 8, xw + WB, a0);
-                word(d1, 8, xw + WB, a1);
-                word(c2, 8, xw + 2 * WB, a0);
-                word(d2, 8, xw + 2 * WB, a1);
-                word(c3, 8, xw + 3 * WB, a0);
-                word(d3, 8, xw + 3 * WB, a1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) word(cw[u][k], 8, xw + k * WB, acc[u]);
             }
             for (; w < Wf; ++w) {
-                const uint32_t c = tw0[code_word(w, lane, V)], d = tw1[code_word(w, lane, V)];
-                word(c, 8, tbase + w * WB, a0);
-                word(d, 8, tbase + w * WB, a1);
+                uint32_t cw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(w, lane, V)];
+#pragma unroll
+                for (int u = 0; u < U; ++u) word(cw[u], 8, tbase + w * WB, acc[u]);
             }
             if (tail) {
-                const uint32_t c = tw0[code_word(Wf, lane, V)], d = tw1[code_word(Wf, lane, V)];
-                word(c, tail, tbase + Wf * WB, a0);
-                word(d, tail, tbase + Wf * WB, a1);
+                uint32_t cw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(Wf, lane, V)];
+#pragma unroll
+                for (int u = 0; u < U; ++u) word(cw[u], tail, tbase + Wf * WB, acc[u]);
             }
-            k0 = a0;
-            k1 = a1;
+#pragma unroll
+            for (int u = 0; u < U; ++u) key[u] = acc[u];
         }
-        keep_if_reaches(v0, k0, slot0, 0, s_q, s_th, s_tl, ix, b);
-        if (two) keep_if_reaches(v1, k1, slot1, 0, s_q, s_th, s_tl, ix, b);
-        ci = cj;
+#pragma unroll
+        for (int u = 0; u < U; ++u) keep_if_reaches(valid[u], key[u], slot[u], 0, s_q, s_th, s_tl, ix, b);
+    };
+    for (int tt = t_begin + warp; tt < t_end; tt += 2 * NW) {
+        if (tt + NW < t_end) run(std::integral_constant<int, 2>{}, tt);   // the same for the whole warp
+        else run(std::integral_constant<int, 1>{}, tt);
     }
 }
 
@@ -2204,8 +2063,13 @@ cudaError_t launch_scan_query(const DeviceIndex& ix, const SearchArgs& a, const 
             return le;
         return cudaGetLastError();
     };
-    if (a.lut_mode == 0) return ix.residual ? go(scan_query_kernel<0, true>) : go(scan_query_kernel<0, false>);
-    return go(scan_query_kernel<1, false>);
+    auto by_v = [&](auto k4, auto k2, auto k1) { return ix.V == 4 ? go(k4) : ix.V == 2 ? go(k2) : go(k1); };
+    if (a.lut_mode == 0) {
+        if (ix.residual)
+            return by_v(scan_query_kernel<0, true, 4>, scan_query_kernel<0, true, 2>, scan_query_kernel<0, true, 1>);
+        return by_v(scan_query_kernel<0, false, 4>, scan_query_kernel<0, false, 2>, scan_query_kernel<0, false, 1>);
+    }
+    return by_v(scan_query_kernel<1, false, 4>, scan_query_kernel<1, false, 2>, scan_query_kernel<1, false, 1>);
 }
 
 // ---------------------------------------------------------------------------
