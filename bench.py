@@ -50,7 +50,8 @@ def parse():
     p.add_argument("--steps", type=int, default=400)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="openai")
+    p.add_argument("--workload", default=None,
+                   help="openai (the default), glove, bigann, tiny, sweep; --encode and --kmeans default to glove")
     p.add_argument("--lut-mode", type=int, default=0, choices=[0, 1])
     p.add_argument("--nq", type=int, default=None)
     p.add_argument("--leaves", type=int, default=None, help="num_leaves_to_search")
@@ -70,7 +71,12 @@ def parse():
                         "candidates are gathered and merged exactly (strong scaling)")
     p.add_argument("--kmeans", action="store_true",
                    help="index build: time one k-means iteration (assignment + update) over the workload's points")
-    return p.parse_args()
+    args = p.parse_args()
+    if args.workload is None:
+        args.workload = "glove" if (args.encode or args.kmeans) else "openai"
+    if (args.encode or args.kmeans) and "--steps" not in sys.argv:
+        args.steps = 20                                  # the index-build lines time whole passes over n points
+    return args
 
 
 def cpu_model() -> str:
