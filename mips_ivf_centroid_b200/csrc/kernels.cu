@@ -1425,7 +1425,18 @@ __host__ __device__ __forceinline__ int scan_entry_bytes(int mode, bool split) {
 #ifndef AH_U8_SPLIT_BYTES
 #define AH_U8_SPLIT_BYTES (64 * 1024)
 #endif
-__host__ __device__ __forceinline__ bool u8_split(int B) { return B * kCenters * 2 * kGroupU8 <= AH_U8_SPLIT_BYTES; }
+// uint8 tables of up to 100 KB per group of 8 (256 < B <= 400) in the split
+// layout too, as two 512-thread CTAs per SM with groups kept at 8 (the
+// OpenAI-shaped uint8 step: 15.14 ms against 15.61 ms with packed words)
+#ifndef AH_U8_WIDE_SPLIT
+#define AH_U8_WIDE_SPLIT 1
+#endif
+__host__ __device__ __forceinline__ bool u8_wide_split(int B) {
+    return AH_U8_WIDE_SPLIT && B * kCenters * 2 * kGroupU8 > AH_U8_SPLIT_BYTES && B * kCenters * 2 * kGroupU8 <= 100 * 1024;
+}
+__host__ __device__ __forceinline__ bool u8_split(int B) {
+    return B * kCenters * 2 * kGroupU8 <= AH_U8_SPLIT_BYTES || u8_wide_split(B);
+}
 
 struct TileJob {
     int t0, t1;          // code tiles [t0, t1) of one leaf
@@ -1761,7 +1772,10 @@ __global__ void __launch_bounds__(NT, (NT == 256 ? (MODE == 0 ? AH_SCAN_MIN_BLOC
 void scan_shape(const DeviceIndex& ix, int lut_mode, int* nt, int* gmax) {
     const int g = lut_mode == 0 ? kGroupF32 : kGroupU8;
     const size_t table = static_cast<size_t>(ix.B) * kCenters * scan_entry_bytes(lut_mode, u8_split(ix.B)) * g;
-    if (table <= 64 * 1024) {
+    if (lut_mode == 1 && u8_wide_split(ix.B)) {
+        *nt = 512;
+        *gmax = g;
+    } else if (table <= 64 * 1024) {
         *nt = 256;
         *gmax = g;
     } else if (AH_WIDE_SPLIT && table / 2 <= 100 * 1024) {
@@ -1820,7 +1834,10 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
         return launch_scan_t<0, 1024, kGroupF32, false>(ix, a, b, num_sms, s);
     }
     // uint8 tables are refused for residual codes before any launch
-    if (u8_split(ix.B)) return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
+    if (u8_split(ix.B)) {
+        if (nt == 512) return launch_scan_t<1, 512, kGroupU8, false, true>(ix, a, b, num_sms, s);
+        return launch_scan_t<1, 256, kGroupU8, false, true>(ix, a, b, num_sms, s);
+    }
     if (nt == 256) return launch_scan_t<1, 256, kGroupU8, false>(ix, a, b, num_sms, s);
     if (nt == 512) return launch_scan_t<1, 512, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
     return launch_scan_t<1, 1024, kGroupU8 / 2, false>(ix, a, b, num_sms, s);
