@@ -1868,6 +1868,29 @@ size_t scan_query_smem_bytes(int mode, int B, int leaves) {
     return qscan_table_bytes(mode, B) + sizeof(int32_t) * (5 * static_cast<size_t>(leaves) + 1);
 }
 
+// All W <= 8 code words of one lane's slot in a tile, V words per load (V
+// divides W), zero past W: one round of loads for the whole tile.
+template <int V>
+__device__ __forceinline__ void tile_words8(const uint32_t* __restrict__ tw, int lane, int W, uint32_t (&cw)[8]) {
+#pragma unroll
+    for (int w = 0; w < 8; w += V) {
+        if (w < W) {
+            if (V == 4) {
+                const uint4 v = *reinterpret_cast<const uint4*>(tw + w * 32 + lane * 4);
+                cw[w] = v.x; cw[w + 1] = v.y; cw[w + 2] = v.z; cw[w + 3] = v.w;
+            } else if (V == 2) {
+                const uint2 v = *reinterpret_cast<const uint2*>(tw + w * 32 + lane * 2);
+                cw[w] = v.x; cw[w + 1] = v.y;
+            } else {
+                cw[w] = tw[w * 32 + lane];
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < V; ++j) cw[w + j] = 0u;
+        }
+    }
+}
+
 // VW: the code copy's words per vector load (ix.V), fixed per instantiation so
 // the per-word index arithmetic folds (each word feeds only 8 lookups here).
 template <int MODE, bool RES, int VW>
@@ -1981,6 +2004,26 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
             float acc[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) acc[u] = 0.0f;
+            if (W <= 8) {
+                // narrow codes (up to 64 blocks): both tiles' words in one round of loads
+                uint32_t cw[U][8];
+#pragma unroll
+                for (int u = 0; u < U; ++u) tile_words8<V>(tw[u], lane, W, cw[u]);
+#pragma unroll
+                for (int w8 = 0; w8 < 8; ++w8)
+                    if (w8 < Wf)
+#pragma unroll
+                        for (int u = 0; u < U; ++u) word(cw[u][w8], 8, tbase + w8 * WB, acc[u]);
+                if (tail) {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        uint32_t last = 0u;
+#pragma unroll
+                        for (int w8 = 0; w8 < 8; ++w8) last = (w8 == Wf) ? cw[u][w8] : last;
+                        word(last, tail, tbase + Wf * WB, acc[u]);
+                    }
+                }
+            } else {
             int w = 0;
             for (; w + 4 <= Wf; w += 4) {
                 uint32_t cw[U][4];
@@ -2005,6 +2048,7 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
                 for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(Wf, lane, V)];
 #pragma unroll
                 for (int u = 0; u < U; ++u) word(cw[u], tail, tbase + Wf * WB, acc[u]);
+            }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) key[u] = float_key(RES ? __fadd_rn(acc[u], s_lo[cr[u]]) : acc[u]);
@@ -2019,6 +2063,26 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
             uint32_t acc[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) acc[u] = 0u;
+            if (W <= 8) {
+                // narrow codes (up to 64 blocks): both tiles' words in one round of loads
+                uint32_t cw[U][8];
+#pragma unroll
+                for (int u = 0; u < U; ++u) tile_words8<V>(tw[u], lane, W, cw[u]);
+#pragma unroll
+                for (int w8 = 0; w8 < 8; ++w8)
+                    if (w8 < Wf)
+#pragma unroll
+                        for (int u = 0; u < U; ++u) word(cw[u][w8], 8, tbase + w8 * WB, acc[u]);
+                if (tail) {
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        uint32_t last = 0u;
+#pragma unroll
+                        for (int w8 = 0; w8 < 8; ++w8) last = (w8 == Wf) ? cw[u][w8] : last;
+                        word(last, tail, tbase + Wf * WB, acc[u]);
+                    }
+                }
+            } else {
             int w = 0;
             for (; w + 4 <= Wf; w += 4) {
                 uint32_t cw[U][4];
@@ -2043,6 +2107,7 @@ __global__ void __launch_bounds__(kQScanThreads) scan_query_kernel(DeviceIndex i
                 for (int u = 0; u < U; ++u) cw[u] = tw[u][code_word(Wf, lane, V)];
 #pragma unroll
                 for (int u = 0; u < U; ++u) word(cw[u], tail, tbase + Wf * WB, acc[u]);
+            }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) key[u] = acc[u];
