@@ -1040,6 +1040,9 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 
 
 constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
+#ifndef AH_THR_REG16
+#define AH_THR_REG16 0
+#endif
 
 // One CTA per query, or `threshold_parts` CTAs per query for batches too
 // small to fill the GPU: each scores an even share of the sample into the
@@ -1218,6 +1221,18 @@ __global__ void __launch_bounds__(kSelThreads, 5) threshold_kernel(DeviceIndex i
                 kk[j] = (i < taken) ? vals[i] : 0ull;
             }
             tau = block_kth_reg<8, kSelThreads>(kk, taken, R, rs);
+        }
+        if (threadIdx.x == 0) b.tau[q] = tau;
+    } else if (AH_THR_REG16 && taken <= 16 * kSelThreads) {
+        uint64_t tau = 0ull;
+        if (taken >= R) {
+            uint64_t kk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = threadIdx.x + kSelThreads * j;
+                kk[j] = (i < taken) ? vals[i] : 0ull;
+            }
+            tau = block_kth_reg<16, kSelThreads>(kk, taken, R, rs);
         }
         if (threadIdx.x == 0) b.tau[q] = tau;
     } else {
