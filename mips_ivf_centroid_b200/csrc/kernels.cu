@@ -1040,8 +1040,12 @@ __host__ __device__ __forceinline__ int table_bytes(int mode, int B) {
 
 
 constexpr int kThresholdSegs = 256;      // sample segments (leaves) per query at most
+// samples above 2,048 keys (batches under 1,024 queries grow theirs up to
+// 4,096): the bound by the register-held bitwise selection, 16 keys per
+// thread, rather than the shared-memory radix (threshold stage at one query
+// and L = 256: 20.6 us against 22.8 us; 16 queries: 24.7 against 35.0 us)
 #ifndef AH_THR_REG16
-#define AH_THR_REG16 0
+#define AH_THR_REG16 1
 #endif
 
 // One CTA per query, or `threshold_parts` CTAs per query for batches too
