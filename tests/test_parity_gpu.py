@@ -351,12 +351,26 @@ def test_speed_knobs_do_not_change_results(Index, lut_mode):
     ref = index.search(qg, 10, 64, 100, lut_mode)
     for opt, val in [(Index.OPT_PROGRESSIVE_LEAVES, -1), (Index.OPT_PROGRESSIVE_LEAVES, 3),
                      (Index.OPT_THRESHOLD_SAMPLE, 64), (Index.OPT_THRESHOLD_LEAVES, 8),
-                     (Index.OPT_SCAN_CHUNK_TILES, 3)]:
+                     (Index.OPT_SCAN_CHUNK_TILES, 3), (Index.OPT_QUERY_MAJOR_SCAN, 1),
+                     (Index.OPT_QUERY_MAJOR_SCAN, -1)]:
         index.set_option(opt, val)
         got = index.search(qg, 10, 64, 100, lut_mode)
         torch.testing.assert_close(got[0], ref[0], rtol=0, atol=0)
         torch.testing.assert_close(got[1], ref[1], rtol=0, atol=0)
     index.sync_status()
+    index.close()
+
+
+def test_speed_knobs_reject_values_out_of_range(Index):
+    from mips_ivf_centroid_b200 import AhError
+    w, X, Q, ix, arr = _workload("tiny")
+    index = Index(ix)
+    for opt, val in [(Index.OPT_QUERY_MAJOR_SCAN, 2), (Index.OPT_QUERY_MAJOR_SCAN, -2),
+                     (Index.OPT_UINT8_TENSOR_CORES, 2), (Index.OPT_THRESHOLD_SAMPLE, 0),
+                     (Index.OPT_SCAN_CHUNK_TILES, 2000), (99, 0)]:
+        with pytest.raises(AhError) as e:
+            index.set_option(opt, val)
+        assert e.value.status == 1
     index.close()
 
 
