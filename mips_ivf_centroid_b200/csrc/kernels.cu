@@ -1874,8 +1874,8 @@ cudaError_t launch_scan(const DeviceIndex& ix, const SearchArgs& a, const Search
 // in shared memory, and each warp scans two tiles at a time so that two
 // tiles' code loads are in flight together.  The sums run over blocks in
 // order, as in every other kernel that scores a slot.
-// The table starts 256-byte aligned in the shared window with a block's 16
-// entries 64 bytes apart (fp32) or 32 bytes apart (uint8: 16 bytes and 16 of
+// The table starts 256-byte aligned in the shared window and a block's 16
+// entries take 64 bytes (fp32) or 32 bytes (uint8: 16 bytes and 16 of
 // padding), so a code word's 8 blocks span a multiple of 256 bytes and each
 // lookup's address is one byte permute of the word's address.
 
